@@ -1,0 +1,460 @@
+#!/usr/bin/env python
+"""Benchmark of the fused routed-expert MoE layer on B200.
+
+One step = one moe_forward (route -> permute -> grouped gate/up GEMM with
+SwiGLU -> grouped down GEMM -> weighted combine) over one batch of synthetic
+tokens, with every expert's weights resident in HBM.  Prints ONE JSON line
+(rank 0).  Default workload: the Qwen-3.5-like decode step (T=512,
+H=4096, E=512, I=1024, top-10); the prefill chunk (T=8192) with the same
+weights is measured in the same run and reported under "prefill".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own replica
+of the layer on its own batch (weak scaling, no data-path collective); the
+device time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "fused MoE layer tokens/s (T=8192 prefill, T=512 decode); % of TC/HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 256 << 20  # > 126 MB L2
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------- inputs
+def device_inputs(cfg, rank):
+    """Seeded synthetic inputs on the device: x per rank, weights shared."""
+    import torch
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+    t0 = time.time()
+    inp = synth.make_inputs(cfg.with_(seed=cfg.seed), experts=False)
+    x = inp.x if rank == 0 else synth.make_x(cfg.with_(seed=cfg.seed + rank))
+    E, H, I = cfg.E, cfg.H, cfg.I
+    wgu = torch.empty(E, H, 2 * I, dtype=torch.bfloat16, device="cuda")
+    wd = torch.empty(E, I, H, dtype=torch.bfloat16, device="cuda")
+    chunk = 32
+    for e0 in range(0, E, chunk):
+        e1 = min(E, e0 + chunk)
+        hgu = np.empty((e1 - e0, H, 2 * I), np.uint16)
+        hd = np.empty((e1 - e0, I, H), np.uint16)
+        # fill_expert_weights indexes its output by expert id; use a shifted view
+        synth.fill_expert_weights(cfg, "gate_up", _Shift(hgu, e0), experts=range(e0, e1))
+        synth.fill_expert_weights(cfg, "down", _Shift(hd, e0), experts=range(e0, e1))
+        wgu[e0:e1].copy_(torch.from_numpy(hgu.view(np.int16)).view(torch.bfloat16))
+        wd[e0:e1].copy_(torch.from_numpy(hd.view(np.int16)).view(torch.bfloat16))
+    d = dict(x=bf(x), w_router=torch.from_numpy(inp.w_router).cuda(),
+             bias=None if inp.bias is None else torch.from_numpy(inp.bias).cuda(),
+             w_gate_up=wgu, w_down=wd,
+             w_sh_gate_up=None if inp.w_sh_gate_up is None else bf(inp.w_sh_gate_up),
+             w_sh_down=None if inp.w_sh_down is None else bf(inp.w_sh_down))
+    torch.cuda.synchronize()
+    log(f"[bench] rank {rank}: inputs for {cfg.name} ready in {time.time() - t0:.1f}s")
+    return d, x
+
+
+class _Shift:
+    """Array view indexed by absolute expert id (e - e0)."""
+
+    def __init__(self, a, e0):
+        self.a, self.e0 = a, e0
+
+    def __setitem__(self, e, v):
+        self.a[e - self.e0] = v
+
+
+# ---------------------------------------------------------------- accounting
+def layer_accounting(cfg, counts):
+    """Algorithmic FLOPs and bytes of one step (activated experts only)."""
+    touched = int((counts > 0).sum())
+    H, I, T, k = cfg.H, cfg.I, cfg.T, cfg.k
+    flops = 6.0 * k * H * I * T + (6.0 * H * cfg.I_s * T if cfg.I_s else 0.0)
+    w_bytes = touched * 3 * H * I * 2 + (3 * H * cfg.I_s * 2 if cfg.I_s else 0)
+    layer_bytes = w_bytes + T * H * 2 + H * cfg.E * 4 + T * H * 2
+    gate_up_bytes = touched * H * 2 * I * 2 + T * H * 2 + T * k * I * 2
+    return dict(touched=touched, flops=flops, layer_bytes=layer_bytes, gate_up_bytes=gate_up_bytes)
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("grouped_gemm.cu", "common.cuh", "kernels.h"):
+        h.update(open(os.path.join(ROOT, "routed_expert_ffn_prefix_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per launch of the gate/up kernel from a committed ncu summary,
+    only if it was taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "gate_up_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+    except ValueError:
+        return None
+    if d.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return d.get("per_launch_bytes", {}).get(workload)
+
+
+# ---------------------------------------------------------------- timed runs
+def time_workload(cfg, d, ws, steps, warmup, rank, world, flush, moe, gpu_index, sample_clocks=True):
+    import torch
+    import torch.distributed as dist
+    T = cfg.T
+
+    def step(evs=None, info=None):
+        return moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws,
+                           d["w_sh_gate_up"], d["w_sh_down"], stage_events=evs, info=info)
+
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st = moe.device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {moe.STATUS.get(st, st)} after warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(steps)]
+    info = {}
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = ClockSampler(gpu_index) if sample_clocks else None
+    if clk:
+        clk.start()
+        time.sleep(0.3)
+    for i in range(steps):
+        flush.zero_()  # L2 flush between steps, outside the timed events
+        step(evs[i], info)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = clk.stop() if clk else None
+    step_ms = [e[0].elapsed_time(e[6]) for e in evs]
+    stage_ms = [[e[j].elapsed_time(e[j + 1]) for j in range(6)] for e in evs]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    mean_stage = [statistics.mean(s[j] for s in stage_ms) for j in range(6)]
+    return dict(total_ms=total_ms, ms_per_step=total_ms / steps, value=T * world * steps / (total_ms / 1e3),
+                stage_ms=mean_stage, launches=info.get("launches", 0) * steps, clocks=clocks,
+                step_ms_median=statistics.median(step_ms))
+
+
+def time_e2e(cfg, d, ws, steps, warmup, rank, world, moe):
+    """Same metric through the public call with host buffers: pinned x in,
+    y out, both copies inside the timed region."""
+    import torch
+    import torch.distributed as dist
+    x_h = d["x"].cpu().pin_memory()
+    y_h = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory()
+    x_d = torch.empty_like(d["x"])
+    y_d = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        x_d.copy_(x_h, non_blocking=True)
+        moe.forward(x_d, d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws, d["w_sh_gate_up"],
+                    d["w_sh_down"], out=y_d)
+        y_h.copy_(y_d, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": cfg.T * world * steps / (ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2,
+            "ms_per_step": ms / steps}
+
+
+# ---------------------------------------------------------------- CPU oracle baseline
+def oracle_sample(cfg, n_tokens, reps=1):
+    """Times the CPU oracle (as it stands) on the first n_tokens tokens of the
+    workload: fp64 router, top-k, and the k expert FFNs per token.  Expert
+    weights are drawn before the clock starts."""
+    import oracle  # test infrastructure: only this CPU-baseline leg runs it
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        cores = 1
+    inp = synth.make_inputs(cfg, experts=False)
+    toks = np.arange(min(n_tokens, cfg.T))
+    l = oracle.router_logits(inp.x[toks], inp.w_router, inp.bias)
+    ids, _ = oracle.topk_route(l, cfg.k)
+    need = sorted(set(ids.reshape(-1).tolist()))
+    wgu = {e: synth.expert_gate_up(cfg, e) for e in need}
+    wd = {e: synth.expert_down(cfg, e) for e in need}
+    times = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        lg = oracle.router_logits(inp.x[toks], inp.w_router, inp.bias)
+        ids2, w2 = oracle.topk_route(lg, cfg.k)
+        xs = inp.x[toks]
+        oracle.layer_forward_tokens(xs, np.arange(len(toks)), ids2, w2, lambda e: wgu[e], lambda e: wd[e],
+                                    inp.w_sh_gate_up, inp.w_sh_down)
+        times.append(time.perf_counter() - t0)
+    return dict(seconds=times, tokens=len(toks), cores=cores, experts=len(need))
+
+
+# ---------------------------------------------------------------- main
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import routed_expert_ffn_prefix_b200 as moe
+    from routed_expert_ffn_prefix_b200 import build as moe_build
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if rank == 0:
+        moe_build.build()
+    if world > 1:
+        dist.barrier()
+    moe.lib()
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else local
+    pk, pk_kind = peaks()
+    cfg = synth.CONFIGS[args.workload]
+    d, _ = device_inputs(cfg, rank)
+    ws = moe.alloc_workspace(cfg.T, cfg.H, cfg.E, cfg.I, cfg.k, cfg.I_s)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    main = time_workload(cfg, d, ws, args.steps, args.warmup, rank, world, flush, moe, gpu_index)
+    counts = moe.workspace_view(ws, cfg.T, cfg.H, cfg.E, cfg.I, cfg.k, cfg.I_s)["counts"].cpu().numpy()
+    acc = layer_accounting(cfg, counts)
+    e2e = time_e2e(cfg, d, ws, args.steps, args.warmup, rank, world, moe)
+
+    def roof(cfg_, res, acc_):
+        gate_up_ms = res["stage_ms"][3]
+        achieved = acc_["gate_up_bytes"] / (gate_up_ms / 1e3) / 1e9
+        t_bytes = acc_["layer_bytes"] / (pk["hbm_gbs"] * 1e9)
+        t_flops = acc_["flops"] / (pk["bf16_tflops_sustained"] * 1e12)
+        t_roof = max(t_bytes, t_flops)
+        return {
+            "roofline": {"bound": "hbm", "kernel": "grouped gate/up GEMM + SwiGLU (tcgen05)",
+                         "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": recorded_traffic(cfg_.name),
+                         "algorithmic_bytes_per_launch": acc_["gate_up_bytes"],
+                         "launch_ms": round(gate_up_ms, 4), "peak_source": pk_kind},
+            "layer_roofline": {"t_roofline_ms": round(t_roof * 1e3, 4),
+                               "binding": "hbm" if t_bytes >= t_flops else "tensor",
+                               "frac": round(t_roof * 1e3 / res["ms_per_step"], 4),
+                               "tflops": round(acc_["flops"] / (res["ms_per_step"] / 1e3) / 1e12, 1),
+                               "gbs": round(acc_["layer_bytes"] / (res["ms_per_step"] / 1e3) / 1e9, 1),
+                               "touched_experts": acc_["touched"], "peak_source": pk_kind},
+            "stage_ms": {n: round(v, 4) for n, v in zip(
+                ("route", "permute", "shared_expert", "gate_up", "down", "combine"), res["stage_ms"])},
+        }
+
+    out_main = roof(cfg, main, acc)
+    prefill = None
+    if not args.no_prefill and cfg.name == "qwen_decode_t512":
+        pcfg = synth.CONFIGS["qwen_prefill_t8192"]
+        px = synth.make_x(pcfg.with_(seed=pcfg.seed + rank))
+        d2 = dict(d)
+        d2["x"] = torch.from_numpy(px.view(np.int16)).view(torch.bfloat16).cuda()
+        ws2 = moe.alloc_workspace(pcfg.T, pcfg.H, pcfg.E, pcfg.I, pcfg.k, pcfg.I_s)
+        pres = time_workload(pcfg, d2, ws2, args.steps, args.warmup, rank, world, flush, moe, gpu_index,
+                             sample_clocks=False)
+        pcounts = moe.workspace_view(ws2, pcfg.T, pcfg.H, pcfg.E, pcfg.I, pcfg.k)["counts"].cpu().numpy()
+        pacc = layer_accounting(pcfg, pcounts)
+        pe2e = time_e2e(pcfg, d2, ws2, max(3, args.steps // 2), args.warmup, rank, world, moe)
+        prefill = {"workload": pcfg.name, "value": round(pres["value"], 1), "unit": "tokens/s",
+                   "ms_per_step": round(pres["ms_per_step"], 4), "gpu_launches": pres["launches"],
+                   "e2e": {k: (round(v, 1) if isinstance(v, float) else v) for k, v in pe2e.items()},
+                   **roof(pcfg, pres, pacc)}
+        del ws2
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        smp = oracle_sample(cfg, args.cpu_sample_tokens)
+        secs = min(smp["seconds"])
+        cpu = {"value": round(smp["tokens"] / secs, 3), "unit": "tokens/s", "cores": smp["cores"],
+               "kind": "oracle",
+               "sample": f"first {smp['tokens']} tokens of {cfg.name} (router + top-k + {cfg.k} expert FFNs "
+                         f"each, {smp['experts']} distinct experts), float64 numpy, {secs:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(main["value"], 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(main["ms_per_step"], 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) router and expert weights; no dataset)",
+            "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "I": cfg.I, "k": cfg.k,
+                       "I_s": cfg.I_s, "bias": cfg.bias, "seed": cfg.seed,
+                       "parallelism": f"replicas x{world} (no collective in the layer)",
+                       "l2": "flushed (256 MiB write) before every timed step; expert weights 12.9 GB >> L2"},
+            **out_main,
+            "e2e": {k: (round(v, 1) if isinstance(v, float) else v) for k, v in e2e.items()},
+            "gpu_launches": main["launches"],
+            "clocks": main["clocks"],
+            "cpu_baseline": cpu,
+        }
+        if prefill:
+            line["prefill"] = prefill
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The oracle on the host cores, on this arm's workload and metric, one
+    bounded sample of tokens per step."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    cfg = synth.CONFIGS[args.workload]
+    n = args.ref_sample_tokens
+    smp = oracle_sample(cfg, n, reps=args.warmup + args.steps)
+    timed = smp["seconds"][args.warmup:]
+    total = sum(timed)
+    value = smp["tokens"] * len(timed) / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total / len(timed), 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "I": cfg.I, "k": cfg.k,
+                   "I_s": cfg.I_s, "sample_tokens_per_step": smp["tokens"]},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": smp["cores"], "kind": "oracle",
+                         "sample": f"first {smp['tokens']} tokens of {cfg.name} per step, float64 numpy oracle"},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen_decode_t512", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--no-prefill", action="store_true", help="skip the T=8192 prefill measurement")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=16)
+    ap.add_argument("--ref-sample-tokens", type=int, default=2)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,218 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) routed-expert MoE FFN layer.
+ *
+ * The layer (one GPU, all experts resident):
+ *
+ *   route    l = x . W_router (+ bias), fp32; p = softmax(l) over E experts;
+ *            the k largest p per token (descending, ties to the lower id);
+ *            w_j = p_j / sum of the k selected p.
+ *   permute  slots (t, j) sorted into expert-contiguous order, experts
+ *            ascending, tokens ascending within an expert.
+ *   gate/up  per permuted row r (token t, expert e):
+ *            [g | u] = x[t] . W_gate_up[e];  h[r] = bf16(silu(g) * u).
+ *   down     o[r] = h[r] . W_down[e]  (fp32).
+ *   combine  y[t] = bf16( sum_{j=0..k-1} w[t,j] * o[inv_perm[t,j]]  (j ascending,
+ *            fp32)  + s[t] ),  s = shared-expert FFN of x[t] when present.
+ *
+ * Passages defining the steps (page title, section):
+ *   - Qwen 3.5-397B MoE on Ironwood (TPU v7x), sec. 4.2 "MoE track":
+ *     top_k = 10 routing, SparseCore ragged gather of token rows straight
+ *     from HBM (no padded permuted tensor), grouped GEMM V2 with SwiGLU
+ *     fused into the main matmul loop, minimal per-expert padding.
+ *   - same page, sec. 7.2 "chunked pipeline": un-permute and
+ *     gather-reduce of the [T*k, H] expert outputs back to token order.
+ *   - same page, sec. 8.2: router gating projection fused with top-k.
+ *   - Ling-2.6-1T on TPU v7x with SGLang-JAX, "Fused MoE V2" paragraph:
+ *     scatter + expert FFN + gather as one fused unit; top-8 routing plus
+ *     a shared expert.
+ *   - the benchmark workload definitions: softmax over router logits,
+ *     then top-k, then renormalise.
+ *
+ * Conventions for every call:
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller, row
+ *     major, densely packed.  bf16 tensors are passed as uint16_t bit
+ *     patterns.  The library never allocates, frees or keeps a pointer
+ *     past the call; work is enqueued on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream) and the call returns without waiting.
+ *   - Shapes: T >= 1 tokens, H % 256 == 0, I % 128 == 0 (I_s likewise),
+ *     1 <= k <= min(E, 64), E <= 1024, T*k < 2^31.
+ *   - Alignment: every pointer 16-byte aligned (workspace 256-byte).
+ *   - Workspace: caller-allocated device memory of at least
+ *     moe_workspace_size() bytes for the layer's shapes; every call takes
+ *     the same workspace (each stage uses its own region of it).  Calls
+ *     that share a workspace must be stream-ordered.
+ *   - Errors in the arguments are found on the host before anything is
+ *     enqueued: the call returns the status and launches nothing.
+ *     Errors found on the device (a bounds check on routing metadata, a
+ *     bounded wait that ran out) are written to a status word in the
+ *     workspace, read with moe_get_device_status(); the kernel that finds
+ *     one skips the rest of its work and exits.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,      /* null pointer, bad shape, k > E, ... */
+  MOE_ERR_ALIGNMENT = 2,        /* pointer or shape not aligned as required */
+  MOE_ERR_WORKSPACE = 3,        /* workspace missing or too small */
+  MOE_ERR_CUDA = 4,             /* a CUDA runtime/driver call failed */
+  MOE_ERR_DEVICE_TIMEOUT = 5,   /* a bounded device-side wait ran out */
+  MOE_ERR_UNSUPPORTED_ARCH = 6, /* current device is not sm_100 */
+  MOE_ERR_DEVICE_BOUNDS = 7     /* device found routing metadata out of range */
+} moe_status_t;
+
+/* Tile policy of the grouped expert GEMMs (moe_forward_ex / grouped calls). */
+enum {
+  MOE_TILES_AUTO = 0,   /* chosen from the mean rows per expert, T*k/E */
+  MOE_TILES_SMALL = 1,  /* <= 64 token rows per tile pass, 5-stage ring: decode */
+  MOE_TILES_LARGE = 2   /* <= 256 token rows per tile pass, 3-stage ring: prefill */
+};
+
+/* Router logits implementation. */
+enum {
+  MOE_ROUTER_AUTO = 0,
+  MOE_ROUTER_FMA = 1,   /* fp32 CUDA-core dot products */
+  MOE_ROUTER_TC = 2     /* fp32 W split into three bf16 terms, tcgen05 MMA, fp32 accumulate */
+};
+
+/* Human-readable name of a status code (static storage). */
+const char *moe_status_string(int status);
+
+/* ABI version of this header (incremented on incompatible changes). */
+int moe_abi_version(void);
+
+/* Byte offsets of the intermediates inside the workspace (for inspection
+ * after moe_forward; all 256-byte aligned).  Regions:
+ *   topk_ids [T,k] i32, topk_w [T,k] f32, counts [E] i32, offsets [E+1] i32,
+ *   sorted_token_ids [T*k] i32, inv_perm [T,k] i32, h [T*k, I] bf16,
+ *   o [T*k, H] f32, h_shared [T, I_s] bf16, o_shared [T, H] f32,
+ *   logits [T, E] f32, router_split [3, H, E] bf16, block_hist (permute). */
+typedef struct moe_workspace_layout {
+  size_t status, topk_ids, topk_w, counts, offsets, sorted_token_ids, inv_perm;
+  size_t h, o, h_shared, o_shared, logits, router_split, block_hist;
+  size_t total;
+} moe_workspace_layout_t;
+
+moe_status_t moe_workspace_layout(int T, int H, int E, int I, int k, int I_s,
+                                  moe_workspace_layout_t *out);
+
+/* Workspace bytes needed for the layer shapes (I_s = 0: no shared expert). */
+moe_status_t moe_workspace_size(int T, int H, int E, int I, int k, int I_s, size_t *bytes);
+
+/* Reads the device status word of `workspace` (synchronises `stream`).
+ * *out receives MOE_OK or the first error a kernel recorded. */
+moe_status_t moe_get_device_status(const void *workspace, void *stream, int32_t *out);
+
+/* Resets the device status word to MOE_OK (stream-ordered). */
+moe_status_t moe_clear_device_status(void *workspace, void *stream);
+
+/* Route: topk_ids [T,k] i32 and topk_w [T,k] f32 from x [T,H] bf16,
+ * W_router [H,E] f32 and an optional per-expert logit bias [E] f32 (NULL
+ * for none; added before softmax).  Logits are fp32; ids follow descending
+ * logit with ties to the lower expert id. */
+moe_status_t moe_route(const uint16_t *x, const float *w_router, const float *bias,
+                       int T, int H, int E, int k,
+                       int32_t *topk_ids, float *topk_w,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/* Same, with the logits implementation chosen explicitly (MOE_ROUTER_*). */
+moe_status_t moe_route_ex(const uint16_t *x, const float *w_router, const float *bias,
+                          int T, int H, int E, int k,
+                          int32_t *topk_ids, float *topk_w, int router_impl,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/* Permute: counts [E], offsets [E+1] (exclusive prefix sum, offsets[E] =
+ * T*k), sorted_token_ids [T*k] (permuted row -> token) and inv_perm [T,k]
+ * (slot -> permuted row) from topk_ids [T,k].  Deterministic: experts
+ * ascending, tokens ascending within an expert.  An id outside [0,E) sets
+ * MOE_ERR_DEVICE_BOUNDS in the device status word. */
+moe_status_t moe_permute(const int32_t *topk_ids, int T, int E, int k,
+                         int32_t *counts, int32_t *offsets,
+                         int32_t *sorted_token_ids, int32_t *inv_perm,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
+/* Grouped gate/up GEMM with SwiGLU: for every permuted row r in
+ * [offsets[e], offsets[e+1]), h[r, :] = bf16(silu(g) * u) with
+ * [g | u] = x[sorted_token_ids[r], :] . W_gate_up[e]  (W_gate_up [E, H, 2I],
+ * columns [0,I) gate, [I,2I) up; fp32 accumulation).  The rows of x are
+ * gathered inside the kernel; no permuted copy of x is made.  h is
+ * [T*k, I] bf16.  tile_policy: MOE_TILES_*. */
+moe_status_t moe_grouped_swiglu(const uint16_t *x, const uint16_t *w_gate_up,
+                                const int32_t *offsets, const int32_t *sorted_token_ids,
+                                int T, int H, int E, int I, int k, int tile_policy,
+                                uint16_t *h, void *workspace, size_t workspace_bytes,
+                                void *stream);
+
+/* Grouped down GEMM: o[r, :] = h[r, :] . W_down[e] for every permuted row
+ * (W_down [E, I, H] bf16, h [R, I] bf16, o [R, H] f32, R = offsets[E]).
+ * offsets may be NULL for one group of R = rows rows (E must then be 1). */
+moe_status_t moe_grouped_down(const uint16_t *h, const uint16_t *w_down, const int32_t *offsets,
+                              int rows, int H, int E, int I, int tile_policy, float *o,
+                              void *workspace, size_t workspace_bytes, void *stream);
+
+/* Down GEMM + weighted combine: y [T,H] bf16 from h [T*k, I] bf16 (permuted
+ * order), W_down [E, I, H] bf16, topk_w [T,k] f32, inv_perm [T,k] i32,
+ * offsets [E+1] i32 and an optional shared-expert output shared_out [T,H]
+ * f32 (NULL for none), added after the k routed terms.  The k terms of a
+ * token are summed in slot order j = 0..k-1 in fp32, so y is bitwise
+ * reproducible. */
+moe_status_t moe_down_combine(const uint16_t *h, const uint16_t *w_down,
+                              const float *topk_w, const int32_t *inv_perm,
+                              const int32_t *offsets, const float *shared_out,
+                              int T, int H, int E, int I, int k, int tile_policy,
+                              uint16_t *y, void *workspace, size_t workspace_bytes,
+                              void *stream);
+
+/* The whole layer: y [T,H] bf16.  W_sh_gate_up [H, 2 I_s] and W_sh_down
+ * [I_s, H] describe the optional shared expert (both NULL and I_s = 0 for
+ * none).  Intermediates stay in the workspace (moe_workspace_layout). */
+moe_status_t moe_forward(const uint16_t *x, const float *w_router, const float *bias,
+                         const uint16_t *w_gate_up, const uint16_t *w_down,
+                         const uint16_t *w_sh_gate_up, const uint16_t *w_sh_down, int I_s,
+                         int T, int H, int E, int I, int k,
+                         uint16_t *y, void *workspace, size_t workspace_bytes, void *stream);
+
+/* moe_forward with explicit choices (MOE_TILES_*, MOE_ROUTER_*), optional
+ * stage timing events and a launch count. */
+typedef struct moe_forward_options {
+  int tile_policy;
+  int router_impl;
+  /* Optional timing hooks: a non-NULL stage_events[i] (a cudaEvent_t owned
+   * by the caller) is recorded on the stream at stage boundary i:
+   * 0 before routing, 1 after routing, 2 after the permutation, 3 after the
+   * shared expert, 4 after the gate/up GEMM, 5 after the down GEMM, 6 after
+   * the combine. */
+  void *stage_events[7];
+  /* Output: the number of kernels this call enqueued. */
+  int launches;
+  int reserved[5];
+} moe_forward_options_t;
+
+moe_status_t moe_forward_ex(const uint16_t *x, const float *w_router, const float *bias,
+                            const uint16_t *w_gate_up, const uint16_t *w_down,
+                            const uint16_t *w_sh_gate_up, const uint16_t *w_sh_down, int I_s,
+                            int T, int H, int E, int I, int k,
+                            uint16_t *y, void *workspace, size_t workspace_bytes,
+                            moe_forward_options_t *options, void *stream);
+
+/* Failure-detection self test: launches one block that waits, with the
+ * library's bounded wait, on a barrier nothing will complete.  After
+ * timeout_ns the wait gives up, the kernel records MOE_ERR_DEVICE_TIMEOUT
+ * in the workspace status word and returns; the context stays usable.
+ * Read the result with moe_get_device_status(). */
+moe_status_t moe_selftest_timeout(void *workspace, size_t workspace_bytes,
+                                  uint64_t timeout_ns, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

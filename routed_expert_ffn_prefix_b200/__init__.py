@@ -1,0 +1,277 @@
+"""Python binding of the B200 routed-expert MoE layer (libmoe_b200.so).
+
+Argument marshalling only: every step of the layer runs in the library's
+CUDA kernels.  Tensors are torch CUDA tensors (bf16 as torch.bfloat16);
+calls are enqueued on torch's current CUDA stream.  The C ABI and its
+conventions are documented in include/moe.h.
+
+There is no fallback: if the shared library is missing or the device is not
+an sm_100 GPU, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+from . import build as _build
+
+__all__ = [
+    "MoEError", "lib", "TILES_AUTO", "TILES_SMALL", "TILES_LARGE", "ROUTER_AUTO", "ROUTER_FMA", "ROUTER_TC",
+    "workspace_size", "workspace_layout", "alloc_workspace", "route", "permute", "grouped_swiglu",
+    "grouped_down", "down_combine", "forward", "device_status", "clear_device_status", "selftest_timeout",
+    "STATUS",
+]
+
+TILES_AUTO, TILES_SMALL, TILES_LARGE = 0, 1, 2
+ROUTER_AUTO, ROUTER_FMA, ROUTER_TC = 0, 1, 2
+
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_ALIGNMENT", 3: "MOE_ERR_WORKSPACE",
+          4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT", 6: "MOE_ERR_UNSUPPORTED_ARCH",
+          7: "MOE_ERR_DEVICE_BOUNDS"}
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {lib().moe_status_string(status).decode()}")
+
+
+class _Layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in (
+        "status", "topk_ids", "topk_w", "counts", "offsets", "sorted_token_ids", "inv_perm",
+        "h", "o", "h_shared", "o_shared", "logits", "router_split", "block_hist", "total")]
+
+
+class _Options(ctypes.Structure):
+    _fields_ = [("tile_policy", ctypes.c_int), ("router_impl", ctypes.c_int),
+                ("stage_events", ctypes.c_void_p * 7), ("launches", ctypes.c_int), ("reserved", ctypes.c_int * 5)]
+
+
+_P, _I, _Z, _U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint64
+_SIGS = {
+    "moe_status_string": ([_I], ctypes.c_char_p),
+    "moe_abi_version": ([], _I),
+    "moe_workspace_layout": ([_I] * 6 + [ctypes.POINTER(_Layout)], _I),
+    "moe_workspace_size": ([_I] * 6 + [ctypes.POINTER(ctypes.c_size_t)], _I),
+    "moe_get_device_status": ([_P, _P, ctypes.POINTER(ctypes.c_int32)], _I),
+    "moe_clear_device_status": ([_P, _P], _I),
+    "moe_route": ([_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _Z, _P], _I),
+    "moe_route_ex": ([_P, _P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _Z, _P], _I),
+    "moe_permute": ([_P, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P], _I),
+    "moe_grouped_swiglu": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _Z, _P], _I),
+    "moe_grouped_down": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _Z, _P], _I),
+    "moe_down_combine": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _Z, _P], _I),
+    "moe_forward": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _Z, _P], _I),
+    "moe_forward_ex": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _Z,
+                        ctypes.POINTER(_Options), _P], _I),
+    "moe_selftest_timeout": ([_P, _Z, _U64, _P], _I),
+}
+
+_LIB = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (loaded on first use; raises if it was never built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(_build.LIB_PATH):
+            raise ImportError(f"{_build.LIB_PATH} is missing; build it with "
+                              "routed_expert_ffn_prefix_b200.build.build()")
+        handle = ctypes.CDLL(_build.LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            fn = getattr(handle, name)
+            fn.argtypes, fn.restype = args, res
+        _LIB = handle
+    return _LIB
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise MoEError(status, what)
+
+
+def _stream():
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t, dtype, name, ndim=None):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims")
+
+
+def workspace_layout(T, H, E, I, k, I_s=0) -> dict:
+    L = _Layout()
+    _check(lib().moe_workspace_layout(T, H, E, I, k, I_s, ctypes.byref(L)), "moe_workspace_layout")
+    return {n: getattr(L, n) for n, _ in _Layout._fields_}
+
+
+def workspace_size(T, H, E, I, k, I_s=0) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().moe_workspace_size(T, H, E, I, k, I_s, ctypes.byref(n)), "moe_workspace_size")
+    return n.value
+
+
+def alloc_workspace(T, H, E, I, k, I_s=0, device="cuda"):
+    """Device workspace for the layer shapes, status word cleared."""
+    import torch
+    ws = torch.empty(workspace_size(T, H, E, I, k, I_s), dtype=torch.uint8, device=device)
+    clear_device_status(ws)
+    return ws
+
+
+def device_status(ws) -> int:
+    out = ctypes.c_int32()
+    _check(lib().moe_get_device_status(_ptr(ws), _stream(), ctypes.byref(out)), "moe_get_device_status")
+    return out.value
+
+
+def clear_device_status(ws) -> None:
+    _check(lib().moe_clear_device_status(_ptr(ws), _stream()), "moe_clear_device_status")
+
+
+def route(x, w_router, bias, k, ws, impl=ROUTER_AUTO, out=None):
+    """topk_ids [T,k] int32, topk_w [T,k] float32."""
+    import torch
+    _need(x, torch.bfloat16, "x", 2)
+    _need(w_router, torch.float32, "w_router", 2)
+    if bias is not None:
+        _need(bias, torch.float32, "bias", 1)
+    T, H = x.shape
+    E = w_router.shape[1]
+    ids, w = out if out is not None else (
+        torch.empty(T, k, dtype=torch.int32, device=x.device), torch.empty(T, k, dtype=torch.float32, device=x.device))
+    _check(lib().moe_route_ex(_ptr(x), _ptr(w_router), _ptr(bias), T, H, E, k, _ptr(ids), _ptr(w), impl,
+                              _ptr(ws), ws.numel(), _stream()), "moe_route")
+    return ids, w
+
+
+def permute(topk_ids, E, ws):
+    """counts [E], offsets [E+1], sorted_token_ids [T*k], inv_perm [T,k] (int32)."""
+    import torch
+    _need(topk_ids, torch.int32, "topk_ids", 2)
+    T, k = topk_ids.shape
+    dev = topk_ids.device
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    sids = torch.empty(T * k, dtype=torch.int32, device=dev)
+    inv = torch.empty(T, k, dtype=torch.int32, device=dev)
+    _check(lib().moe_permute(_ptr(topk_ids), T, E, k, _ptr(counts), _ptr(offsets), _ptr(sids), _ptr(inv),
+                             _ptr(ws), ws.numel(), _stream()), "moe_permute")
+    return counts, offsets, sids, inv
+
+
+def grouped_swiglu(x, w_gate_up, offsets, sorted_token_ids, k, ws, tiles=TILES_AUTO, out=None):
+    """h [T*k, I] bf16 in permuted order."""
+    import torch
+    _need(x, torch.bfloat16, "x", 2)
+    _need(w_gate_up, torch.bfloat16, "w_gate_up", 3)
+    _need(offsets, torch.int32, "offsets", 1)
+    _need(sorted_token_ids, torch.int32, "sorted_token_ids", 1)
+    T, H = x.shape
+    E, _, I2 = w_gate_up.shape
+    I = I2 // 2
+    h = out if out is not None else torch.empty(T * k, I, dtype=torch.bfloat16, device=x.device)
+    _check(lib().moe_grouped_swiglu(_ptr(x), _ptr(w_gate_up), _ptr(offsets), _ptr(sorted_token_ids), T, H, E, I, k,
+                                    tiles, _ptr(h), _ptr(ws), ws.numel(), _stream()), "moe_grouped_swiglu")
+    return h
+
+
+def grouped_down(h, w_down, offsets, ws, tiles=TILES_AUTO, out=None):
+    """o [rows, H] float32 = h . W_down[e] per group (offsets None: one group)."""
+    import torch
+    _need(h, torch.bfloat16, "h", 2)
+    _need(w_down, torch.bfloat16, "w_down", 3)
+    rows, I = h.shape
+    E, _, H = w_down.shape
+    o = out if out is not None else torch.empty(rows, H, dtype=torch.float32, device=h.device)
+    _check(lib().moe_grouped_down(_ptr(h), _ptr(w_down), _ptr(offsets), rows, H, E, I, tiles, _ptr(o),
+                                  _ptr(ws), ws.numel(), _stream()), "moe_grouped_down")
+    return o
+
+
+def down_combine(h, w_down, topk_w, inv_perm, offsets, shared_out, ws, tiles=TILES_AUTO, out=None):
+    """y [T,H] bf16."""
+    import torch
+    _need(h, torch.bfloat16, "h", 2)
+    _need(w_down, torch.bfloat16, "w_down", 3)
+    _need(topk_w, torch.float32, "topk_w", 2)
+    _need(inv_perm, torch.int32, "inv_perm", 2)
+    if shared_out is not None:
+        _need(shared_out, torch.float32, "shared_out", 2)
+    T, k = topk_w.shape
+    E, I, H = w_down.shape
+    y = out if out is not None else torch.empty(T, H, dtype=torch.bfloat16, device=h.device)
+    _check(lib().moe_down_combine(_ptr(h), _ptr(w_down), _ptr(topk_w), _ptr(inv_perm), _ptr(offsets),
+                                  _ptr(shared_out), T, H, E, I, k, tiles, _ptr(y), _ptr(ws), ws.numel(),
+                                  _stream()), "moe_down_combine")
+    return y
+
+
+def forward(x, w_router, bias, w_gate_up, w_down, k, ws, w_sh_gate_up=None, w_sh_down=None,
+            tiles=TILES_AUTO, router=ROUTER_AUTO, out=None, stage_events=None, info=None):
+    """The whole layer: y [T,H] bf16.
+
+    stage_events: optional list of 7 torch.cuda.Event recorded at the stage
+    boundaries (see include/moe.h); info: optional dict that receives the
+    number of kernels enqueued under "launches"."""
+    import torch
+    _need(x, torch.bfloat16, "x", 2)
+    _need(w_router, torch.float32, "w_router", 2)
+    _need(w_gate_up, torch.bfloat16, "w_gate_up", 3)
+    _need(w_down, torch.bfloat16, "w_down", 3)
+    T, H = x.shape
+    E, _, I2 = w_gate_up.shape
+    I = I2 // 2
+    I_s = 0
+    if w_sh_gate_up is not None:
+        _need(w_sh_gate_up, torch.bfloat16, "w_sh_gate_up", 2)
+        _need(w_sh_down, torch.bfloat16, "w_sh_down", 2)
+        I_s = w_sh_gate_up.shape[1] // 2
+    y = out if out is not None else torch.empty(T, H, dtype=torch.bfloat16, device=x.device)
+    opt = _Options(tiles, router)
+    if stage_events is not None:
+        for i, ev in enumerate(stage_events):
+            if ev is not None:
+                opt.stage_events[i] = ev.cuda_event
+    _check(lib().moe_forward_ex(_ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate_up), _ptr(w_down),
+                                _ptr(w_sh_gate_up), _ptr(w_sh_down), I_s, T, H, E, I, k, _ptr(y), _ptr(ws),
+                                ws.numel(), ctypes.byref(opt), _stream()), "moe_forward")
+    if info is not None:
+        info["launches"] = opt.launches
+    return y
+
+
+def selftest_timeout(ws, timeout_ns: int) -> None:
+    _check(lib().moe_selftest_timeout(_ptr(ws), ws.numel(), timeout_ns, _stream()), "moe_selftest_timeout")
+
+
+def workspace_view(ws, T, H, E, I, k, I_s=0) -> dict:
+    """Typed views of the intermediates inside a workspace (after forward)."""
+    import torch
+    L = workspace_layout(T, H, E, I, k, I_s)
+
+    def view(name, dtype, shape):
+        n = 1
+        for s in shape:
+            n *= s
+        nbytes = n * torch.empty(0, dtype=dtype).element_size()
+        return ws[L[name]:L[name] + nbytes].view(dtype).view(*shape)
+
+    return dict(topk_ids=view("topk_ids", torch.int32, (T, k)), topk_w=view("topk_w", torch.float32, (T, k)),
+                counts=view("counts", torch.int32, (E,)), offsets=view("offsets", torch.int32, (E + 1,)),
+                sorted_token_ids=view("sorted_token_ids", torch.int32, (T * k,)),
+                inv_perm=view("inv_perm", torch.int32, (T, k)), h=view("h", torch.bfloat16, (T * k, I)),
+                logits=view("logits", torch.float32, (T, E)))

@@ -1,0 +1,470 @@
+// api.cu -- the C ABI declared in include/moe.h: argument checks, workspace
+// layout, TMA descriptors and the order of the layer's kernels.
+#include <mutex>
+
+#include "kernels.h"
+
+using namespace moe;
+
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded device wait
+constexpr int kMaxK = 64;
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- workspace
+moe_workspace_layout_t make_layout(int T, int H, int E, int I, int k, int I_s) {
+  moe_workspace_layout_t L{};
+  const size_t tk = (size_t)T * k;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  L.status = take(sizeof(DevStatus));
+  L.topk_ids = take(tk * 4);
+  L.topk_w = take(tk * 4);
+  L.counts = take((size_t)E * 4);
+  L.offsets = take((size_t)(E + 1) * 4);
+  L.sorted_token_ids = take(tk * 4);
+  L.inv_perm = take(tk * 4);
+  L.block_hist = take((size_t)permute_num_blocks(T, k) * E * 4);
+  L.logits = take((size_t)T * E * 4);
+  L.router_split = take((size_t)3 * H * E * 2);
+  L.h = take(tk * I * 2);
+  L.o = take(tk * H * 4);
+  L.h_shared = take((size_t)T * I_s * 2);
+  L.o_shared = take(I_s > 0 ? (size_t)T * H * 4 : 0);
+  L.total = off;
+  return L;
+}
+
+// ---------------------------------------------------------------- CUDA helpers
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor [d2][d1][d0] (d0 contiguous), box 64 x 64 x 1, 128-byte swizzle.
+bool make_weight_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct DeviceInfo {
+  int num_sms;
+};
+
+moe_status_t check_device(DeviceInfo* info) {
+  int dev = 0, major = 0, minor = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (major != 10 || minor != 0) return MOE_ERR_UNSUPPORTED_ARCH;
+  info->num_sms = sms;
+  return MOE_OK;
+}
+
+inline moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                     \
+  do {                                    \
+    const moe_status_t _s = (expr);       \
+    if (_s != MOE_OK) return _s;          \
+  } while (0)
+
+// ---------------------------------------------------------------- argument checks
+moe_status_t check_shapes(int T, int H, int E, int I, int k, bool need_I) {
+  if (T < 1 || H < 1 || E < 1 || E > kMaxExperts || k < 1 || k > E || k > kMaxK) return MOE_ERR_INVALID_ARG;
+  if ((long long)T * k >= (1ll << 31)) return MOE_ERR_INVALID_ARG;
+  if (H % 256 != 0) return MOE_ERR_ALIGNMENT;
+  if (need_I) {
+    if (I < 1) return MOE_ERR_INVALID_ARG;
+    if (I % 128 != 0) return MOE_ERR_ALIGNMENT;
+  }
+  return MOE_OK;
+}
+
+moe_status_t check_ws(const void* ws, size_t ws_bytes, size_t need) {
+  if (ws == nullptr || ws_bytes < need) return MOE_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return MOE_ERR_ALIGNMENT;
+  return MOE_OK;
+}
+
+template <typename... P>
+bool all_nonnull(P... p) {
+  return ((p != nullptr) && ...);
+}
+template <typename... P>
+bool all_aligned(P... p) {
+  return (aligned16(p) && ...);
+}
+
+inline DevStatus* status_of(void* ws) { return reinterpret_cast<DevStatus*>(ws); }
+template <typename Tp>
+inline Tp* at(void* ws, size_t off) {
+  return reinterpret_cast<Tp*>(static_cast<char*>(ws) + off);
+}
+
+int choose_tiles(int policy, long long rows, int groups) {
+  if (policy == MOE_TILES_SMALL || policy == MOE_TILES_LARGE) return policy;
+  // mean rows per group: small groups stream weights under few rows
+  return rows > 48ll * groups ? MOE_TILES_LARGE : MOE_TILES_SMALL;
+}
+
+// ---------------------------------------------------------------- stage launchers (no checks)
+moe_status_t run_route(const uint16_t* x, const float* w_router, const float* bias, int T, int H, int E, int k,
+                       int32_t* ids, float* w, int impl, void* ws, const moe_workspace_layout_t& L,
+                       const DeviceInfo& dev, cudaStream_t s) {
+  DevStatus* st = status_of(ws);
+  float* logits = at<float>(ws, L.logits);
+  if (impl == MOE_ROUTER_AUTO) impl = (T >= 1024 && E % 8 == 0) ? MOE_ROUTER_TC : MOE_ROUTER_FMA;
+  if (impl == MOE_ROUTER_TC) {
+    if (E % 8 != 0) return MOE_ERR_ALIGNMENT;
+    uint16_t* planes = at<uint16_t>(ws, L.router_split);
+    MOE_TRY(cuda_status(launch_router_split(w_router, H, E, planes, s)));
+    CUtensorMap map;
+    if (!make_weight_map(&map, planes, (uint64_t)E, (uint64_t)H, 3)) return MOE_ERR_CUDA;
+    GemmArgs a{};
+    a.offsets = nullptr;
+    a.row_index = nullptr;
+    a.b_src = x;
+    a.src_rows = T;
+    a.groups = 1;
+    a.single_rows = T;
+    a.K = H;
+    a.krep = 3;
+    a.a_dim2_rep = 1;
+    a.n_blocks = (E + 255) / 256;
+    a.col_stride = 256;
+    a.col1_off = 128;
+    a.out = logits;
+    a.ld_out = E;
+    a.out_col_stride = 256;
+    a.out_col1_off = 128;
+    a.n_valid = E;
+    a.rows_cap = T;
+    a.status = st;
+    a.timeout_ns = kDefaultTimeoutNs;
+    const int tiles = T >= 2048 ? MOE_TILES_LARGE : MOE_TILES_SMALL;
+    MOE_TRY(cuda_status(launch_grouped_gemm(map, a, EPI_STORE_F32, tiles, dev.num_sms, s)));
+  } else {
+    MOE_TRY(cuda_status(launch_router_logits_fma(x, w_router, T, H, E, logits, s)));
+  }
+  return cuda_status(launch_topk(logits, bias, T, E, k, ids, w, st, s));
+}
+
+moe_status_t run_swiglu(const uint16_t* x, int src_rows, const uint16_t* w_gate_up, const int32_t* offsets,
+                        const int32_t* row_index, int rows, int H, int E, int I, int tiles, uint16_t* h,
+                        DevStatus* st, const DeviceInfo& dev, cudaStream_t s) {
+  CUtensorMap map;
+  if (!make_weight_map(&map, w_gate_up, 2ull * I, (uint64_t)H, (uint64_t)E)) return MOE_ERR_CUDA;
+  GemmArgs a{};
+  a.offsets = offsets;
+  a.row_index = row_index;
+  a.b_src = x;
+  a.src_rows = src_rows;
+  a.groups = E;
+  a.single_rows = rows;
+  a.K = H;
+  a.krep = 1;
+  a.a_dim2_rep = 0;
+  a.n_blocks = I / 128;
+  a.col_stride = 128;
+  a.col1_off = I;
+  a.out = h;
+  a.ld_out = I;
+  a.out_col_stride = 128;
+  a.out_col1_off = 0;
+  a.n_valid = I;
+  a.rows_cap = rows;
+  a.status = st;
+  a.timeout_ns = kDefaultTimeoutNs;
+  return cuda_status(launch_grouped_gemm(map, a, EPI_SWIGLU, tiles, dev.num_sms, s));
+}
+
+moe_status_t run_down(const uint16_t* h, const uint16_t* w_down, const int32_t* offsets, int rows, int H, int E,
+                      int I, int tiles, float* o, DevStatus* st, const DeviceInfo& dev, cudaStream_t s) {
+  CUtensorMap map;
+  if (!make_weight_map(&map, w_down, (uint64_t)H, (uint64_t)I, (uint64_t)E)) return MOE_ERR_CUDA;
+  GemmArgs a{};
+  a.offsets = offsets;
+  a.row_index = nullptr;
+  a.b_src = h;
+  a.src_rows = rows;
+  a.groups = E;
+  a.single_rows = rows;
+  a.K = I;
+  a.krep = 1;
+  a.a_dim2_rep = 0;
+  a.n_blocks = H / 256;
+  a.col_stride = 256;
+  a.col1_off = 128;
+  a.out = o;
+  a.ld_out = H;
+  a.out_col_stride = 256;
+  a.out_col1_off = 128;
+  a.n_valid = H;
+  a.rows_cap = rows;
+  a.status = st;
+  a.timeout_ns = kDefaultTimeoutNs;
+  return cuda_status(launch_grouped_gemm(map, a, EPI_STORE_F32, tiles, dev.num_sms, s));
+}
+
+}  // namespace
+
+// ==================================================================== C ABI
+extern "C" {
+
+const char* moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: null pointer or unsupported shape";
+    case MOE_ERR_ALIGNMENT: return "MOE_ERR_ALIGNMENT: pointer or dimension not aligned as required";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing or too small";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call failed";
+    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT: a bounded device wait ran out";
+    case MOE_ERR_UNSUPPORTED_ARCH: return "MOE_ERR_UNSUPPORTED_ARCH: device is not sm_100";
+    case MOE_ERR_DEVICE_BOUNDS: return "MOE_ERR_DEVICE_BOUNDS: routing metadata out of range on the device";
+    default: return "unknown moe status";
+  }
+}
+
+int moe_abi_version(void) { return 1; }
+
+moe_status_t moe_workspace_layout(int T, int H, int E, int I, int k, int I_s, moe_workspace_layout_t* out) {
+  if (out == nullptr || I_s < 0) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_shapes(T, H, E, I, k, true));
+  if (I_s > 0 && I_s % 128 != 0) return MOE_ERR_ALIGNMENT;
+  *out = make_layout(T, H, E, I, k, I_s);
+  return MOE_OK;
+}
+
+moe_status_t moe_workspace_size(int T, int H, int E, int I, int k, int I_s, size_t* bytes) {
+  if (bytes == nullptr) return MOE_ERR_INVALID_ARG;
+  moe_workspace_layout_t L;
+  MOE_TRY(moe_workspace_layout(T, H, E, I, k, I_s, &L));
+  *bytes = L.total;
+  return MOE_OK;
+}
+
+moe_status_t moe_get_device_status(const void* workspace, void* stream, int32_t* out) {
+  if (workspace == nullptr || out == nullptr) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DevStatus h{};
+  if (cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  *out = h.code;
+  return MOE_OK;
+}
+
+moe_status_t moe_clear_device_status(void* workspace, void* stream) {
+  if (workspace == nullptr) return MOE_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(workspace, 0, sizeof(DevStatus), static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_route_ex(const uint16_t* x, const float* w_router, const float* bias, int T, int H, int E, int k,
+                          int32_t* topk_ids, float* topk_w, int router_impl, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  if (!all_nonnull(x, w_router, topk_ids, topk_w)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_shapes(T, H, E, 0, k, false));
+  if (router_impl < MOE_ROUTER_AUTO || router_impl > MOE_ROUTER_TC) return MOE_ERR_INVALID_ARG;
+  if (!all_aligned(x, w_router, topk_ids, topk_w) || (bias && !aligned16(bias))) return MOE_ERR_ALIGNMENT;
+  const moe_workspace_layout_t L = make_layout(T, H, E, 0, k, 0);
+  MOE_TRY(check_ws(workspace, workspace_bytes, L.h));
+  DeviceInfo dev;
+  MOE_TRY(check_device(&dev));
+  return run_route(x, w_router, bias, T, H, E, k, topk_ids, topk_w, router_impl, workspace, L, dev,
+                   static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_route(const uint16_t* x, const float* w_router, const float* bias, int T, int H, int E, int k,
+                       int32_t* topk_ids, float* topk_w, void* workspace, size_t workspace_bytes, void* stream) {
+  return moe_route_ex(x, w_router, bias, T, H, E, k, topk_ids, topk_w, MOE_ROUTER_AUTO, workspace,
+                      workspace_bytes, stream);
+}
+
+moe_status_t moe_permute(const int32_t* topk_ids, int T, int E, int k, int32_t* counts, int32_t* offsets,
+                         int32_t* sorted_token_ids, int32_t* inv_perm, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  if (!all_nonnull(topk_ids, counts, offsets, sorted_token_ids, inv_perm)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_shapes(T, 256, E, 0, k, false));
+  if (!all_aligned(topk_ids, counts, offsets, sorted_token_ids, inv_perm)) return MOE_ERR_ALIGNMENT;
+  const moe_workspace_layout_t L = make_layout(T, 0, E, 0, k, 0);
+  MOE_TRY(check_ws(workspace, workspace_bytes, L.logits));
+  DeviceInfo dev;
+  MOE_TRY(check_device(&dev));
+  return cuda_status(launch_permute(topk_ids, T, E, k, counts, offsets, sorted_token_ids, inv_perm,
+                                    at<int32_t>(workspace, L.block_hist), status_of(workspace),
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_grouped_swiglu(const uint16_t* x, const uint16_t* w_gate_up, const int32_t* offsets,
+                                const int32_t* sorted_token_ids, int T, int H, int E, int I, int k,
+                                int tile_policy, uint16_t* h, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  if (!all_nonnull(x, w_gate_up, offsets, sorted_token_ids, h)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_shapes(T, H, E, I, k, true));
+  if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_LARGE) return MOE_ERR_INVALID_ARG;
+  if (!all_aligned(x, w_gate_up, offsets, sorted_token_ids, h)) return MOE_ERR_ALIGNMENT;
+  MOE_TRY(check_ws(workspace, workspace_bytes, sizeof(DevStatus)));
+  DeviceInfo dev;
+  MOE_TRY(check_device(&dev));
+  const int rows = T * k;
+  return run_swiglu(x, T, w_gate_up, offsets, sorted_token_ids, rows, H, E, I,
+                    choose_tiles(tile_policy, rows, E), h, status_of(workspace), dev,
+                    static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_grouped_down(const uint16_t* h, const uint16_t* w_down, const int32_t* offsets, int rows, int H,
+                              int E, int I, int tile_policy, float* o, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  if (!all_nonnull(h, w_down, o)) return MOE_ERR_INVALID_ARG;
+  if (rows < 1 || E < 1 || E > kMaxExperts || H < 1 || I < 1) return MOE_ERR_INVALID_ARG;
+  if (offsets == nullptr && E != 1) return MOE_ERR_INVALID_ARG;
+  if (H % 256 != 0 || I % 128 != 0) return MOE_ERR_ALIGNMENT;
+  if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_LARGE) return MOE_ERR_INVALID_ARG;
+  if (!all_aligned(h, w_down, o) || (offsets && !aligned16(offsets))) return MOE_ERR_ALIGNMENT;
+  MOE_TRY(check_ws(workspace, workspace_bytes, sizeof(DevStatus)));
+  DeviceInfo dev;
+  MOE_TRY(check_device(&dev));
+  return run_down(h, w_down, offsets, rows, H, E, I, choose_tiles(tile_policy, rows, E), o, status_of(workspace),
+                  dev, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_down_combine(const uint16_t* h, const uint16_t* w_down, const float* topk_w,
+                              const int32_t* inv_perm, const int32_t* offsets, const float* shared_out, int T,
+                              int H, int E, int I, int k, int tile_policy, uint16_t* y, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (!all_nonnull(h, w_down, topk_w, inv_perm, offsets, y)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_shapes(T, H, E, I, k, true));
+  if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_LARGE) return MOE_ERR_INVALID_ARG;
+  if (!all_aligned(h, w_down, topk_w, inv_perm, offsets, y) || (shared_out && !aligned16(shared_out)))
+    return MOE_ERR_ALIGNMENT;
+  const moe_workspace_layout_t L = make_layout(T, H, E, I, k, 0);
+  MOE_TRY(check_ws(workspace, workspace_bytes, L.h_shared));
+  DeviceInfo dev;
+  MOE_TRY(check_device(&dev));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int rows = T * k;
+  float* o = at<float>(workspace, L.o);
+  DevStatus* st = status_of(workspace);
+  MOE_TRY(run_down(h, w_down, offsets, rows, H, E, I, choose_tiles(tile_policy, rows, E), o, st, dev, s));
+  return cuda_status(launch_combine(o, topk_w, inv_perm, shared_out, T, H, k, rows, y, st, s));
+}
+
+moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const float* bias, const uint16_t* w_gate_up,
+                            const uint16_t* w_down, const uint16_t* w_sh_gate_up, const uint16_t* w_sh_down, int I_s,
+                            int T, int H, int E, int I, int k, uint16_t* y, void* workspace,
+                            size_t workspace_bytes, moe_forward_options_t* options, void* stream) {
+  if (!all_nonnull(x, w_router, w_gate_up, w_down, y)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_shapes(T, H, E, I, k, true));
+  const bool shared = w_sh_gate_up != nullptr || w_sh_down != nullptr || I_s != 0;
+  if (shared) {
+    if (!all_nonnull(w_sh_gate_up, w_sh_down) || I_s < 1) return MOE_ERR_INVALID_ARG;
+    if (I_s % 128 != 0) return MOE_ERR_ALIGNMENT;
+    if (!all_aligned(w_sh_gate_up, w_sh_down)) return MOE_ERR_ALIGNMENT;
+  }
+  const int tile_policy = options ? options->tile_policy : MOE_TILES_AUTO;
+  const int router_impl = options ? options->router_impl : MOE_ROUTER_AUTO;
+  if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_LARGE) return MOE_ERR_INVALID_ARG;
+  if (router_impl < MOE_ROUTER_AUTO || router_impl > MOE_ROUTER_TC) return MOE_ERR_INVALID_ARG;
+  if (!all_aligned(x, w_router, w_gate_up, w_down, y) || (bias && !aligned16(bias))) return MOE_ERR_ALIGNMENT;
+  const moe_workspace_layout_t L = make_layout(T, H, E, I, k, shared ? I_s : 0);
+  MOE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  DeviceInfo dev;
+  MOE_TRY(check_device(&dev));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* ws = workspace;
+  DevStatus* st = status_of(ws);
+  int32_t* ids = at<int32_t>(ws, L.topk_ids);
+  float* tw = at<float>(ws, L.topk_w);
+  int32_t* counts = at<int32_t>(ws, L.counts);
+  int32_t* offs = at<int32_t>(ws, L.offsets);
+  int32_t* sids = at<int32_t>(ws, L.sorted_token_ids);
+  int32_t* inv = at<int32_t>(ws, L.inv_perm);
+  uint16_t* h = at<uint16_t>(ws, L.h);
+  float* o = at<float>(ws, L.o);
+  const int rows = T * k;
+
+  void* const* ev = options ? options->stage_events : nullptr;
+  auto mark = [&](int i) -> moe_status_t {
+    if (ev && ev[i]) return cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s));
+    return MOE_OK;
+  };
+  int launches = 0;
+  const int ri = router_impl == MOE_ROUTER_AUTO ? ((T >= 1024 && E % 8 == 0) ? MOE_ROUTER_TC : MOE_ROUTER_FMA)
+                                                : router_impl;
+  MOE_TRY(mark(0));
+  MOE_TRY(run_route(x, w_router, bias, T, H, E, k, ids, tw, ri, ws, L, dev, s));
+  launches += ri == MOE_ROUTER_TC ? 3 : 2;
+  MOE_TRY(mark(1));
+  MOE_TRY(cuda_status(
+      launch_permute(ids, T, E, k, counts, offs, sids, inv, at<int32_t>(ws, L.block_hist), st, s)));
+  launches += 3;
+  MOE_TRY(mark(2));
+  const int tiles = choose_tiles(tile_policy, rows, E);
+  float* o_sh = nullptr;
+  if (shared) {
+    uint16_t* h_sh = at<uint16_t>(ws, L.h_shared);
+    o_sh = at<float>(ws, L.o_shared);
+    const int sh_tiles = choose_tiles(tile_policy, T, 1);
+    MOE_TRY(run_swiglu(x, T, w_sh_gate_up, nullptr, nullptr, T, H, 1, I_s, sh_tiles, h_sh, st, dev, s));
+    MOE_TRY(run_down(h_sh, w_sh_down, nullptr, T, H, 1, I_s, sh_tiles, o_sh, st, dev, s));
+    launches += 2;
+  }
+  MOE_TRY(mark(3));
+  MOE_TRY(run_swiglu(x, T, w_gate_up, offs, sids, rows, H, E, I, tiles, h, st, dev, s));
+  launches += 1;
+  MOE_TRY(mark(4));
+  MOE_TRY(run_down(h, w_down, offs, rows, H, E, I, tiles, o, st, dev, s));
+  launches += 1;
+  MOE_TRY(mark(5));
+  MOE_TRY(cuda_status(launch_combine(o, tw, inv, o_sh, T, H, k, rows, y, st, s)));
+  launches += 1;
+  MOE_TRY(mark(6));
+  if (options) options->launches = launches;
+  return MOE_OK;
+}
+
+moe_status_t moe_forward(const uint16_t* x, const float* w_router, const float* bias, const uint16_t* w_gate_up,
+                         const uint16_t* w_down, const uint16_t* w_sh_gate_up, const uint16_t* w_sh_down, int I_s,
+                         int T, int H, int E, int I, int k, uint16_t* y, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  return moe_forward_ex(x, w_router, bias, w_gate_up, w_down, w_sh_gate_up, w_sh_down, I_s, T, H, E, I, k, y,
+                        workspace, workspace_bytes, nullptr, stream);
+}
+
+moe_status_t moe_selftest_timeout(void* workspace, size_t workspace_bytes, uint64_t timeout_ns, void* stream) {
+  MOE_TRY(check_ws(workspace, workspace_bytes, sizeof(DevStatus)));
+  if (timeout_ns == 0 || timeout_ns > 10000000000ull) return MOE_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  MOE_TRY(check_device(&dev));
+  return cuda_status(launch_selftest_timeout(status_of(workspace), timeout_ns, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

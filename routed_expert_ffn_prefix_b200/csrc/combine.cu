@@ -1,0 +1,79 @@
+// combine.cu -- weighted gather-combine of the expert outputs back to token order.
+//
+// The Qwen 3.5-397B-on-Ironwood page (sec. 7.2) un-permutes the [T*k, H]
+// expert outputs and gather-reduces them per token; the Ling-2.6-1T /
+// SGLang-JAX page fuses scatter, expert FFN and gather ("Fused MoE V2").
+// Here each token's k expert rows are read through inv_perm and summed in
+// slot order j = 0..k-1 in fp32 (w_j * o_j, one fused multiply-add per
+// term), the shared-expert row (weight 1) is added last, and y is rounded
+// to bf16 once.  A fixed summation order makes y bitwise reproducible
+// run to run, whatever order the expert GEMM tiles finished in.
+//
+// Memory-bound: one block per token, float4 loads along H.
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+__global__ void __launch_bounds__(kThreads) combine_kernel(const float* __restrict__ o, const float* __restrict__ w,
+                                                         const int32_t* __restrict__ inv_perm,
+                                                         const float* __restrict__ shared, int H, int k, int rows,
+                                                         __nv_bfloat16* __restrict__ y, DevStatus* st) {
+  const int t = blockIdx.x;
+  __shared__ int32_t srow[64];
+  __shared__ float sw[64];
+  __shared__ int bad;
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  for (int j = threadIdx.x; j < k; j += blockDim.x) {
+    const int r = inv_perm[(size_t)t * k + j];
+    if (r < 0 || r >= rows) {
+      raise_error(st, MOE_ERR_DEVICE_BOUNDS, SITE_COMBINE, t);
+      bad = 1;
+    }
+    srow[j] = r;
+    sw[j] = w[(size_t)t * k + j];
+  }
+  __syncthreads();
+  if (bad) return;
+  const int H4 = H >> 2;
+  for (int c = threadIdx.x; c < H4; c += blockDim.x) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+      const float4 v = __ldcs(reinterpret_cast<const float4*>(o + (size_t)srow[j] * H) + c);
+      const float wj = sw[j];
+      acc.x = fmaf(wj, v.x, acc.x);
+      acc.y = fmaf(wj, v.y, acc.y);
+      acc.z = fmaf(wj, v.z, acc.z);
+      acc.w = fmaf(wj, v.w, acc.w);
+    }
+    if (shared) {
+      const float4 s = __ldcs(reinterpret_cast<const float4*>(shared + (size_t)t * H) + c);
+      acc.x += s.x;
+      acc.y += s.y;
+      acc.z += s.z;
+      acc.w += s.w;
+    }
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 packed;
+    packed.x = *reinterpret_cast<uint32_t*>(&lo);
+    packed.y = *reinterpret_cast<uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(y + (size_t)t * H)[c] = packed;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const float* o, const float* topk_w, const int32_t* inv_perm, const float* shared, int T,
+                           int H, int k, int rows, uint16_t* y, DevStatus* st, cudaStream_t s) {
+  if (k > 64) return cudaErrorInvalidValue;
+  combine_kernel<<<T, kThreads, 0, s>>>(o, topk_w, inv_perm, shared, H, k, rows,
+                                        reinterpret_cast<__nv_bfloat16*>(y), st);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

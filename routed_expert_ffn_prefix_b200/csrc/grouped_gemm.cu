@@ -1,0 +1,362 @@
+// grouped_gemm.cu -- persistent grouped GEMM on tcgen05/TMEM for the MoE expert FFN.
+//
+// Both expert GEMMs of the layer (gate/up with the SwiGLU epilogue, and
+// down) and the tensor-core router run through this kernel.  It follows
+// the grouped matmul of the Qwen 3.5-397B-on-Ironwood page (sec. 4.2,
+// "grouped GEMM V2 with fused activation": SwiGLU inside the matmul, ragged
+// per-expert row counts with minimal padding, token rows gathered straight
+// from HBM with no padded permuted copy), re-designed for sm_100a:
+//
+//   * Orientation: the weight columns are the MMA's M side (128 per MMA
+//     tile) and the expert's token rows are the N side (16..256).  An
+//     expert's weight tile is therefore streamed from HBM once and applied
+//     to every row routed to it, whatever the row count -- the layer is
+//     bound by streaming the activated experts' weights, and decode-sized
+//     groups of 1..30 rows need no padding to 128.
+//   * A work unit = (group, column block, row pass).  A column block holds
+//     two 128-column MMA tiles sharing the same token rows: for gate/up they
+//     are the gate and the up columns of the same 128 intermediate units,
+//     so SwiGLU is computed in the epilogue from two TMEM accumulators; for
+//     down they are 256 adjacent output columns.
+//   * Weight tiles arrive by TMA (128-byte swizzle, MN-major operand), token
+//     rows by cp.async 16-byte gathers written in the same swizzle (K-major
+//     operand), both into a multi-stage shared-memory ring guarded by
+//     mbarriers.  One thread issues tcgen05.mma into TMEM; four epilogue
+//     warps drain TMEM with tcgen05.ld.  Accumulators are double-buffered in
+//     TMEM when they fit, so a unit's epilogue overlaps the next unit's MMAs.
+//   * Every wait is bounded (see common.cuh); routing metadata is range
+//     checked before it is used as an address.
+//
+// Warp roles (288 threads): warps 0-3 epilogue, warps 4-7 producers,
+// warp 8 TMEM allocation + MMA issue.
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 288;
+constexpr int kATileBytes = 128 * 64 * 2;  // 128 weight columns x 64 k, bf16
+constexpr int kBK = 64;                    // k per pipeline stage (one 128-byte swizzle row)
+
+template <int NT, int ST>
+struct Cfg {
+  static constexpr int B_BYTES = NT * kBK * 2;
+  static constexpr int STAGE_BYTES = 2 * kATileBytes + B_BYTES;
+  static constexpr int NBUF = (4 * NT <= 512) ? 2 : 1;
+  static constexpr int ACC_COLS = NBUF * 2 * NT;
+  static constexpr int TMEM_COLS = ACC_COLS <= 32 ? 32 : ACC_COLS <= 64 ? 64 : ACC_COLS <= 128 ? 128
+                                   : ACC_COLS <= 256 ? 256 : 512;
+  // ring + barriers/flags (256) + unit prefix (kMaxExperts+1 ints) + alignment slack
+  static constexpr int SMEM_BYTES = ST * STAGE_BYTES + 256 + 4 * (kMaxExperts + 1) + 1024;
+  static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "row pass must be 16..256, multiple of 16");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+struct Unit {
+  int group, nb, row0, rows;
+};
+
+__device__ __forceinline__ int group_rows_begin(const GemmArgs& a, int g) {
+  return a.offsets ? __ldg(a.offsets + g) : 0;
+}
+__device__ __forceinline__ int group_rows_end(const GemmArgs& a, int g) {
+  return a.offsets ? __ldg(a.offsets + g + 1) : a.single_rows;
+}
+
+template <int NT>
+__device__ __forceinline__ Unit decode_unit(const GemmArgs& a, const int* ustart, int ngroups, int u) {
+  int lo = 0, hi = ngroups - 1;  // last group with ustart[g] <= u
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (ustart[mid] <= u) lo = mid; else hi = mid - 1;
+  }
+  const int g = lo;
+  const int b = group_rows_begin(a, g), e = group_rows_end(a, g);
+  const int passes = (e - b + NT - 1) / NT;
+  const int local = u - ustart[g];
+  Unit r;
+  r.group = g;
+  r.nb = local / passes;
+  const int pass = local - r.nb * passes;
+  r.row0 = b + pass * NT;
+  r.rows = min(NT, e - r.row0);
+  return r;
+}
+
+// Warp 0: per-group unit counts -> exclusive prefix in shared memory, with
+// the row ranges checked.  Returns the total unit count (0 on bad metadata).
+template <int NT>
+__device__ void build_unit_prefix(const GemmArgs& a, int ngroups, int* ustart, int* total_out) {
+  const int lane = lane_id();
+  const int per = (ngroups + 31) / 32;
+  const int g0 = min(ngroups, lane * per), g1 = min(ngroups, g0 + per);
+  int sum = 0, bad = -1;
+  for (int g = g0; g < g1; ++g) {
+    const int b = group_rows_begin(a, g), e = group_rows_end(a, g);
+    if (b < 0 || e < b || e > a.rows_cap) bad = g;
+    ustart[g] = sum;
+    sum += (e > b && bad < 0) ? ((e - b + NT - 1) / NT) * a.n_blocks : 0;
+  }
+  int incl = sum;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += v;
+  }
+  const int base = incl - sum;
+  for (int g = g0; g < g1; ++g) ustart[g] += base;
+  const int any_bad = __reduce_max_sync(0xffffffffu, bad);
+  if (lane == 31) {
+    if (any_bad >= 0) {
+      raise_error(a.status, MOE_ERR_DEVICE_BOUNDS, SITE_GEMM_OFFSETS, any_bad);
+      *total_out = 0;
+    } else {
+      *total_out = incl;
+    }
+  }
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+
+template <int NT, int ST, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap wmap, const GemmArgs a) {
+  using C = Cfg<NT, ST>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * C::STAGE_BYTES);
+  uint64_t* empty = full + ST;
+  uint64_t* tfull = empty + ST;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int* total_units = abort_flag + 1;
+  int* ustart = reinterpret_cast<int*>(smem + ST * C::STAGE_BYTES + 256);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int ngroups = a.offsets ? a.groups : 1;
+
+  if (tid == 0) {
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(full + s, 128 + 1);  // 128 producer cp.async arrivals + 1 expect_tx arrival
+      mbar_init(empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull + b, 1);
+      mbar_init(tempty + b, 128);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) build_unit_prefix<NT>(a, ngroups, ustart, total_units);
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) prefetch_tmap(&wmap);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int total = *total_units;
+  const int kiters = (a.K / kBK) * a.krep;
+  const int kt_per_rep = a.K / kBK;
+
+  if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ producers
+    const WaitCtx wc{a.status, abort_flag, a.timeout_ns, SITE_GEMM_PRODUCER};
+    const int pt = tid - 128;
+    const int chunk = pt & 7, rsub = pt >> 3;
+    const uint64_t pol_w = policy_evict_first();
+    const __nv_bfloat16* bsrc = reinterpret_cast<const __nv_bfloat16*>(a.b_src);
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued_mask = 0, issued_par = 0;  // per stage: loads issued / parity of the last issue
+    bool ok = true;
+    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+      const Unit un = decode_unit<NT>(a, ustart, ngroups, u);
+      int src[NT / 16];
+#pragma unroll
+      for (int i = 0; i < NT / 16; ++i) {
+        const int c = rsub + 16 * i;
+        int s = -1;
+        if (c < un.rows) {
+          const int r = un.row0 + c;
+          s = a.row_index ? __ldg(a.row_index + r) : r;
+          if (s < 0 || s >= a.src_rows) {
+            raise_error(a.status, MOE_ERR_DEVICE_BOUNDS, SITE_GEMM_GATHER, r);
+            s = -1;
+          }
+        }
+        src[i] = s;
+      }
+      const int colA0 = un.nb * a.col_stride, colA1 = colA0 + a.col1_off;
+      for (int it = 0; it < kiters; ++it) {
+        const int rep = it / kt_per_rep, kt = it - rep * kt_per_rep;
+        if (!mbar_wait(&empty[stage], phase ^ 1u, wc, 100 + stage)) { ok = false; break; }
+        uint8_t* sA0 = smem + stage * C::STAGE_BYTES;
+        uint8_t* sA1 = sA0 + kATileBytes;
+        const uint32_t sB = smem_u32(sA0 + 2 * kATileBytes);
+#pragma unroll
+        for (int i = 0; i < NT / 16; ++i) {
+          if (src[i] >= 0) {
+            const int c = rsub + 16 * i;
+            cp_async_16(sB + c * 128 + ((chunk ^ (c & 7)) << 4),
+                        bsrc + (size_t)src[i] * a.K + kt * kBK + chunk * 8);
+          }
+        }
+        cp_async_arrive_noinc(&full[stage]);
+        if (pt == 0) {
+          mbar_arrive_expect_tx(&full[stage], 4 * (kATileBytes / 2));
+          const int d2 = a.a_dim2_rep ? rep : un.group;
+          const int k0 = kt * kBK;
+          tma_load_3d(sA0, &wmap, &full[stage], colA0, k0, d2, pol_w);
+          tma_load_3d(sA0 + kATileBytes / 2, &wmap, &full[stage], colA0 + 64, k0, d2, pol_w);
+          tma_load_3d(sA1, &wmap, &full[stage], colA1, k0, d2, pol_w);
+          tma_load_3d(sA1 + kATileBytes / 2, &wmap, &full[stage], colA1 + 64, k0, d2, pol_w);
+        }
+        issued_mask |= 1u << stage;
+        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == ST) { stage = 0; phase ^= 1u; }
+      }
+    }
+    cp_async_wait_all();
+    if (!ok && pt == 0) {
+      // Aborted: let every load still in flight land before the block exits.
+      const WaitCtx drain{nullptr, abort_flag, a.timeout_ns, SITE_GEMM_PRODUCER};
+      for (int s = 0; s < ST; ++s) {
+        if (!(issued_mask >> s & 1u)) continue;
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&full[s], (issued_par >> s) & 1u) && globaltimer_ns() - t0 < drain.timeout_ns) {
+        }
+      }
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const WaitCtx wc{a.status, abort_flag, a.timeout_ns, SITE_GEMM_MMA};
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc_it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+        const Unit un = decode_unit<NT>(a, ustart, ngroups, u);
+        const int buf = C::NBUF == 2 ? (acc_it & 1) : 0;
+        const uint32_t apar = C::NBUF == 2 ? ((acc_it >> 1) & 1) : (acc_it & 1);
+        if (!mbar_wait(&tempty[buf], apar ^ 1u, wc, 200 + buf)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem + buf * 2 * NT, d1 = d0 + NT;
+        const int N = (un.rows + 15) & ~15;
+        const uint32_t idesc = idesc_bf16_f32(128, N, /*A MN-major*/ true, /*B K-major*/ false);
+        uint32_t acc = 0;
+        for (int it = 0; it < kiters; ++it) {
+          if (!mbar_wait(&full[stage], phase, wc, 300 + stage)) { ok = false; break; }
+          tc_fence_after();
+          fence_proxy_async_smem();
+          const uint32_t sA0 = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sA1 = sA0 + kATileBytes, sB = sA0 + 2 * kATileBytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            // A (weights, MN-major): +16 k = two 8-row groups = 2048 B; the two
+            // 64-column halves sit 8192 B apart.  B (rows, K-major): +16 k = 32 B.
+            const uint64_t a0 = smem_desc_sw128(sA0 + kk * 2048, 8192, 1024);
+            const uint64_t a1 = smem_desc_sw128(sA1 + kk * 2048, 8192, 1024);
+            const uint64_t bd = smem_desc_sw128(sB + kk * 32, 16, 1024);
+            mma_bf16(d0, a0, bd, idesc, acc);
+            mma_bf16(d1, a1, bd, idesc, acc);
+            acc = 1;
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == ST) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(&tfull[buf]);
+        ++acc_it;
+      }
+      // Every MMA issued by this thread has finished once mma_done flips.
+      mma_commit(mma_done);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(mma_done, 0) && globaltimer_ns() - t0 < a.timeout_ns) {
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 0-3)
+    const WaitCtx wc{a.status, abort_flag, a.timeout_ns, SITE_GEMM_EPILOGUE};
+    int acc_it = 0;
+    for (int u = blockIdx.x; u < total; u += gridDim.x) {
+      const Unit un = decode_unit<NT>(a, ustart, ngroups, u);
+      const int buf = C::NBUF == 2 ? (acc_it & 1) : 0;
+      const uint32_t apar = C::NBUF == 2 ? ((acc_it >> 1) & 1) : (acc_it & 1);
+      if (!mbar_wait(&tfull[buf], apar, wc, 400 + buf)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + buf * 2 * NT;
+      const int col = un.nb * a.out_col_stride + warp * 32 + lane;
+      for (int c0 = 0; c0 < un.rows; c0 += 16) {
+        float v0[16], v1[16];
+        tmem_ld_2x16(tbase + c0, tbase + NT + c0, v0, v1);
+        const int nr = min(16, un.rows - c0);
+        if (EPI == EPI_SWIGLU) {
+          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+          if (col < a.n_valid) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              if (j < nr) {
+                const float hv = silu_f(v0[j]) * v1[j];
+                out[(size_t)(un.row0 + c0 + j) * a.ld_out + col] = __float2bfloat16_rn(hv);
+              }
+            }
+          }
+        } else {
+          float* out = reinterpret_cast<float*>(a.out);
+          const bool ok0 = col < a.n_valid, ok1 = col + a.out_col1_off < a.n_valid;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (j < nr) {
+              float* orow = out + (size_t)(un.row0 + c0 + j) * a.ld_out;
+              if (ok0) orow[col] = v0[j];
+              if (ok1) orow[col + a.out_col1_off] = v1[j];
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[buf]);
+      ++acc_it;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int NT, int ST, int EPI>
+cudaError_t launch_cfg(const CUtensorMap& wmap, const GemmArgs& a, int num_sms, cudaStream_t stream) {
+  using C = Cfg<NT, ST>;
+  auto kern = grouped_gemm_kernel<NT, ST, EPI>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (err != cudaSuccess) return err;
+  kern<<<num_sms, kThreads, C::SMEM_BYTES, stream>>>(wmap, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_gemm(const CUtensorMap& wmap, const GemmArgs& a, int epilogue, int tiles, int num_sms,
+                                cudaStream_t stream) {
+  if (tiles == MOE_TILES_LARGE) {
+    return epilogue == EPI_SWIGLU ? launch_cfg<256, 3, EPI_SWIGLU>(wmap, a, num_sms, stream)
+                                  : launch_cfg<256, 3, EPI_STORE_F32>(wmap, a, num_sms, stream);
+  }
+  return epilogue == EPI_SWIGLU ? launch_cfg<64, 5, EPI_SWIGLU>(wmap, a, num_sms, stream)
+                                : launch_cfg<64, 5, EPI_STORE_F32>(wmap, a, num_sms, stream);
+}
+
+}  // namespace moe

@@ -1,0 +1,64 @@
+// kernels.h -- host-side launchers of the MoE kernels (internal to the library).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kMaxExperts = 1024;
+
+// Arguments of the grouped GEMM (see grouped_gemm.cu).  "Rows" are token
+// rows (the MMA's N side); "columns" are weight columns (the MMA's M side).
+struct GemmArgs {
+  const int32_t* offsets;  // [groups+1] row ranges per group, or nullptr: one group of single_rows rows
+  const int32_t* row_index;  // permuted row -> source row of b_src (gather), or nullptr: identity
+  const uint16_t* b_src;     // [src_rows, K] bf16, K contiguous
+  int src_rows;
+  int groups;
+  int single_rows;
+  int K;            // reduction length, multiple of 64
+  int krep;         // repeats of the K loop (weight planes summed into one accumulator)
+  int a_dim2_rep;   // 1: weight tile's 3rd coordinate is the repeat index; 0: the group index
+  int n_blocks;     // column blocks per group (each = two 128-column MMA tiles)
+  int col_stride;   // first weight column of block nb = nb * col_stride
+  int col1_off;     // second MMA tile's columns start col1_off after the first
+  void* out;
+  int ld_out;          // output row stride (elements)
+  int out_col_stride;  // output column of block nb = nb * out_col_stride (+ lane)
+  int out_col1_off;    // store epilogue: second tile's output columns offset
+  int n_valid;         // output columns < n_valid are written
+  int rows_cap;        // offsets[groups] may not exceed this (rows of out / row_index)
+  DevStatus* status;
+  uint64_t timeout_ns;
+};
+
+enum Epilogue { EPI_SWIGLU = 0, EPI_STORE_F32 = 1 };
+
+// tiles: MOE_TILES_SMALL or MOE_TILES_LARGE.
+cudaError_t launch_grouped_gemm(const CUtensorMap& wmap, const GemmArgs& a, int epilogue, int tiles,
+                                int num_sms, cudaStream_t stream);
+
+// Router.
+cudaError_t launch_router_split(const float* w, int H, int E, uint16_t* planes, cudaStream_t s);
+cudaError_t launch_router_logits_fma(const uint16_t* x, const float* w, int T, int H, int E, float* logits,
+                                     cudaStream_t s);
+cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, int32_t* ids, float* w,
+                        DevStatus* st, cudaStream_t s);
+
+// Permutation.
+int permute_num_blocks(int T, int k);
+cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* counts, int32_t* offsets,
+                           int32_t* sorted_ids, int32_t* inv_perm, int32_t* block_hist, DevStatus* st,
+                           cudaStream_t s);
+
+// Combine.
+cudaError_t launch_combine(const float* o, const float* topk_w, const int32_t* inv_perm, const float* shared,
+                           int T, int H, int k, int rows, uint16_t* y, DevStatus* st, cudaStream_t s);
+
+cudaError_t launch_selftest_timeout(DevStatus* st, uint64_t timeout_ns, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,149 @@
+// permute.cu -- routing metadata: per-expert counts, offsets, the permutation
+// of slots (t, j) into expert-contiguous order and its inverse.
+//
+// The pages gather each expert's token rows into a contiguous buffer from
+// the routing indices and handle each expert's variable row count with
+// minimal padding (Qwen 3.5-397B-on-Ironwood page, sec. 4.2); the gathered
+// order must later be undone to bring results back to token order
+// (same page, sec. 7.2).  Here the order is fixed: experts ascending, and
+// within an expert the slots in ascending flattened index s = t*k + j
+// (token ascending), so the permutation is deterministic and can be
+// checked bit for bit.  Atomics would make positions run-dependent; instead:
+//
+//   1. hist:    block b counts the expert ids of its chunk of slots.
+//   2. scan:    one block turns the [blocks, E] counts into per-(block,
+//               expert) starting rows (column scan over blocks, then an
+//               exclusive scan over experts), and writes counts/offsets.
+//   3. scatter: one warp per chunk walks its slots in order, 32 at a time;
+//               lanes with the same expert are ranked by __match_any_sync, so
+//               each slot's row = start[b][e] + earlier slots of e in the chunk.
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kChunk = 256;  // slots per block (hist/scatter)
+
+__global__ void hist_kernel(const int32_t* __restrict__ ids, int n, int E, int32_t* __restrict__ block_hist,
+                            DevStatus* st) {
+  extern __shared__ int32_t h[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
+  __syncthreads();
+  const int s0 = blockIdx.x * kChunk;
+  for (int i = threadIdx.x; i < kChunk; i += blockDim.x) {
+    const int s = s0 + i;
+    if (s < n) {
+      const int e = ids[s];
+      if (e < 0 || e >= E) {
+        raise_error(st, MOE_ERR_DEVICE_BOUNDS, SITE_PERMUTE_IDS, s);
+      } else {
+        atomicAdd(&h[e], 1);
+      }
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) block_hist[(size_t)blockIdx.x * E + e] = h[e];
+}
+
+// Single block of 1024 threads.
+__global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ block_hist, int nblk, int E,
+                                                    int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+  __shared__ int32_t tot[kMaxExperts];
+  __shared__ int32_t warp_sums[32];
+  const int tid = threadIdx.x;
+  // column scan over blocks: block_hist[b][e] <- rows of e in blocks < b
+  for (int e = tid; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int b = 0; b < nblk; ++b) {
+      const int v = block_hist[(size_t)b * E + e];
+      block_hist[(size_t)b * E + e] = run;
+      run += v;
+    }
+    tot[e] = run;
+    counts[e] = run;
+  }
+  __syncthreads();
+  // exclusive scan of tot over experts (E <= 1024 = blockDim)
+  const int v = tid < E ? tot[tid] : 0;
+  int incl = v;
+  const int lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += o;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int ws = warp_sums[lane];
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, ws, d);
+      if (lane >= d) ws += o;
+    }
+    warp_sums[lane] = ws;  // inclusive over warps
+  }
+  __syncthreads();
+  const int excl = incl - v + (warp > 0 ? warp_sums[warp - 1] : 0);
+  if (tid < E) offsets[tid] = excl;
+  if (tid == E - 1) offsets[E] = excl + v;
+  __syncthreads();
+  if (tid < E) tot[tid] = excl;
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    const int base = tot[e];
+    for (int b = 0; b < nblk; ++b) block_hist[(size_t)b * E + e] += base;
+  }
+}
+
+// One warp per block.
+__global__ void __launch_bounds__(32) scatter_kernel(const int32_t* __restrict__ ids, int n, int E, int k,
+                                                   const int32_t* __restrict__ block_hist,
+                                                   int32_t* __restrict__ sorted_ids,
+                                                   int32_t* __restrict__ inv_perm) {
+  extern __shared__ int32_t run[];
+  const int lane = threadIdx.x;
+  for (int e = lane; e < E; e += 32) run[e] = block_hist[(size_t)blockIdx.x * E + e];
+  __syncwarp();
+  const int s0 = blockIdx.x * kChunk;
+  for (int r = 0; r < kChunk; r += 32) {
+    const int s = s0 + r + lane;
+    const bool valid = s < n;
+    int e = valid ? ids[s] : -1;
+    if (e >= E) e = -1;  // out-of-range ids were reported by hist_kernel; skip them here
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    int pos = -1;
+    if (e >= 0) pos = run[e] + rank;
+    __syncwarp();
+    if (e >= 0 && rank == 0) run[e] += __popc(peers);
+    __syncwarp();
+    if (e >= 0) {
+      sorted_ids[pos] = s / k;
+      inv_perm[s] = pos;
+    }
+  }
+}
+
+}  // namespace
+
+int permute_num_blocks(int T, int k) { return (T * k + kChunk - 1) / kChunk; }
+
+cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* counts, int32_t* offsets,
+                           int32_t* sorted_ids, int32_t* inv_perm, int32_t* block_hist, DevStatus* st,
+                           cudaStream_t s) {
+  const int n = T * k;
+  const int nblk = permute_num_blocks(T, k);
+  const size_t sh = (size_t)E * sizeof(int32_t);
+  hist_kernel<<<nblk, 256, sh, s>>>(ids, n, E, block_hist, st);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  scan_kernel<<<1, 1024, 0, s>>>(block_hist, nblk, E, counts, offsets);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  scatter_kernel<<<nblk, 32, sh, s>>>(ids, n, E, k, block_hist, sorted_ids, inv_perm);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,234 @@
+"""GPU parity of every stage and of the whole layer against the CPU oracle,
+at sizes the oracle finishes in seconds: several tiles per expert, ragged
+per-expert row counts, empty experts, one token, k = E, a shared expert,
+experts with more rows than one tile pass, and both tile policies and both
+router implementations.  Routing (ids, counts, offsets, permutation) must
+match bit for bit; floating-point outputs within the layer's tolerance."""
+import numpy as np
+import pytest
+
+import oracle
+import routed_expert_ffn_prefix_b200 as moe
+import synth
+from synth import Config
+
+from helpers import (W_ABS, assert_close_output, dev_bf16, dev_f32, dev_i32, host_f64)
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    c.name: c for c in [
+        synth.CONFIGS["tiny"],
+        Config("ragged", T=300, H=512, E=16, I=256, k=3),          # ragged counts, tails not /16
+        Config("multipass", T=700, H=256, E=4, I=128, k=2),        # ~350 rows/expert: several row passes
+        Config("shared_zipf", T=200, H=512, E=8, I=256, k=2, I_s=256, bias="zipf:1.2"),
+        Config("k_eq_E", T=33, H=256, E=4, I=128, k=4),
+        Config("one_token", T=1, H=512, E=16, I=256, k=4),
+        Config("sparse", T=5, H=256, E=64, I=128, k=2),            # most experts empty
+        Config("wide", T=96, H=1024, E=32, I=384, k=6, I_s=128),   # I not a power of two
+    ]
+}
+
+_cache = {}
+
+
+def case(name):
+    if name not in _cache:
+        cfg = CASES[name]
+        inp = synth.make_inputs(cfg)
+        oracle.enforce_logit_gap(inp)
+        ref = oracle.layer_forward(inp.x, inp.w_router, inp.bias, inp.w_gate_up, inp.w_down, cfg.k,
+                                   inp.w_sh_gate_up, inp.w_sh_down)
+        _cache[name] = (cfg, inp, ref)
+    return _cache[name]
+
+
+def dev_inputs(inp):
+    d = dict(x=dev_bf16(inp.x), w_router=dev_f32(inp.w_router),
+             bias=None if inp.bias is None else dev_f32(inp.bias),
+             w_gate_up=dev_bf16(inp.w_gate_up), w_down=dev_bf16(inp.w_down))
+    d["w_sh_gate_up"] = None if inp.w_sh_gate_up is None else dev_bf16(inp.w_sh_gate_up)
+    d["w_sh_down"] = None if inp.w_sh_down is None else dev_bf16(inp.w_sh_down)
+    return d
+
+
+def workspace(cfg):
+    return moe.alloc_workspace(cfg.T, cfg.H, cfg.E, cfg.I, cfg.k, cfg.I_s)
+
+
+def assert_ok(ws):
+    st = moe.device_status(ws)
+    assert st == 0, moe.STATUS.get(st, st)
+
+
+@pytest.mark.parametrize("impl", [moe.ROUTER_FMA, moe.ROUTER_TC])
+@pytest.mark.parametrize("name", list(CASES))
+def test_route_matches_oracle(name, impl):
+    cfg, inp, ref = case(name)
+    if impl == moe.ROUTER_TC and cfg.E % 8:
+        pytest.skip("tensor-core router needs E % 8 == 0")
+    d = dev_inputs(inp)
+    ws = workspace(cfg)
+    ids, w = moe.route(d["x"], d["w_router"], d["bias"], cfg.k, ws, impl=impl)
+    assert_ok(ws)
+    np.testing.assert_array_equal(ids.cpu().numpy(), ref["ids"])
+    wg = host_f64(w)
+    assert np.abs(wg - ref["w"]).max() <= W_ABS
+    assert np.abs(wg.sum(1) - 1).max() <= 1e-6
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_permute_bit_exact(name):
+    cfg, inp, ref = case(name)
+    ws = workspace(cfg)
+    counts, offsets, sids, inv = moe.permute(dev_i32(ref["ids"]), cfg.E, ws)
+    assert_ok(ws)
+    np.testing.assert_array_equal(counts.cpu().numpy(), ref["counts"])
+    np.testing.assert_array_equal(offsets.cpu().numpy(), ref["offsets"])
+    np.testing.assert_array_equal(sids.cpu().numpy(), ref["sorted_token_ids"])
+    np.testing.assert_array_equal(inv.cpu().numpy(), ref["inv_perm"])
+
+
+def test_permute_random_ids_large():
+    """81,920 slots (the prefill shape's permuted row count) over 512 experts."""
+    rng = np.random.default_rng(3)
+    T, E, k = 8192, 512, 10
+    ids = np.argsort(rng.random((T, E)), axis=1)[:, :k].astype(np.int32)
+    want = oracle.permute(ids, E)
+    ws = moe.alloc_workspace(T, 256, E, 128, k)
+    got = moe.permute(dev_i32(ids), E, ws)
+    assert_ok(ws)
+    for g, w in zip(got, want):
+        np.testing.assert_array_equal(g.cpu().numpy().reshape(w.shape), w)
+
+
+@pytest.mark.parametrize("tiles", [moe.TILES_SMALL, moe.TILES_LARGE])
+@pytest.mark.parametrize("name", list(CASES))
+def test_grouped_swiglu_matches_oracle(name, tiles):
+    cfg, inp, ref = case(name)
+    d = dev_inputs(inp)
+    ws = workspace(cfg)
+    h = moe.grouped_swiglu(d["x"], d["w_gate_up"], dev_i32(ref["offsets"]), dev_i32(ref["sorted_token_ids"]),
+                           cfg.k, ws, tiles=tiles)
+    assert_ok(ws)
+    assert_close_output(host_f64(h), ref["h"], "h")
+
+
+@pytest.mark.parametrize("tiles", [moe.TILES_SMALL, moe.TILES_LARGE])
+@pytest.mark.parametrize("name", list(CASES))
+def test_down_combine_matches_oracle(name, tiles):
+    """Fed a synthetic h (not the GPU's): y = sum_j w o[inv_perm] + shared."""
+    cfg, inp, ref = case(name)
+    R = cfg.T * cfg.k
+    h_bits = synth.normal_bf16(cfg.seed, synth.TID["h_stage"], 0, (R, cfg.I), 0.5)
+    shared = synth.normal_f32(cfg.seed, synth.TID["misc"], 1, (cfg.T, cfg.H), 0.1) if cfg.I_s else None
+    ws = workspace(cfg)
+    y = moe.down_combine(dev_bf16(h_bits), dev_bf16(inp.w_down), dev_f32(ref["w"]), dev_i32(ref["inv_perm"]),
+                         dev_i32(ref["offsets"]), None if shared is None else dev_f32(shared), ws, tiles=tiles)
+    assert_ok(ws)
+    want = oracle.down_combine(oracle.bf16_to_f64(h_bits), ref["offsets"], ref["inv_perm"], ref["w"],
+                               lambda e: inp.w_down[e], None if shared is None else shared.astype(np.float64))
+    assert_close_output(host_f64(y), want)
+
+
+def test_grouped_down_single_group():
+    cfg = CASES["wide"]
+    rng_bits = synth.normal_bf16(1, synth.TID["misc"], 2, (77, cfg.I), 0.5)
+    w = synth.normal_bf16(1, synth.TID["misc"], 3, (1, cfg.I, cfg.H), 0.05)
+    ws = workspace(cfg)
+    o = moe.grouped_down(dev_bf16(rng_bits), dev_bf16(w), None, ws)
+    assert_ok(ws)
+    want = oracle.bf16_to_f64(rng_bits) @ oracle.bf16_to_f64(w[0])
+    assert_close_output(host_f64(o), want, "o")
+
+
+@pytest.mark.parametrize("router", [moe.ROUTER_FMA, moe.ROUTER_TC])
+@pytest.mark.parametrize("tiles", [moe.TILES_SMALL, moe.TILES_LARGE])
+@pytest.mark.parametrize("name", list(CASES))
+def test_forward_matches_oracle(name, tiles, router):
+    cfg, inp, ref = case(name)
+    if router == moe.ROUTER_TC and cfg.E % 8:
+        pytest.skip("tensor-core router needs E % 8 == 0")
+    d = dev_inputs(inp)
+    ws = workspace(cfg)
+    y = moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws,
+                    d["w_sh_gate_up"], d["w_sh_down"], tiles=tiles, router=router)
+    assert_ok(ws)
+    v = moe.workspace_view(ws, cfg.T, cfg.H, cfg.E, cfg.I, cfg.k, cfg.I_s)
+    np.testing.assert_array_equal(v["topk_ids"].cpu().numpy(), ref["ids"])
+    np.testing.assert_array_equal(v["counts"].cpu().numpy(), ref["counts"])
+    np.testing.assert_array_equal(v["offsets"].cpu().numpy(), ref["offsets"])
+    np.testing.assert_array_equal(v["sorted_token_ids"].cpu().numpy(), ref["sorted_token_ids"])
+    np.testing.assert_array_equal(v["inv_perm"].cpu().numpy(), ref["inv_perm"])
+    assert_close_output(host_f64(y), ref["y"])
+
+
+def test_forward_bitwise_deterministic():
+    """The combine sums each token's slots in a fixed order: repeated runs
+    (with other work in between) give identical bits."""
+    import torch
+    cfg, inp, ref = case("ragged")
+    d = dev_inputs(inp)
+    ws = workspace(cfg)
+    ys = []
+    for _ in range(3):
+        ys.append(moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws,
+                              tiles=moe.TILES_LARGE).cpu())
+        moe.forward(d["x"][:7], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k,
+                    moe.alloc_workspace(7, cfg.H, cfg.E, cfg.I, cfg.k))
+    assert_ok(ws)
+    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[0], ys[2])
+
+
+def test_all_tokens_to_the_same_experts():
+    """A bias far above the logits' spread sends every token to experts 0..k-1."""
+    cfg = Config("hot", T=300, H=256, E=8, I=128, k=2)
+    inp = synth.make_inputs(cfg)
+    inp.bias = np.array([30.0, 20.0] + [0.0] * 6, np.float32)
+    ref = oracle.layer_forward(inp.x, inp.w_router, inp.bias, inp.w_gate_up, inp.w_down, cfg.k)
+    assert ref["counts"].tolist() == [300, 300, 0, 0, 0, 0, 0, 0]
+    d = dev_inputs(inp)
+    for tiles in (moe.TILES_SMALL, moe.TILES_LARGE):
+        ws = workspace(cfg)
+        y = moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws, tiles=tiles)
+        assert_ok(ws)
+        assert_close_output(host_f64(y), ref["y"])
+
+
+# ---------------------------------------------------------------- failure detection (no GPU fault)
+
+def test_bounded_wait_times_out_and_context_stays_usable():
+    cfg, inp, ref = case("tiny")
+    ws = workspace(cfg)
+    moe.selftest_timeout(ws, 50_000_000)  # 50 ms on a barrier nothing completes
+    assert moe.device_status(ws) == 5     # MOE_ERR_DEVICE_TIMEOUT
+    moe.clear_device_status(ws)
+    d = dev_inputs(inp)
+    y = moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws)
+    assert_ok(ws)
+    assert_close_output(host_f64(y), ref["y"])
+
+
+def test_corrupt_offsets_are_reported_not_followed():
+    cfg, inp, ref = case("ragged")
+    d = dev_inputs(inp)
+    ws = workspace(cfg)
+    bad = ref["offsets"].copy()
+    bad[5] = cfg.T * cfg.k + 1000  # past the end of h and of sorted_token_ids
+    h = moe.grouped_swiglu(d["x"], d["w_gate_up"], dev_i32(bad), dev_i32(ref["sorted_token_ids"]), cfg.k, ws)
+    assert moe.device_status(ws) == 7  # MOE_ERR_DEVICE_BOUNDS
+    moe.clear_device_status(ws)
+    bad_ids = ref["sorted_token_ids"].copy()
+    bad_ids[7] = cfg.T + 5  # a token that does not exist
+    moe.grouped_swiglu(d["x"], d["w_gate_up"], dev_i32(ref["offsets"]), dev_i32(bad_ids), cfg.k, ws, out=h)
+    assert moe.device_status(ws) == 7
+    moe.clear_device_status(ws)
+    ids = ref["ids"].copy()
+    ids[3, 1] = cfg.E + 2
+    moe.permute(dev_i32(ids), cfg.E, ws)
+    assert moe.device_status(ws) == 7
+    moe.clear_device_status(ws)
+    # the library still works afterwards
+    y = moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws)
+    assert_ok(ws)
+    assert_close_output(host_f64(y), ref["y"])
