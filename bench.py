@@ -212,6 +212,10 @@ def time_workload(cfg, d, ws, steps, warmup, rank, world, flush, moe, gpu_index,
     if st != 0:
         raise RuntimeError(f"device status {moe.STATUS.get(st, st)} after warm-up")
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(steps)]
+    for row in evs:  # torch creates an event on its first record; the library re-records the same handle
+        for ev in row:
+            ev.record()
+    torch.cuda.synchronize()
     info = {}
     if world > 1:
         dist.barrier()
