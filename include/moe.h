@@ -139,6 +139,27 @@ moe_status_t moe_permute(const int32_t *topk_ids, int T, int E, int k,
                          int32_t *sorted_token_ids, int32_t *inv_perm,
                          void *workspace, size_t workspace_bytes, void *stream);
 
+/* moe_permute without a workspace.  The source pages have no counterpart to
+ * this call; it exists for callers that cannot allocate device memory when
+ * they call -- a serving loop that reserves all memory at start-up and
+ * forbids allocation afterwards, a plugin inside a framework that owns every
+ * device allocation, or code that must avoid the device-wide
+ * synchronisation cudaMalloc/cudaFree can cause.  The outputs are identical
+ * to moe_permute's.  The kernels' scratch lives in a 2 MiB array built into
+ * the library, which every GPU that loads the library holds until the
+ * process exits; the call itself allocates and frees nothing.
+ * Limits: T*k <= 131072 and E <= 1024 (larger sizes return
+ * MOE_ERR_WORKSPACE and enqueue nothing).
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * All calls share the one array: calls that overlap on the GPU (other
+ * streams, other host threads) race and must be serialised by the caller.
+ * No device status word is kept: an id outside [0,E) is skipped, so
+ * offsets[E] then falls short of T*k. */
+moe_status_t moe_permute_noalloc(const int32_t *topk_ids, int T, int E, int k,
+                                 int32_t *counts, int32_t *offsets,
+                                 int32_t *sorted_token_ids, int32_t *inv_perm, void *stream);
+
 /* Grouped gate/up GEMM with SwiGLU: for every permuted row r in
  * [offsets[e], offsets[e+1]), h[r, :] = bf16(silu(g) * u) with
  * [g | u] = x[sorted_token_ids[r], :] . W_gate_up[e]  (W_gate_up [E, H, 2I],
