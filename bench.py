@@ -400,7 +400,8 @@ def run_ours(args):
             "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "I": cfg.I, "k": cfg.k,
                        "I_s": cfg.I_s, "bias": cfg.bias, "seed": cfg.seed,
                        "parallelism": f"replicas x{world} (no collective in the layer)",
-                       "l2": "flushed (256 MiB write) before every timed step; expert weights 12.9 GB >> L2"},
+                       "l2": "flushed (256 MiB write) before every timed step; expert weights "
+                             f"{synth.expert_weight_bytes(cfg) / 1e9:.1f} GB > 126 MB L2"},
             **out_main,
             "e2e": {k: (round(v, 1) if isinstance(v, float) else v) for k, v in e2e.items()},
             "gpu_launches": main["launches"],

@@ -88,6 +88,13 @@ CONFIGS: dict[str, Config] = {
         *[Config(f"sweep_decode_t{t}", T=t, H=4096, E=256, I=1536, k=8,
                  note="small-batch decode sweep: few experts active, pure weight streaming")
           for t in (1, 4, 16, 64)],
+        # Reduced expert counts with the per-expert row counts of the decode
+        # (~10 rows) and prefill (~160 rows) shapes: 1.6 GB of weights, larger
+        # than L2 but small enough for multi-pass profiler captures.
+        Config("prof_decode_e64", T=64, H=4096, E=64, I=1024, k=10,
+               note="profiling case: decode-like rows per expert, 64 experts"),
+        Config("prof_prefill_e64", T=1024, H=4096, E=64, I=1024, k=10,
+               note="profiling case: prefill-like rows per expert, 64 experts"),
     ]
 }
 
