@@ -12,6 +12,30 @@ constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded device
 constexpr int kMaxK = 64;
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+constexpr int kPrefetchSteps = 8;  // weight tiles prefetched into L2 this many ring steps ahead
+
+// Tensor-core router tiling: row tiles of 256 tokens from T >= 2048, else 64;
+// the K range (H) is split so that about two work units land on each of the
+// 148 SMs.  A function of the shapes only, so the workspace layout and the
+// launch always agree.
+// MOE_ROUTER_AUTO: tensor cores whenever the 16-byte row pitch of the split
+// planes allows it (E % 8 == 0), else fp32 CUDA cores.
+inline int resolve_router(int impl, int E) {
+  if (impl != MOE_ROUTER_AUTO) return impl;
+  return E % 8 == 0 ? MOE_ROUTER_TC : MOE_ROUTER_FMA;
+}
+
+inline int router_tiles(int T) { return T >= 2048 ? MOE_TILES_LARGE : MOE_TILES_SMALL; }
+inline int router_splits(int T, int H, int E) {
+  const int nt = router_tiles(T) == MOE_TILES_LARGE ? 256 : 64;
+  const int base = ((T + nt - 1) / nt) * ((E + 255) / 256);
+  int s = (296 + base - 1) / base;
+  const int nkt = H / 64;
+  if (s > nkt) s = nkt;
+  if (s > 32) s = 32;
+  return s < 1 ? 1 : s;
+}
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // ---------------------------------------------------------------- workspace
@@ -32,7 +56,7 @@ moe_workspace_layout_t make_layout(int T, int H, int E, int I, int k, int I_s) {
   L.sorted_token_ids = take(tk * 4);
   L.inv_perm = take(tk * 4);
   L.block_hist = take((size_t)permute_num_blocks(T, k) * E * 4);
-  L.logits = take((size_t)T * E * 4);
+  L.logits = take((size_t)(H > 0 ? router_splits(T, H, E) : 1) * T * E * 4);
   L.router_split = take((size_t)3 * H * E * 2);
   L.h = take(tk * I * 2);
   L.o = take(tk * H * 4);
@@ -142,13 +166,15 @@ moe_status_t run_route(const uint16_t* x, const float* w_router, const float* bi
                        const DeviceInfo& dev, cudaStream_t s) {
   DevStatus* st = status_of(ws);
   float* logits = at<float>(ws, L.logits);
-  if (impl == MOE_ROUTER_AUTO) impl = (T >= 1024 && E % 8 == 0) ? MOE_ROUTER_TC : MOE_ROUTER_FMA;
+  impl = resolve_router(impl, E);
+  int nsplit = 1;
   if (impl == MOE_ROUTER_TC) {
     if (E % 8 != 0) return MOE_ERR_ALIGNMENT;
     uint16_t* planes = at<uint16_t>(ws, L.router_split);
     MOE_TRY(cuda_status(launch_router_split(w_router, H, E, planes, s)));
     CUtensorMap map;
     if (!make_weight_map(&map, planes, (uint64_t)E, (uint64_t)H, 3)) return MOE_ERR_CUDA;
+    nsplit = router_splits(T, H, E);
     GemmArgs a{};
     a.offsets = nullptr;
     a.row_index = nullptr;
@@ -168,14 +194,16 @@ moe_status_t run_route(const uint16_t* x, const float* w_router, const float* bi
     a.out_col1_off = 128;
     a.n_valid = E;
     a.rows_cap = T;
+    a.k_splits = nsplit;
+    a.split_stride = (size_t)T * E;
+    a.prefetch_steps = kPrefetchSteps;
     a.status = st;
     a.timeout_ns = kDefaultTimeoutNs;
-    const int tiles = T >= 2048 ? MOE_TILES_LARGE : MOE_TILES_SMALL;
-    MOE_TRY(cuda_status(launch_grouped_gemm(map, a, EPI_STORE_F32, tiles, dev.num_sms, s)));
+    MOE_TRY(cuda_status(launch_grouped_gemm(map, a, EPI_STORE_F32, router_tiles(T), dev.num_sms, s)));
   } else {
     MOE_TRY(cuda_status(launch_router_logits_fma(x, w_router, T, H, E, logits, s)));
   }
-  return cuda_status(launch_topk(logits, bias, T, E, k, ids, w, st, s));
+  return cuda_status(launch_topk(logits, nsplit, (size_t)T * E, bias, T, E, k, ids, w, st, s));
 }
 
 moe_status_t run_swiglu(const uint16_t* x, int src_rows, const uint16_t* w_gate_up, const int32_t* offsets,
@@ -202,6 +230,9 @@ moe_status_t run_swiglu(const uint16_t* x, int src_rows, const uint16_t* w_gate_
   a.out_col1_off = 0;
   a.n_valid = I;
   a.rows_cap = rows;
+  a.k_splits = 1;
+  a.split_stride = 0;
+  a.prefetch_steps = kPrefetchSteps;
   a.status = st;
   a.timeout_ns = kDefaultTimeoutNs;
   return cuda_status(launch_grouped_gemm(map, a, EPI_SWIGLU, tiles, dev.num_sms, s));
@@ -230,6 +261,9 @@ moe_status_t run_down(const uint16_t* h, const uint16_t* w_down, const int32_t* 
   a.out_col1_off = 128;
   a.n_valid = H;
   a.rows_cap = rows;
+  a.k_splits = 1;
+  a.split_stride = 0;
+  a.prefetch_steps = kPrefetchSteps;
   a.status = st;
   a.timeout_ns = kDefaultTimeoutNs;
   return cuda_status(launch_grouped_gemm(map, a, EPI_STORE_F32, tiles, dev.num_sms, s));
@@ -417,8 +451,7 @@ moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const floa
     return MOE_OK;
   };
   int launches = 0;
-  const int ri = router_impl == MOE_ROUTER_AUTO ? ((T >= 1024 && E % 8 == 0) ? MOE_ROUTER_TC : MOE_ROUTER_FMA)
-                                                : router_impl;
+  const int ri = resolve_router(router_impl, E);
   MOE_TRY(mark(0));
   MOE_TRY(run_route(x, w_router, bias, T, H, E, k, ids, tw, ri, ws, L, dev, s));
   launches += ri == MOE_ROUTER_TC ? 3 : 2;

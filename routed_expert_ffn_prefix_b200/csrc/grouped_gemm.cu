@@ -24,6 +24,14 @@
 //     mbarriers.  One thread issues tcgen05.mma into TMEM; four epilogue
 //     warps drain TMEM with tcgen05.ld.  Accumulators are double-buffered in
 //     TMEM when they fit, so a unit's epilogue overlaps the next unit's MMAs.
+//   * The weight stream is what bounds the layer, and shared memory only
+//     holds a few stages, so the producer also prefetches weight tiles into
+//     L2 a fixed number of pipeline steps ahead (across unit boundaries):
+//     the ring then only has to cover L2 latency, not HBM latency.
+//   * A unit may cover a slice of K (split-K, store epilogue only): each
+//     slice writes its own partial slab, summed later in a fixed order, so
+//     results stay bitwise reproducible.  The router uses this to spread
+//     small token counts over every SM.
 //   * Every wait is bounded (see common.cuh); routing metadata is range
 //     checked before it is used as an address.
 //
@@ -54,7 +62,7 @@ struct Cfg {
 };
 
 struct Unit {
-  int group, nb, row0, rows;
+  int group, nb, row0, rows, ks, kb, ke;  // ks: K split; [kb, ke): its k-steps (of kBK)
 };
 
 __device__ __forceinline__ int group_rows_begin(const GemmArgs& a, int g) {
@@ -66,7 +74,7 @@ __device__ __forceinline__ int group_rows_end(const GemmArgs& a, int g) {
 
 template <int NT>
 __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, const int* ustart, int ngroups, int u) {
-  int lo = 0, hi = ngroups - 1;  // last group with ustart[g] <= u
+  int lo = 0, hi = ngroups - 1;  // last group with ustart[g] <= u (skips empty groups)
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (ustart[mid] <= u) lo = mid; else hi = mid - 1;
@@ -74,13 +82,19 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, const int* ustart
   const int g = lo;
   const int b = group_rows_begin(a, g), e = group_rows_end(a, g);
   const int passes = (e - b + NT - 1) / NT;
+  const int S = a.k_splits;
   const int local = u - ustart[g];
   Unit r;
   r.group = g;
-  r.nb = local / passes;
-  const int pass = local - r.nb * passes;
+  r.nb = local / (passes * S);
+  const int rem = local - r.nb * passes * S;
+  const int pass = rem / S;
+  r.ks = rem - pass * S;
   r.row0 = b + pass * NT;
   r.rows = min(NT, e - r.row0);
+  const int nkt = a.K / kBK;
+  r.kb = r.ks * nkt / S;
+  r.ke = (r.ks + 1) * nkt / S;
   return r;
 }
 
@@ -96,7 +110,7 @@ __device__ void build_unit_prefix(const GemmArgs& a, int ngroups, int* ustart, i
     const int b = group_rows_begin(a, g), e = group_rows_end(a, g);
     if (b < 0 || e < b || e > a.rows_cap) bad = g;
     ustart[g] = sum;
-    sum += (e > b && bad < 0) ? ((e - b + NT - 1) / NT) * a.n_blocks : 0;
+    sum += (e > b && bad < 0) ? ((e - b + NT - 1) / NT) * a.n_blocks * a.k_splits : 0;
   }
   int incl = sum;
 #pragma unroll
@@ -118,6 +132,44 @@ __device__ void build_unit_prefix(const GemmArgs& a, int ngroups, int* ustart, i
 }
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+
+// Walks the same (unit, k-step) sequence as the producer, a fixed number of
+// steps ahead, and prefetches each step's weight tiles into L2.
+template <int NT>
+struct PrefetchCursor {
+  int u, it, nk, kiters;
+  Unit un;
+
+  __device__ void load(const GemmArgs& a, const int* ustart, int ngroups, int total) {
+    if (u < total) {
+      un = decode_unit<NT>(a, ustart, ngroups, u);
+      nk = un.ke - un.kb;
+      kiters = nk * a.krep;
+    }
+  }
+  __device__ void init(const GemmArgs& a, const int* ustart, int ngroups, int total) {
+    u = blockIdx.x;
+    it = 0;
+    load(a, ustart, ngroups, total);
+  }
+  __device__ void issue_and_advance(const GemmArgs& a, const CUtensorMap* map, const int* ustart, int ngroups,
+                                    int total) {
+    if (u >= total) return;
+    const int rep = it / nk, kt = un.kb + (it - rep * nk);
+    const int c0 = un.nb * a.col_stride, c1 = c0 + a.col1_off;
+    const int d2 = a.a_dim2_rep ? rep : un.group;
+    const int k0 = kt * kBK;
+    tma_prefetch_3d(map, c0, k0, d2);
+    tma_prefetch_3d(map, c0 + 64, k0, d2);
+    tma_prefetch_3d(map, c1, k0, d2);
+    tma_prefetch_3d(map, c1 + 64, k0, d2);
+    if (++it == kiters) {
+      u += gridDim.x;
+      it = 0;
+      load(a, ustart, ngroups, total);
+    }
+  }
+};
 
 template <int NT, int ST, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -162,8 +214,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int total = *total_units;
-  const int kiters = (a.K / kBK) * a.krep;
-  const int kt_per_rep = a.K / kBK;
 
   if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ producers
@@ -172,6 +222,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int chunk = pt & 7, rsub = pt >> 3;
     const uint64_t pol_w = policy_evict_first();
     const __nv_bfloat16* bsrc = reinterpret_cast<const __nv_bfloat16*>(a.b_src);
+    PrefetchCursor<NT> pf;
+    if (pt == 0) {
+      pf.init(a, ustart, ngroups, total);
+      for (int i = 0; i < a.prefetch_steps; ++i) pf.issue_and_advance(a, &wmap, ustart, ngroups, total);
+    }
     int stage = 0;
     uint32_t phase = 0;
     uint32_t issued_mask = 0, issued_par = 0;  // per stage: loads issued / parity of the last issue
@@ -194,8 +249,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         src[i] = s;
       }
       const int colA0 = un.nb * a.col_stride, colA1 = colA0 + a.col1_off;
+      const int nk = un.ke - un.kb, kiters = nk * a.krep;
       for (int it = 0; it < kiters; ++it) {
-        const int rep = it / kt_per_rep, kt = it - rep * kt_per_rep;
+        const int rep = it / nk, kt = un.kb + (it - rep * nk);
         if (!mbar_wait(&empty[stage], phase ^ 1u, wc, 100 + stage)) { ok = false; break; }
         uint8_t* sA0 = smem + stage * C::STAGE_BYTES;
         uint8_t* sA1 = sA0 + kATileBytes;
@@ -217,6 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(sA0 + kATileBytes / 2, &wmap, &full[stage], colA0 + 64, k0, d2, pol_w);
           tma_load_3d(sA1, &wmap, &full[stage], colA1, k0, d2, pol_w);
           tma_load_3d(sA1 + kATileBytes / 2, &wmap, &full[stage], colA1 + 64, k0, d2, pol_w);
+          pf.issue_and_advance(a, &wmap, ustart, ngroups, total);
         }
         issued_mask |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -251,6 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d0 = tmem + buf * 2 * NT, d1 = d0 + NT;
         const int N = (un.rows + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(128, N, /*A MN-major*/ true, /*B K-major*/ false);
+        const int kiters = (un.ke - un.kb) * a.krep;
         uint32_t acc = 0;
         for (int it = 0; it < kiters; ++it) {
           if (!mbar_wait(&full[stage], phase, wc, 300 + stage)) { ok = false; break; }
@@ -311,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         } else {
-          float* out = reinterpret_cast<float*>(a.out);
+          float* out = reinterpret_cast<float*>(a.out) + (size_t)un.ks * a.split_stride;
           const bool ok0 = col < a.n_valid, ok1 = col + a.out_col1_off < a.n_valid;
 #pragma unroll
           for (int j = 0; j < 16; ++j) {

@@ -32,6 +32,9 @@ struct GemmArgs {
   int out_col1_off;    // store epilogue: second tile's output columns offset
   int n_valid;         // output columns < n_valid are written
   int rows_cap;        // offsets[groups] may not exceed this (rows of out / row_index)
+  int k_splits;        // K range split across this many work units (store epilogue only)
+  size_t split_stride; // elements between the partial-result slabs of consecutive K splits
+  int prefetch_steps;  // weight tiles are prefetched into L2 this many pipeline steps ahead
   DevStatus* status;
   uint64_t timeout_ns;
 };
@@ -46,8 +49,9 @@ cudaError_t launch_grouped_gemm(const CUtensorMap& wmap, const GemmArgs& a, int 
 cudaError_t launch_router_split(const float* w, int H, int E, uint16_t* planes, cudaStream_t s);
 cudaError_t launch_router_logits_fma(const uint16_t* x, const float* w, int T, int H, int E, float* logits,
                                      cudaStream_t s);
-cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, int32_t* ids, float* w,
-                        DevStatus* st, cudaStream_t s);
+// logits: nsplit partial slabs of [T, E], split_stride elements apart, summed in slab order.
+cudaError_t launch_topk(const float* logits, int nsplit, size_t split_stride, const float* bias, int T, int E, int k,
+                        int32_t* ids, float* w, DevStatus* st, cudaStream_t s);
 
 // Permutation.
 int permute_num_blocks(int T, int k);

@@ -10,20 +10,25 @@
 // (token ascending), so the permutation is deterministic and can be
 // checked bit for bit.  Atomics would make positions run-dependent; instead:
 //
-//   1. hist:    block b counts the expert ids of its chunk of slots.
-//   2. scan:    one block turns the [blocks, E] counts into per-(block,
-//               expert) starting rows (column scan over blocks, then an
-//               exclusive scan over experts), and writes counts/offsets.
-//   3. scatter: one warp per chunk walks its slots in order, 32 at a time;
-//               lanes with the same expert are ranked by __match_any_sync, so
-//               each slot's row = start[b][e] + earlier slots of e in the chunk.
+//   1. hist:    block b counts the expert ids of its chunk of 1024 slots.
+//   2. scan:    one block turns the [blocks, E] counts into each block's
+//               starting rank within each expert (a warp-parallel scan down
+//               every column), then scans the expert totals into offsets.
+//   3. scatter: each block splits its chunk into four 256-slot runs, one per
+//               warp, ranks the runs against each other per expert, and each
+//               warp walks its run in order, 32 slots at a time; lanes with
+//               the same expert are ranked by __match_any_sync, so a slot's
+//               row = offsets[e] + earlier slots of e in earlier blocks, runs
+//               and lanes.
 #include "kernels.h"
 
 namespace moe {
 
 namespace {
 
-constexpr int kChunk = 256;  // slots per block (hist/scatter)
+constexpr int kChunk = 1024;  // slots per block (hist/scatter)
+constexpr int kScatterWarps = 4;
+constexpr int kRun = kChunk / kScatterWarps;  // slots walked in order by one warp
 
 __global__ void hist_kernel(const int32_t* __restrict__ ids, int n, int E, int32_t* __restrict__ block_hist,
                             DevStatus* st) {
@@ -51,23 +56,31 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ block_
                                                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
   __shared__ int32_t tot[kMaxExperts];
   __shared__ int32_t warp_sums[32];
-  const int tid = threadIdx.x;
-  // column scan over blocks: block_hist[b][e] <- rows of e in blocks < b
-  for (int e = tid; e < E; e += blockDim.x) {
-    int run = 0;
-    for (int b = 0; b < nblk; ++b) {
-      const int v = block_hist[(size_t)b * E + e];
-      block_hist[(size_t)b * E + e] = run;
-      run += v;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // block_hist[b][e] <- rows of expert e in blocks < b (one warp per column)
+  for (int e = warp; e < E; e += 32) {
+    int carry = 0;
+    for (int b0 = 0; b0 < nblk; b0 += 32) {
+      const int b = b0 + lane;
+      const int v = b < nblk ? block_hist[(size_t)b * E + e] : 0;
+      int incl = v;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += o;
+      }
+      if (b < nblk) block_hist[(size_t)b * E + e] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    tot[e] = run;
-    counts[e] = run;
+    if (lane == 0) {
+      tot[e] = carry;
+      counts[e] = carry;
+    }
   }
   __syncthreads();
-  // exclusive scan of tot over experts (E <= 1024 = blockDim)
+  // exclusive scan of the expert totals (E <= 1024 = blockDim)
   const int v = tid < E ? tot[tid] : 0;
   int incl = v;
-  const int lane = tid & 31, warp = tid >> 5;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
     const int o = __shfl_up_sync(0xffffffffu, incl, d);
@@ -88,36 +101,45 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ block_
   const int excl = incl - v + (warp > 0 ? warp_sums[warp - 1] : 0);
   if (tid < E) offsets[tid] = excl;
   if (tid == E - 1) offsets[E] = excl + v;
-  __syncthreads();
-  if (tid < E) tot[tid] = excl;
-  __syncthreads();
-  for (int e = tid; e < E; e += blockDim.x) {
-    const int base = tot[e];
-    for (int b = 0; b < nblk; ++b) block_hist[(size_t)b * E + e] += base;
-  }
 }
 
-// One warp per block.
-__global__ void __launch_bounds__(32) scatter_kernel(const int32_t* __restrict__ ids, int n, int E, int k,
-                                                   const int32_t* __restrict__ block_hist,
-                                                   int32_t* __restrict__ sorted_ids,
-                                                   int32_t* __restrict__ inv_perm) {
-  extern __shared__ int32_t run[];
-  const int lane = threadIdx.x;
-  for (int e = lane; e < E; e += 32) run[e] = block_hist[(size_t)blockIdx.x * E + e];
-  __syncwarp();
-  const int s0 = blockIdx.x * kChunk;
-  for (int r = 0; r < kChunk; r += 32) {
+__global__ void __launch_bounds__(kScatterWarps * 32) scatter_kernel(const int32_t* __restrict__ ids, int n, int E,
+                                                                   int k, const int32_t* __restrict__ block_hist,
+                                                                   const int32_t* __restrict__ offsets,
+                                                                   int32_t* __restrict__ sorted_ids,
+                                                                   int32_t* __restrict__ inv_perm) {
+  extern __shared__ int32_t base[];  // [kScatterWarps][E]: next row of expert e for warp w
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int s0 = blockIdx.x * kChunk + w * kRun;
+  for (int i = tid; i < kScatterWarps * E; i += blockDim.x) base[i] = 0;
+  __syncthreads();
+  for (int i = lane; i < kRun; i += 32) {
+    const int s = s0 + i;
+    if (s < n) {
+      const int e = ids[s];
+      if (e >= 0 && e < E) atomicAdd(&base[w * E + e], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    int run = offsets[e] + block_hist[(size_t)blockIdx.x * E + e];
+    for (int j = 0; j < kScatterWarps; ++j) {
+      const int c = base[j * E + e];
+      base[j * E + e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  int* mine = base + w * E;
+  for (int r = 0; r < kRun; r += 32) {
     const int s = s0 + r + lane;
-    const bool valid = s < n;
-    int e = valid ? ids[s] : -1;
+    int e = s < n ? ids[s] : -1;
     if (e >= E) e = -1;  // out-of-range ids were reported by hist_kernel; skip them here
     const uint32_t peers = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(peers & ((1u << lane) - 1u));
-    int pos = -1;
-    if (e >= 0) pos = run[e] + rank;
+    const int pos = e >= 0 ? mine[e] + rank : -1;
     __syncwarp();
-    if (e >= 0 && rank == 0) run[e] += __popc(peers);
+    if (e >= 0 && rank == 0) mine[e] += __popc(peers);
     __syncwarp();
     if (e >= 0) {
       sorted_ids[pos] = s / k;
@@ -135,14 +157,14 @@ cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* cou
                            cudaStream_t s) {
   const int n = T * k;
   const int nblk = permute_num_blocks(T, k);
-  const size_t sh = (size_t)E * sizeof(int32_t);
-  hist_kernel<<<nblk, 256, sh, s>>>(ids, n, E, block_hist, st);
+  hist_kernel<<<nblk, 256, (size_t)E * sizeof(int32_t), s>>>(ids, n, E, block_hist, st);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   scan_kernel<<<1, 1024, 0, s>>>(block_hist, nblk, E, counts, offsets);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  scatter_kernel<<<nblk, 32, sh, s>>>(ids, n, E, k, block_hist, sorted_ids, inv_perm);
+  scatter_kernel<<<nblk, kScatterWarps * 32, (size_t)kScatterWarps * E * sizeof(int32_t), s>>>(
+      ids, n, E, k, block_hist, offsets, sorted_ids, inv_perm);
   return cudaGetLastError();
 }
 

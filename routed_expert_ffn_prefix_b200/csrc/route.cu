@@ -91,7 +91,8 @@ __global__ void __launch_bounds__(kFmaThreads) router_logits_fma_kernel(const __
 constexpr int kTopkWarps = 8;
 constexpr int kPerLane = kMaxExperts / 32;
 
-__global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __restrict__ logits,
+__global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __restrict__ logits, int nsplit,
+                                                             size_t split_stride,
                                                              const float* __restrict__ bias, int T, int E,
                                                              int k, int32_t* __restrict__ ids,
                                                              float* __restrict__ wout, DevStatus* st) {
@@ -104,7 +105,13 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
 #pragma unroll
   for (int i = 0; i < kPerLane; ++i) {
     const int e = lane + 32 * i;
-    v[i] = e < E ? row[e] + (bias ? bias[e] : 0.f) : NEG;
+    if (e < E) {
+      float l = row[e];
+      for (int sp = 1; sp < nsplit; ++sp) l += row[sp * split_stride + e];  // K-split partials, in order
+      v[i] = l + (bias ? bias[e] : 0.f);
+    } else {
+      v[i] = NEG;
+    }
   }
   uint32_t taken = 0;
   const int nper = (E + 31) / 32;
@@ -162,9 +169,10 @@ cudaError_t launch_router_logits_fma(const uint16_t* x, const float* w, int T, i
   return cudaGetLastError();
 }
 
-cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, int32_t* ids, float* w,
-                        DevStatus* st, cudaStream_t s) {
-  topk_kernel<<<(T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, s>>>(logits, bias, T, E, k, ids, w, st);
+cudaError_t launch_topk(const float* logits, int nsplit, size_t split_stride, const float* bias, int T, int E, int k,
+                        int32_t* ids, float* w, DevStatus* st, cudaStream_t s) {
+  topk_kernel<<<(T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, s>>>(logits, nsplit, split_stride, bias, T, E,
+                                                                            k, ids, w, st);
   return cudaGetLastError();
 }
 
