@@ -13,8 +13,6 @@ constexpr int kMaxK = 64;
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-constexpr int kPrefetchSteps = 8;  // weight tiles prefetched into L2 this many ring steps ahead
-
 // Tensor-core router tiling: row tiles of 256 tokens from T >= 2048, else 64;
 // the K range (H) is split so that about two work units land on each of the
 // 148 SMs.  A function of the shapes only, so the workspace layout and the
@@ -29,7 +27,8 @@ inline int resolve_router(int impl, int E) {
 inline int router_tiles(int T) { return T >= 2048 ? MOE_TILES_LARGE : MOE_TILES_SMALL; }
 inline int router_splits(int T, int H, int E) {
   const int nt = router_tiles(T) == MOE_TILES_LARGE ? 256 : 64;
-  const int base = ((T + nt - 1) / nt) * ((E + 255) / 256);
+  const int cols = 128 * gemm_tiles_per_unit(router_tiles(T), EPI_STORE_F32);
+  const int base = ((T + nt - 1) / nt) * ((E + cols - 1) / cols);
   int s = (296 + base - 1) / base;
   const int nkt = H / 64;
   if (s > nkt) s = nkt;
@@ -175,6 +174,7 @@ moe_status_t run_route(const uint16_t* x, const float* w_router, const float* bi
     CUtensorMap map;
     if (!make_weight_map(&map, planes, (uint64_t)E, (uint64_t)H, 3)) return MOE_ERR_CUDA;
     nsplit = router_splits(T, H, E);
+    const int cols = 128 * gemm_tiles_per_unit(router_tiles(T), EPI_STORE_F32);
     GemmArgs a{};
     a.offsets = nullptr;
     a.row_index = nullptr;
@@ -185,18 +185,17 @@ moe_status_t run_route(const uint16_t* x, const float* w_router, const float* bi
     a.K = H;
     a.krep = 3;
     a.a_dim2_rep = 1;
-    a.n_blocks = (E + 255) / 256;
-    a.col_stride = 256;
+    a.n_blocks = (E + cols - 1) / cols;
+    a.col_stride = cols;
     a.col1_off = 128;
     a.out = logits;
     a.ld_out = E;
-    a.out_col_stride = 256;
+    a.out_col_stride = cols;
     a.out_col1_off = 128;
     a.n_valid = E;
     a.rows_cap = T;
     a.k_splits = nsplit;
     a.split_stride = (size_t)T * E;
-    a.prefetch_steps = kPrefetchSteps;
     a.status = st;
     a.timeout_ns = kDefaultTimeoutNs;
     MOE_TRY(cuda_status(launch_grouped_gemm(map, a, EPI_STORE_F32, router_tiles(T), dev.num_sms, s)));
@@ -232,7 +231,6 @@ moe_status_t run_swiglu(const uint16_t* x, int src_rows, const uint16_t* w_gate_
   a.rows_cap = rows;
   a.k_splits = 1;
   a.split_stride = 0;
-  a.prefetch_steps = kPrefetchSteps;
   a.status = st;
   a.timeout_ns = kDefaultTimeoutNs;
   return cuda_status(launch_grouped_gemm(map, a, EPI_SWIGLU, tiles, dev.num_sms, s));
@@ -242,6 +240,7 @@ moe_status_t run_down(const uint16_t* h, const uint16_t* w_down, const int32_t* 
                       int I, int tiles, float* o, DevStatus* st, const DeviceInfo& dev, cudaStream_t s) {
   CUtensorMap map;
   if (!make_weight_map(&map, w_down, (uint64_t)H, (uint64_t)I, (uint64_t)E)) return MOE_ERR_CUDA;
+  const int cols = 128 * gemm_tiles_per_unit(tiles, EPI_STORE_F32);  // output columns per work unit
   GemmArgs a{};
   a.offsets = offsets;
   a.row_index = nullptr;
@@ -252,18 +251,17 @@ moe_status_t run_down(const uint16_t* h, const uint16_t* w_down, const int32_t* 
   a.K = I;
   a.krep = 1;
   a.a_dim2_rep = 0;
-  a.n_blocks = H / 256;
-  a.col_stride = 256;
+  a.n_blocks = H / cols;
+  a.col_stride = cols;
   a.col1_off = 128;
   a.out = o;
   a.ld_out = H;
-  a.out_col_stride = 256;
+  a.out_col_stride = cols;
   a.out_col1_off = 128;
   a.n_valid = H;
   a.rows_cap = rows;
   a.k_splits = 1;
   a.split_stride = 0;
-  a.prefetch_steps = kPrefetchSteps;
   a.status = st;
   a.timeout_ns = kDefaultTimeoutNs;
   return cuda_status(launch_grouped_gemm(map, a, EPI_STORE_F32, tiles, dev.num_sms, s));

@@ -14,20 +14,19 @@
 //     bound by streaming the activated experts' weights, and decode-sized
 //     groups of 1..30 rows need no padding to 128.
 //   * A work unit = (group, column block, row pass).  A column block holds
-//     two 128-column MMA tiles sharing the same token rows: for gate/up they
-//     are the gate and the up columns of the same 128 intermediate units,
-//     so SwiGLU is computed in the epilogue from two TMEM accumulators; for
-//     down they are 256 adjacent output columns.
+//     MT (1 or 2) 128-column MMA tiles sharing the same token rows: for
+//     gate/up (MT = 2) they are the gate and the up columns of the same 128
+//     intermediate units, so SwiGLU is computed in the epilogue from two TMEM
+//     accumulators; for down they are 128 or 256 adjacent output columns.
 //   * Weight tiles arrive by TMA (128-byte swizzle, MN-major operand), token
 //     rows by cp.async 16-byte gathers written in the same swizzle (K-major
 //     operand), both into a multi-stage shared-memory ring guarded by
-//     mbarriers.  One thread issues tcgen05.mma into TMEM; four epilogue
-//     warps drain TMEM with tcgen05.ld.  Accumulators are double-buffered in
-//     TMEM when they fit, so a unit's epilogue overlaps the next unit's MMAs.
-//   * The weight stream is what bounds the layer, and shared memory only
-//     holds a few stages, so the producer also prefetches weight tiles into
-//     L2 a fixed number of pipeline steps ahead (across unit boundaries):
-//     the ring then only has to cover L2 latency, not HBM latency.
+//     mbarriers.  One thread issues tcgen05.mma into TMEM; eight epilogue
+//     warps (two per TMEM lane quarter, splitting the rows) drain TMEM with
+//     tcgen05.ld.  Accumulators are double-buffered in TMEM when 2*MT*NT
+//     columns fit in its 512, so a unit's epilogue overlaps the next unit's
+//     MMAs; the single-tile mode (MT = 1) exists to get that overlap at 256
+//     rows for the down GEMM, whose short K loop makes its epilogue heavy.
 //   * A unit may cover a slice of K (split-K, store epilogue only): each
 //     slice writes its own partial slab, summed later in a fixed order, so
 //     results stay bitwise reproducible.  The router uses this to spread
@@ -35,30 +34,38 @@
 //   * Every wait is bounded (see common.cuh); routing metadata is range
 //     checked before it is used as an address.
 //
-// Warp roles (288 threads): warps 0-3 epilogue, warps 4-7 producers,
-// warp 8 TMEM allocation + MMA issue.
+// Warp roles (416 threads): warps 0-7 epilogue, warps 8-11 producers,
+// warp 12 TMEM allocation + MMA issue.
 #include "kernels.h"
 
 namespace moe {
 
 namespace {
 
-constexpr int kThreads = 288;
+constexpr int kEpiWarps = 8;
+constexpr int kProdWarps = 4;
+constexpr int kMmaWarp = kEpiWarps + kProdWarps;
+constexpr int kThreads = (kMmaWarp + 1) * 32;
+constexpr int kProdThreads = kProdWarps * 32;
+constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kATileBytes = 128 * 64 * 2;  // 128 weight columns x 64 k, bf16
 constexpr int kBK = 64;                    // k per pipeline stage (one 128-byte swizzle row)
 
-template <int NT, int ST>
+template <int NT, int ST, int MT>
 struct Cfg {
   static constexpr int B_BYTES = NT * kBK * 2;
-  static constexpr int STAGE_BYTES = 2 * kATileBytes + B_BYTES;
-  static constexpr int NBUF = (4 * NT <= 512) ? 2 : 1;
-  static constexpr int ACC_COLS = NBUF * 2 * NT;
+  static constexpr int A_BYTES = MT * kATileBytes;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int NBUF = (2 * MT * NT <= 512) ? 2 : 1;
+  static constexpr int ACC_COLS = NBUF * MT * NT;
   static constexpr int TMEM_COLS = ACC_COLS <= 32 ? 32 : ACC_COLS <= 64 ? 64 : ACC_COLS <= 128 ? 128
                                    : ACC_COLS <= 256 ? 256 : 512;
   // ring + barriers/flags (256) + unit prefix (kMaxExperts+1 ints) + alignment slack
   static constexpr int SMEM_BYTES = ST * STAGE_BYTES + 256 + 4 * (kMaxExperts + 1) + 1024;
-  static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "row pass must be 16..256, multiple of 16");
+  static_assert(NT % 32 == 0 && NT >= 32 && NT <= 256, "row pass must be 32..256, multiple of 32");
+  static_assert(MT == 1 || MT == 2, "one or two MMA tiles per unit");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte swizzle alignment");
 };
 
 struct Unit {
@@ -131,50 +138,14 @@ __device__ void build_unit_prefix(const GemmArgs& a, int ngroups, int* ustart, i
   }
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+// silu(g) = g * sigmoid(g); h is rounded to bf16 right after, so the fast
+// exponential and division are accurate enough.
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-// Walks the same (unit, k-step) sequence as the producer, a fixed number of
-// steps ahead, and prefetches each step's weight tiles into L2.
-template <int NT>
-struct PrefetchCursor {
-  int u, it, nk, kiters;
-  Unit un;
-
-  __device__ void load(const GemmArgs& a, const int* ustart, int ngroups, int total) {
-    if (u < total) {
-      un = decode_unit<NT>(a, ustart, ngroups, u);
-      nk = un.ke - un.kb;
-      kiters = nk * a.krep;
-    }
-  }
-  __device__ void init(const GemmArgs& a, const int* ustart, int ngroups, int total) {
-    u = blockIdx.x;
-    it = 0;
-    load(a, ustart, ngroups, total);
-  }
-  __device__ void issue_and_advance(const GemmArgs& a, const CUtensorMap* map, const int* ustart, int ngroups,
-                                    int total) {
-    if (u >= total) return;
-    const int rep = it / nk, kt = un.kb + (it - rep * nk);
-    const int c0 = un.nb * a.col_stride, c1 = c0 + a.col1_off;
-    const int d2 = a.a_dim2_rep ? rep : un.group;
-    const int k0 = kt * kBK;
-    tma_prefetch_3d(map, c0, k0, d2);
-    tma_prefetch_3d(map, c0 + 64, k0, d2);
-    tma_prefetch_3d(map, c1, k0, d2);
-    tma_prefetch_3d(map, c1 + 64, k0, d2);
-    if (++it == kiters) {
-      u += gridDim.x;
-      it = 0;
-      load(a, ustart, ngroups, total);
-    }
-  }
-};
-
-template <int NT, int ST, int EPI>
+template <int NT, int ST, int MT, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap wmap, const GemmArgs a) {
-  using C = Cfg<NT, ST>;
+  using C = Cfg<NT, ST, MT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * C::STAGE_BYTES);
@@ -192,88 +163,85 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     for (int s = 0; s < ST; ++s) {
-      mbar_init(full + s, 128 + 1);  // 128 producer cp.async arrivals + 1 expect_tx arrival
+      mbar_init(full + s, kProdThreads + 1);  // producer cp.async arrivals + 1 expect_tx arrival
       mbar_init(empty + s, 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull + b, 1);
-      mbar_init(tempty + b, 128);
+      mbar_init(tempty + b, kEpiThreads);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0) build_unit_prefix<NT>(a, ngroups, ustart, total_units);
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) prefetch_tmap(&wmap);
+  if (warp == kEpiWarps && lane == 0) prefetch_tmap(&wmap);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int total = *total_units;
 
-  if (warp >= 4 && warp < 8) {
+  if (warp >= kEpiWarps && warp < kMmaWarp) {
     // ------------------------------------------------------------ producers
     const WaitCtx wc{a.status, abort_flag, a.timeout_ns, SITE_GEMM_PRODUCER};
-    const int pt = tid - 128;
-    const int chunk = pt & 7, rsub = pt >> 3;
+    const int pt = tid - kEpiThreads;
+    const int chunk = pt & 7, rsub = pt >> 3;  // 16-byte chunk of a row; first row of this thread
+    constexpr int kRowStep = kProdThreads / 8;
+    constexpr int kRowsPerThread = NT / kRowStep;
     const uint64_t pol_w = policy_evict_first();
     const __nv_bfloat16* bsrc = reinterpret_cast<const __nv_bfloat16*>(a.b_src);
-    PrefetchCursor<NT> pf;
-    if (pt == 0) {
-      pf.init(a, ustart, ngroups, total);
-      for (int i = 0; i < a.prefetch_steps; ++i) pf.issue_and_advance(a, &wmap, ustart, ngroups, total);
-    }
     int stage = 0;
     uint32_t phase = 0;
     uint32_t issued_mask = 0, issued_par = 0;  // per stage: loads issued / parity of the last issue
     bool ok = true;
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
       const Unit un = decode_unit<NT>(a, ustart, ngroups, u);
-      int src[NT / 16];
+      int src[kRowsPerThread];
 #pragma unroll
-      for (int i = 0; i < NT / 16; ++i) {
-        const int c = rsub + 16 * i;
-        int s = -1;
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        const int c = rsub + kRowStep * i;
+        int sr = -1;
         if (c < un.rows) {
           const int r = un.row0 + c;
-          s = a.row_index ? __ldg(a.row_index + r) : r;
-          if (s < 0 || s >= a.src_rows) {
+          sr = a.row_index ? __ldg(a.row_index + r) : r;
+          if (sr < 0 || sr >= a.src_rows) {
             raise_error(a.status, MOE_ERR_DEVICE_BOUNDS, SITE_GEMM_GATHER, r);
-            s = -1;
+            sr = -1;
           }
         }
-        src[i] = s;
+        src[i] = sr;
       }
-      const int colA0 = un.nb * a.col_stride, colA1 = colA0 + a.col1_off;
+      const int col0 = un.nb * a.col_stride;
       const int nk = un.ke - un.kb, kiters = nk * a.krep;
       for (int it = 0; it < kiters; ++it) {
         const int rep = it / nk, kt = un.kb + (it - rep * nk);
         if (!mbar_wait(&empty[stage], phase ^ 1u, wc, 100 + stage)) { ok = false; break; }
-        uint8_t* sA0 = smem + stage * C::STAGE_BYTES;
-        uint8_t* sA1 = sA0 + kATileBytes;
-        const uint32_t sB = smem_u32(sA0 + 2 * kATileBytes);
+        uint8_t* sA = smem + stage * C::STAGE_BYTES;
+        const uint32_t sB = smem_u32(sA + C::A_BYTES);
 #pragma unroll
-        for (int i = 0; i < NT / 16; ++i) {
+        for (int i = 0; i < kRowsPerThread; ++i) {
           if (src[i] >= 0) {
-            const int c = rsub + 16 * i;
+            const int c = rsub + kRowStep * i;
             cp_async_16(sB + c * 128 + ((chunk ^ (c & 7)) << 4),
                         bsrc + (size_t)src[i] * a.K + kt * kBK + chunk * 8);
           }
         }
         cp_async_arrive_noinc(&full[stage]);
         if (pt == 0) {
-          mbar_arrive_expect_tx(&full[stage], 4 * (kATileBytes / 2));
+          mbar_arrive_expect_tx(&full[stage], C::A_BYTES);
           const int d2 = a.a_dim2_rep ? rep : un.group;
           const int k0 = kt * kBK;
-          tma_load_3d(sA0, &wmap, &full[stage], colA0, k0, d2, pol_w);
-          tma_load_3d(sA0 + kATileBytes / 2, &wmap, &full[stage], colA0 + 64, k0, d2, pol_w);
-          tma_load_3d(sA1, &wmap, &full[stage], colA1, k0, d2, pol_w);
-          tma_load_3d(sA1 + kATileBytes / 2, &wmap, &full[stage], colA1 + 64, k0, d2, pol_w);
-          pf.issue_and_advance(a, &wmap, ustart, ngroups, total);
+#pragma unroll
+          for (int t = 0; t < MT; ++t) {
+            const int c = col0 + t * a.col1_off;
+            tma_load_3d(sA + t * kATileBytes, &wmap, &full[stage], c, k0, d2, pol_w);
+            tma_load_3d(sA + t * kATileBytes + kATileBytes / 2, &wmap, &full[stage], c + 64, k0, d2, pol_w);
+          }
         }
         issued_mask |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -283,15 +251,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     cp_async_wait_all();
     if (!ok && pt == 0) {
       // Aborted: let every load still in flight land before the block exits.
-      const WaitCtx drain{nullptr, abort_flag, a.timeout_ns, SITE_GEMM_PRODUCER};
       for (int s = 0; s < ST; ++s) {
         if (!(issued_mask >> s & 1u)) continue;
         const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(&full[s], (issued_par >> s) & 1u) && globaltimer_ns() - t0 < drain.timeout_ns) {
+        while (!mbar_try_wait(&full[s], (issued_par >> s) & 1u) && globaltimer_ns() - t0 < a.timeout_ns) {
         }
       }
     }
-  } else if (warp == 8) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const WaitCtx wc{a.status, abort_flag, a.timeout_ns, SITE_GEMM_MMA};
@@ -305,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t apar = C::NBUF == 2 ? ((acc_it >> 1) & 1) : (acc_it & 1);
         if (!mbar_wait(&tempty[buf], apar ^ 1u, wc, 200 + buf)) break;
         tc_fence_after();
-        const uint32_t d0 = tmem + buf * 2 * NT, d1 = d0 + NT;
+        const uint32_t d0 = tmem + buf * MT * NT;
         const int N = (un.rows + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(128, N, /*A MN-major*/ true, /*B K-major*/ false);
         const int kiters = (un.ke - un.kb) * a.krep;
@@ -314,17 +281,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&full[stage], phase, wc, 300 + stage)) { ok = false; break; }
           tc_fence_after();
           fence_proxy_async_smem();
-          const uint32_t sA0 = smem_u32(smem + stage * C::STAGE_BYTES);
-          const uint32_t sA1 = sA0 + kATileBytes, sB = sA0 + 2 * kATileBytes;
+          const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sB = sA + C::A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
-            // A (weights, MN-major): +16 k = two 8-row groups = 2048 B; the two
-            // 64-column halves sit 8192 B apart.  B (rows, K-major): +16 k = 32 B.
-            const uint64_t a0 = smem_desc_sw128(sA0 + kk * 2048, 8192, 1024);
-            const uint64_t a1 = smem_desc_sw128(sA1 + kk * 2048, 8192, 1024);
+            // B (rows, K-major): +16 k = 32 B inside the 128-byte swizzle row.
             const uint64_t bd = smem_desc_sw128(sB + kk * 32, 16, 1024);
-            mma_bf16(d0, a0, bd, idesc, acc);
-            mma_bf16(d1, a1, bd, idesc, acc);
+#pragma unroll
+            for (int t = 0; t < MT; ++t) {
+              // A (weights, MN-major): +16 k = two 8-row groups = 2048 B; the two
+              // 64-column halves of a tile sit 8192 B apart.
+              const uint64_t ad = smem_desc_sw128(sA + t * kATileBytes + kk * 2048, 8192, 1024);
+              mma_bf16(d0 + t * NT, ad, bd, idesc, acc);
+            }
             acc = 1;
           }
           mma_commit(&empty[stage]);
@@ -342,8 +311,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ epilogue (warps 0-3)
+    // ------------------------------------------------------------ epilogue (warps 0-7)
+    // Warp w reads TMEM lanes 32*(w%4).. (one weight column per thread) and
+    // handles the 32-row chunks c0 = 32*(w/4) + 64*j of the unit's rows.
     const WaitCtx wc{a.status, abort_flag, a.timeout_ns, SITE_GEMM_EPILOGUE};
+    const int quarter = warp & 3, half = warp >> 2;
     int acc_it = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x) {
       const Unit un = decode_unit<NT>(a, ustart, ngroups, u);
@@ -351,32 +323,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t apar = C::NBUF == 2 ? ((acc_it >> 1) & 1) : (acc_it & 1);
       if (!mbar_wait(&tfull[buf], apar, wc, 400 + buf)) break;
       tc_fence_after();
-      const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + buf * 2 * NT;
-      const int col = un.nb * a.out_col_stride + warp * 32 + lane;
-      for (int c0 = 0; c0 < un.rows; c0 += 16) {
-        float v0[16], v1[16];
-        tmem_ld_2x16(tbase + c0, tbase + NT + c0, v0, v1);
-        const int nr = min(16, un.rows - c0);
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * MT * NT;
+      const int col = un.nb * a.out_col_stride + quarter * 32 + lane;
+      for (int c0 = half * 32; c0 < un.rows; c0 += 64) {
+        const int nr = min(32, un.rows - c0);
         if (EPI == EPI_SWIGLU) {
+          float g[32], v[32];
+          tmem_ld_4x16(tbase + c0, tbase + c0 + 16, tbase + NT + c0, tbase + NT + c0 + 16, g, g + 16, v, v + 16);
           __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
           if (col < a.n_valid) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              if (j < nr) {
-                const float hv = silu_f(v0[j]) * v1[j];
-                out[(size_t)(un.row0 + c0 + j) * a.ld_out + col] = __float2bfloat16_rn(hv);
-              }
+            for (int j = 0; j < 32; ++j) {
+              if (j < nr)
+                out[(size_t)(un.row0 + c0 + j) * a.ld_out + col] = __float2bfloat16_rn(silu_f(g[j]) * v[j]);
             }
           }
         } else {
           float* out = reinterpret_cast<float*>(a.out) + (size_t)un.ks * a.split_stride;
-          const bool ok0 = col < a.n_valid, ok1 = col + a.out_col1_off < a.n_valid;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (j < nr) {
-              float* orow = out + (size_t)(un.row0 + c0 + j) * a.ld_out;
-              if (ok0) orow[col] = v0[j];
-              if (ok1) orow[col + a.out_col1_off] = v1[j];
+          for (int t = 0; t < MT; ++t) {
+            float v[32];
+            tmem_ld_2x16(tbase + t * NT + c0, tbase + t * NT + c0 + 16, v, v + 16);
+            const int ct = col + t * a.out_col1_off;
+            if (ct < a.n_valid) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                if (j < nr) out[(size_t)(un.row0 + c0 + j) * a.ld_out + ct] = v[j];
+              }
             }
           }
         }
@@ -389,16 +362,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
-template <int NT, int ST, int EPI>
+template <int NT, int ST, int MT, int EPI>
 cudaError_t launch_cfg(const CUtensorMap& wmap, const GemmArgs& a, int num_sms, cudaStream_t stream) {
-  using C = Cfg<NT, ST>;
-  auto kern = grouped_gemm_kernel<NT, ST, EPI>;
+  using C = Cfg<NT, ST, MT>;
+  auto kern = grouped_gemm_kernel<NT, ST, MT, EPI>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (err != cudaSuccess) return err;
   kern<<<num_sms, kThreads, C::SMEM_BYTES, stream>>>(wmap, a);
@@ -407,14 +380,20 @@ cudaError_t launch_cfg(const CUtensorMap& wmap, const GemmArgs& a, int num_sms, 
 
 }  // namespace
 
+int gemm_tiles_per_unit(int tiles, int epilogue) {
+  (void)tiles;
+  (void)epilogue;
+  return 2;  // measured: one tile per unit doubles the token-row re-reads and loses more than it overlaps
+}
+
 cudaError_t launch_grouped_gemm(const CUtensorMap& wmap, const GemmArgs& a, int epilogue, int tiles, int num_sms,
                                 cudaStream_t stream) {
   if (tiles == MOE_TILES_LARGE) {
-    return epilogue == EPI_SWIGLU ? launch_cfg<256, 3, EPI_SWIGLU>(wmap, a, num_sms, stream)
-                                  : launch_cfg<256, 3, EPI_STORE_F32>(wmap, a, num_sms, stream);
+    return epilogue == EPI_SWIGLU ? launch_cfg<256, 3, 2, EPI_SWIGLU>(wmap, a, num_sms, stream)
+                                  : launch_cfg<256, 3, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
   }
-  return epilogue == EPI_SWIGLU ? launch_cfg<64, 5, EPI_SWIGLU>(wmap, a, num_sms, stream)
-                                : launch_cfg<64, 5, EPI_STORE_F32>(wmap, a, num_sms, stream);
+  return epilogue == EPI_SWIGLU ? launch_cfg<64, 5, 2, EPI_SWIGLU>(wmap, a, num_sms, stream)
+                                : launch_cfg<64, 5, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
 }
 
 }  // namespace moe

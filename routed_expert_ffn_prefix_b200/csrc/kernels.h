@@ -34,12 +34,16 @@ struct GemmArgs {
   int rows_cap;        // offsets[groups] may not exceed this (rows of out / row_index)
   int k_splits;        // K range split across this many work units (store epilogue only)
   size_t split_stride; // elements between the partial-result slabs of consecutive K splits
-  int prefetch_steps;  // weight tiles are prefetched into L2 this many pipeline steps ahead
   DevStatus* status;
   uint64_t timeout_ns;
 };
 
 enum Epilogue { EPI_SWIGLU = 0, EPI_STORE_F32 = 1 };
+
+// MMA tiles (128 weight columns each) per work unit of the given tile
+// policy and epilogue; the caller sets n_blocks/col_stride/out_col_stride
+// for units of 128 * that many columns.
+int gemm_tiles_per_unit(int tiles, int epilogue);
 
 // tiles: MOE_TILES_SMALL or MOE_TILES_LARGE.
 cudaError_t launch_grouped_gemm(const CUtensorMap& wmap, const GemmArgs& a, int epilogue, int tiles,

@@ -12,8 +12,9 @@
 //
 //   1. hist:    block b counts the expert ids of its chunk of 1024 slots.
 //   2. scan:    one block turns the [blocks, E] counts into each block's
-//               starting rank within each expert (a warp-parallel scan down
-//               every column), then scans the expert totals into offsets.
+//               starting rank within each expert (a running sum down every
+//               column, one thread per expert), then scans the expert totals
+//               into offsets.
 //   3. scatter: each block splits its chunk into four 256-slot runs, one per
 //               warp, ranks the runs against each other per expert, and each
 //               warp walks its run in order, 32 slots at a time; lanes with
@@ -57,25 +58,29 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ block_
   __shared__ int32_t tot[kMaxExperts];
   __shared__ int32_t warp_sums[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // block_hist[b][e] <- rows of expert e in blocks < b (one warp per column)
-  for (int e = warp; e < E; e += 32) {
+  // block_hist[b][e] <- rows of expert e in blocks < b.  One thread per
+  // expert walks its column; consecutive threads read consecutive experts
+  // (coalesced) and each batch of 8 loads is issued before any is used.
+  for (int e = tid; e < E; e += blockDim.x) {
     int carry = 0;
-    for (int b0 = 0; b0 < nblk; b0 += 32) {
-      const int b = b0 + lane;
-      const int v = b < nblk ? block_hist[(size_t)b * E + e] : 0;
-      int incl = v;
+    int b0 = 0;
+    for (; b0 + 8 <= nblk; b0 += 8) {
+      int v[8];
 #pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, incl, d);
-        if (lane >= d) incl += o;
+      for (int j = 0; j < 8; ++j) v[j] = block_hist[(size_t)(b0 + j) * E + e];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        block_hist[(size_t)(b0 + j) * E + e] = carry;
+        carry += v[j];
       }
-      if (b < nblk) block_hist[(size_t)b * E + e] = carry + incl - v;
-      carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) {
-      tot[e] = carry;
-      counts[e] = carry;
+    for (; b0 < nblk; ++b0) {
+      const int v = block_hist[(size_t)b0 * E + e];
+      block_hist[(size_t)b0 * E + e] = carry;
+      carry += v;
     }
+    tot[e] = carry;
+    counts[e] = carry;
   }
   __syncthreads();
   // exclusive scan of the expert totals (E <= 1024 = blockDim)
