@@ -195,14 +195,17 @@ def recorded_traffic(workload):
 
 
 # ---------------------------------------------------------------- timed runs
-def time_workload(cfg, d, ws, steps, warmup, rank, world, flush, moe, gpu_index, sample_clocks=True):
+TILES = {"auto": 0, "small": 1, "large": 2, "pair": 3}
+
+
+def time_workload(cfg, d, ws, steps, warmup, rank, world, flush, moe, gpu_index, sample_clocks=True, tiles=0):
     import torch
     import torch.distributed as dist
     T = cfg.T
 
     def step(evs=None, info=None):
         return moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws,
-                           d["w_sh_gate_up"], d["w_sh_down"], stage_events=evs, info=info)
+                           d["w_sh_gate_up"], d["w_sh_down"], stage_events=evs, info=info, tiles=tiles)
 
     for _ in range(warmup):
         flush.zero_()
@@ -244,7 +247,7 @@ def time_workload(cfg, d, ws, steps, warmup, rank, world, flush, moe, gpu_index,
                 step_ms_median=statistics.median(step_ms))
 
 
-def time_e2e(cfg, d, ws, steps, warmup, rank, world, moe):
+def time_e2e(cfg, d, ws, steps, warmup, rank, world, moe, tiles=0):
     """Same metric through the public call with host buffers: pinned x in,
     y out, both copies inside the timed region."""
     import torch
@@ -257,7 +260,7 @@ def time_e2e(cfg, d, ws, steps, warmup, rank, world, moe):
     def step():
         x_d.copy_(x_h, non_blocking=True)
         moe.forward(x_d, d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws, d["w_sh_gate_up"],
-                    d["w_sh_down"], out=y_d)
+                    d["w_sh_down"], out=y_d, tiles=tiles)
         y_h.copy_(y_d, non_blocking=True)
 
     for _ in range(warmup):
@@ -336,10 +339,11 @@ def run_ours(args):
     d, _ = device_inputs(cfg, rank)
     ws = moe.alloc_workspace(cfg.T, cfg.H, cfg.E, cfg.I, cfg.k, cfg.I_s)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    main = time_workload(cfg, d, ws, args.steps, args.warmup, rank, world, flush, moe, gpu_index)
+    tiles = TILES[args.tiles]
+    main = time_workload(cfg, d, ws, args.steps, args.warmup, rank, world, flush, moe, gpu_index, tiles=tiles)
     counts = moe.workspace_view(ws, cfg.T, cfg.H, cfg.E, cfg.I, cfg.k, cfg.I_s)["counts"].cpu().numpy()
     acc = layer_accounting(cfg, counts)
-    e2e = time_e2e(cfg, d, ws, args.steps, args.warmup, rank, world, moe)
+    e2e = time_e2e(cfg, d, ws, args.steps, args.warmup, rank, world, moe, tiles=tiles)
 
     def roof(cfg_, res, acc_):
         gate_up_ms = res["stage_ms"][3]
@@ -372,15 +376,39 @@ def run_ours(args):
         d2["x"] = torch.from_numpy(px.view(np.int16)).view(torch.bfloat16).cuda()
         ws2 = moe.alloc_workspace(pcfg.T, pcfg.H, pcfg.E, pcfg.I, pcfg.k, pcfg.I_s)
         pres = time_workload(pcfg, d2, ws2, args.steps, args.warmup, rank, world, flush, moe, gpu_index,
-                             sample_clocks=False)
+                             sample_clocks=False, tiles=tiles)
         pcounts = moe.workspace_view(ws2, pcfg.T, pcfg.H, pcfg.E, pcfg.I, pcfg.k)["counts"].cpu().numpy()
         pacc = layer_accounting(pcfg, pcounts)
-        pe2e = time_e2e(pcfg, d2, ws2, max(3, args.steps // 2), args.warmup, rank, world, moe)
+        pe2e = time_e2e(pcfg, d2, ws2, max(3, args.steps // 2), args.warmup, rank, world, moe, tiles=tiles)
         prefill = {"workload": pcfg.name, "value": round(pres["value"], 1), "unit": "tokens/s",
                    "ms_per_step": round(pres["ms_per_step"], 4), "gpu_launches": pres["launches"],
                    "e2e": {k: (round(v, 1) if isinstance(v, float) else v) for k, v in pe2e.items()},
                    **roof(pcfg, pres, pacc)}
         del ws2
+
+    extra = {}
+    if args.extra:
+        del d
+        torch.cuda.empty_cache()
+        loaded = None
+        for name in args.extra.split(","):
+            ecfg = synth.CONFIGS[name]
+            key = (ecfg.H, ecfg.E, ecfg.I, ecfg.I_s, ecfg.bias)
+            if loaded is None or loaded[0] != key:
+                loaded = None
+                torch.cuda.empty_cache()
+                loaded = (key, device_inputs(ecfg, rank)[0])
+            de = dict(loaded[1])
+            de["x"] = torch.from_numpy(synth.make_x(ecfg.with_(seed=ecfg.seed + rank)).view(np.int16)).view(
+                torch.bfloat16).cuda()
+            wse = moe.alloc_workspace(ecfg.T, ecfg.H, ecfg.E, ecfg.I, ecfg.k, ecfg.I_s)
+            eres = time_workload(ecfg, de, wse, args.steps, args.warmup, rank, world, flush, moe, gpu_index,
+                                 sample_clocks=False, tiles=tiles)
+            ecounts = moe.workspace_view(wse, ecfg.T, ecfg.H, ecfg.E, ecfg.I, ecfg.k, ecfg.I_s)["counts"]
+            eacc = layer_accounting(ecfg, ecounts.cpu().numpy())
+            extra[name] = {"value": round(eres["value"], 1), "unit": "tokens/s",
+                           "ms_per_step": round(eres["ms_per_step"], 4), **roof(ecfg, eres, eacc)}
+            del wse
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -410,6 +438,10 @@ def run_ours(args):
         }
         if prefill:
             line["prefill"] = prefill
+        if extra:
+            line["extra"] = extra
+        if args.tiles != "auto":
+            line["config"]["tiles"] = args.tiles
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -452,6 +484,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=16)
     ap.add_argument("--ref-sample-tokens", type=int, default=2)
+    ap.add_argument("--tiles", choices=sorted(TILES), default="auto", help="grouped GEMM tile policy (tuning)")
+    ap.add_argument("--extra", default="", help="comma-separated further workloads to time, e.g. "
+                                                 "ling_skewed_t4096,sweep_decode_t1")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -17,13 +17,13 @@ from dataclasses import dataclass
 from . import build as _build
 
 __all__ = [
-    "MoEError", "lib", "TILES_AUTO", "TILES_SMALL", "TILES_LARGE", "ROUTER_AUTO", "ROUTER_FMA", "ROUTER_TC",
+    "MoEError", "lib", "TILES_AUTO", "TILES_SMALL", "TILES_LARGE", "TILES_PAIR", "ROUTER_AUTO", "ROUTER_FMA", "ROUTER_TC",
     "workspace_size", "workspace_layout", "alloc_workspace", "route", "permute", "grouped_swiglu",
     "grouped_down", "down_combine", "forward", "device_status", "clear_device_status", "selftest_timeout",
     "STATUS",
 ]
 
-TILES_AUTO, TILES_SMALL, TILES_LARGE = 0, 1, 2
+TILES_AUTO, TILES_SMALL, TILES_LARGE, TILES_PAIR = 0, 1, 2, 3
 ROUTER_AUTO, ROUTER_FMA, ROUTER_TC = 0, 1, 2
 
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_ALIGNMENT", 3: "MOE_ERR_WORKSPACE",

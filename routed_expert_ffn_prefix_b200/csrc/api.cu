@@ -154,7 +154,7 @@ inline Tp* at(void* ws, size_t off) {
 }
 
 int choose_tiles(int policy, long long rows, int groups) {
-  if (policy == MOE_TILES_SMALL || policy == MOE_TILES_LARGE) return policy;
+  if (policy == MOE_TILES_SMALL || policy == MOE_TILES_LARGE || policy == MOE_TILES_PAIR) return policy;
   // mean rows per group: small groups stream weights under few rows
   return rows > 48ll * groups ? MOE_TILES_LARGE : MOE_TILES_SMALL;
 }
@@ -233,6 +233,7 @@ moe_status_t run_swiglu(const uint16_t* x, int src_rows, const uint16_t* w_gate_
   a.split_stride = 0;
   a.status = st;
   a.timeout_ns = kDefaultTimeoutNs;
+  if (tiles == MOE_TILES_PAIR) return cuda_status(launch_grouped_gemm_pair(map, a, EPI_SWIGLU, dev.num_sms, s));
   return cuda_status(launch_grouped_gemm(map, a, EPI_SWIGLU, tiles, dev.num_sms, s));
 }
 
@@ -264,6 +265,7 @@ moe_status_t run_down(const uint16_t* h, const uint16_t* w_down, const int32_t* 
   a.split_stride = 0;
   a.status = st;
   a.timeout_ns = kDefaultTimeoutNs;
+  if (tiles == MOE_TILES_PAIR) return cuda_status(launch_grouped_gemm_pair(map, a, EPI_STORE_F32, dev.num_sms, s));
   return cuda_status(launch_grouped_gemm(map, a, EPI_STORE_F32, tiles, dev.num_sms, s));
 }
 
@@ -361,7 +363,7 @@ moe_status_t moe_grouped_swiglu(const uint16_t* x, const uint16_t* w_gate_up, co
                                 void* stream) {
   if (!all_nonnull(x, w_gate_up, offsets, sorted_token_ids, h)) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_shapes(T, H, E, I, k, true));
-  if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_LARGE) return MOE_ERR_INVALID_ARG;
+  if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_PAIR) return MOE_ERR_INVALID_ARG;
   if (!all_aligned(x, w_gate_up, offsets, sorted_token_ids, h)) return MOE_ERR_ALIGNMENT;
   MOE_TRY(check_ws(workspace, workspace_bytes, sizeof(DevStatus)));
   DeviceInfo dev;
@@ -379,7 +381,7 @@ moe_status_t moe_grouped_down(const uint16_t* h, const uint16_t* w_down, const i
   if (rows < 1 || E < 1 || E > kMaxExperts || H < 1 || I < 1) return MOE_ERR_INVALID_ARG;
   if (offsets == nullptr && E != 1) return MOE_ERR_INVALID_ARG;
   if (H % 256 != 0 || I % 128 != 0) return MOE_ERR_ALIGNMENT;
-  if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_LARGE) return MOE_ERR_INVALID_ARG;
+  if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_PAIR) return MOE_ERR_INVALID_ARG;
   if (!all_aligned(h, w_down, o) || (offsets && !aligned16(offsets))) return MOE_ERR_ALIGNMENT;
   MOE_TRY(check_ws(workspace, workspace_bytes, sizeof(DevStatus)));
   DeviceInfo dev;
@@ -394,7 +396,7 @@ moe_status_t moe_down_combine(const uint16_t* h, const uint16_t* w_down, const f
                               size_t workspace_bytes, void* stream) {
   if (!all_nonnull(h, w_down, topk_w, inv_perm, offsets, y)) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_shapes(T, H, E, I, k, true));
-  if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_LARGE) return MOE_ERR_INVALID_ARG;
+  if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_PAIR) return MOE_ERR_INVALID_ARG;
   if (!all_aligned(h, w_down, topk_w, inv_perm, offsets, y) || (shared_out && !aligned16(shared_out)))
     return MOE_ERR_ALIGNMENT;
   const moe_workspace_layout_t L = make_layout(T, H, E, I, k, 0);
@@ -423,7 +425,7 @@ moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const floa
   }
   const int tile_policy = options ? options->tile_policy : MOE_TILES_AUTO;
   const int router_impl = options ? options->router_impl : MOE_ROUTER_AUTO;
-  if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_LARGE) return MOE_ERR_INVALID_ARG;
+  if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_PAIR) return MOE_ERR_INVALID_ARG;
   if (router_impl < MOE_ROUTER_AUTO || router_impl > MOE_ROUTER_TC) return MOE_ERR_INVALID_ARG;
   if (!all_aligned(x, w_router, w_gate_up, w_down, y) || (bias && !aligned16(bias))) return MOE_ERR_ALIGNMENT;
   const moe_workspace_layout_t L = make_layout(T, H, E, I, k, shared ? I_s : 0);

@@ -1,0 +1,439 @@
+// grouped_gemm_pair.cu -- grouped expert GEMM on SM pairs (tcgen05 cta_group::2).
+//
+// A variant of the grouped GEMM for groups that fill 256-row tiles
+// (grouped_gemm.cu has the design notes shared by both; this one is selected
+// with MOE_TILES_PAIR).  Here the token rows are the MMA's M side and one MMA
+// spans two SMs of a cluster (M = 256: 128 rows in each SM's TMEM), with
+// N = 256 weight columns of which each SM loads half.  The MMA work per
+// weight byte is fixed at the full 256 rows, so groups with fewer rows pay
+// for padding; measured on 512 experts x ~160 rows it is slower than the
+// single-SM kernel, which adapts N to the rows.
+//
+//   * gate/up: N = [128 gate | 128 up] columns of the same 128 intermediate
+//     units, so each thread of the epilogue holds gate and up for its row in
+//     its own TMEM lane: SwiGLU is thread-local and each thread writes 64
+//     contiguous bytes of h per 32-column chunk (16-byte vector stores);
+//   * down: N = 256 adjacent output columns, fp32 rows stored likewise.
+//
+// Per SM and pipeline stage: 128 gathered token rows (16 KB, cp.async,
+// 128-byte swizzle, K-major) + half of the weight tile (16 KB, TMA, MN-major)
+// = 32 KB, so six stages fit, and the accumulator (256 TMEM columns) is
+// double-buffered: the weight stream from HBM never waits for an epilogue.
+// Each SM streams a disjoint half of every weight tile exactly once per
+// 256-row pass.
+//
+// Synchronisation (cluster of 2; rank 0 = leader issues every MMA):
+//   full[s]  (leader): 128 cp.async arrivals of the leader's rows, the
+//            leader's expect_tx for both SMs' weight bytes, and one relayed
+//            arrival from the peer once its rows have landed.  Both SMs' TMA
+//            weight loads complete their bytes on the leader's barrier.
+//   xfull[s] (peer):   the peer's 128 cp.async arrivals; the peer's relay
+//            thread waits on it, fences the writes into the async proxy and
+//            arrives on the leader's full[s].
+//   empty[s], tfull[b] (both): arrived by the leader's commits, multicast to
+//            both SMs of the pair.
+//   tempty[b] (leader): one arrival per epilogue warp of both SMs.
+// Every wait is bounded; both SMs meet at a cluster barrier before TMEM is
+// released and the blocks exit.
+//
+// Warp roles (320 threads): warps 0-7 epilogue, warps 8-11 producers
+// (cp.async rows; thread 0 also issues the weight TMA), warp 12: TMEM
+// allocation, MMA issue (leader) or completion relay (peer).
+#include "gemm_units.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kPNt = 256;       // token rows per pair unit (128 per SM)
+constexpr int kPRows = 128;     // token rows per SM
+constexpr int kPStages = 6;
+constexpr int kPEpiWarps = 8;
+constexpr int kPProdWarps = 4;
+constexpr int kPCtlWarp = kPEpiWarps + kPProdWarps;
+constexpr int kPThreads = (kPCtlWarp + 1) * 32;
+constexpr int kPProdThreads = kPProdWarps * 32;
+constexpr int kPXBytes = kPRows * kBK * 2;   // 16 KB of rows per stage
+constexpr int kPWBytes = 128 * kBK * 2;      // 16 KB: this SM's half of the weight tile
+constexpr int kPStageBytes = kPXBytes + kPWBytes;
+constexpr int kPAccCols = 256;
+constexpr int kPTmemCols = 512;              // two accumulator buffers
+constexpr int kPSmemBytes = kPStages * kPStageBytes + 512 + 4 * (kMaxExperts + 1) + 1024;
+static_assert(kPSmemBytes <= 232448, "shared memory budget");
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t out;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(saddr), "r"(rank));
+  return out;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void remote_arrive(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Relayed "rows landed" signal.  The rows were written to this SM's own
+// shared memory and are read by this SM's own tensor core (each SM computes
+// its half of M from its own A tile), and they have fully landed before the
+// relay observes its local barrier; a release at cluster scope here costs
+// about 1,300 cycles per stage (measured) and would pace the whole pipeline,
+// so the arrive is relaxed, after a proxy fence for the tensor core's reads.
+__device__ __forceinline__ void remote_arrive_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// TMA tile load whose completion is signalled on a barrier of either SM of the pair.
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
+                                                 int c1, int c2, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on the barrier at this smem offset in both SMs of the pair once the
+// MMAs issued so far have completed.
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"((uint16_t)3)
+      : "memory");
+}
+
+// Arrive on the leader's barrier (rank 0 only) once the MMAs issued so far have completed.
+__device__ __forceinline__ void mma_commit_pair_leader(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"((uint16_t)1)
+      : "memory");
+}
+
+__device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kPThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap wmap, const GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPStages * kPStageBytes);
+  uint64_t* xfull = full + kPStages;
+  uint64_t* empty = xfull + kPStages;
+  uint64_t* tfull = empty + kPStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int* total_units = abort_flag + 1;
+  int* ustart = reinterpret_cast<int*>(smem + kPStages * kPStageBytes + 512);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int ngroups = a.offsets ? a.groups : 1;
+
+  if (tid == 0) {
+    for (int s = 0; s < kPStages; ++s) {
+      mbar_init(full + s, kPProdThreads + 2);  // leader rows + leader expect_tx + peer relay
+      mbar_init(xfull + s, kPProdThreads);     // peer rows
+      mbar_init(empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull + b, 1);
+      mbar_init(tempty + b, 2 * kPEpiWarps);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) build_unit_prefix<kPNt>(a, ngroups, ustart, total_units);
+  if (warp == kPCtlWarp) {
+    tmem_alloc_pair(tmem_slot, kPTmemCols);
+    tmem_relinquish_pair();
+  }
+  if (warp == kPEpiWarps && lane == 0) prefetch_tmap(&wmap);
+  tc_fence_before();
+  cluster_sync();  // barriers of both SMs initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int total = *total_units;
+
+  if (warp >= kPEpiWarps && warp < kPCtlWarp) {
+    // ------------------------------------------------------------ producers
+    const WaitCtx wc{a.status, abort_flag, a.timeout_ns, SITE_GEMM_PRODUCER};
+    const int pt = tid - kPEpiWarps * 32;
+    const int chunk = pt & 7, rsub = pt >> 3;
+    constexpr int kRowsPerThread = kPRows / (kPProdThreads / 8);
+    const uint64_t pol_w = policy_evict_first();
+    const __nv_bfloat16* bsrc = reinterpret_cast<const __nv_bfloat16*>(a.b_src);
+    uint64_t* rows_bar_base = leader ? full : xfull;
+    const uint32_t full_leader = map_to_rank(smem_u32(full), 0);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int u = pair; u < total && ok; u += npairs) {
+      const Unit un = decode_unit<kPNt>(a, ustart, ngroups, u);
+      const int my0 = (int)rank * kPRows;  // this SM's first row of the unit
+      int src[kRowsPerThread];
+#pragma unroll
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        const int c = my0 + rsub + 16 * i;
+        int sr = -1;
+        if (c < un.rows) {
+          const int r = un.row0 + c;
+          sr = a.row_index ? __ldg(a.row_index + r) : r;
+          if (sr < 0 || sr >= a.src_rows) {
+            raise_error(a.status, MOE_ERR_DEVICE_BOUNDS, SITE_GEMM_GATHER, r);
+            sr = -1;
+          }
+        }
+        src[i] = sr;
+      }
+      const int wcol = un.nb * a.col_stride + (int)rank * a.col1_off;  // this SM's weight-column half
+      const int nk = un.ke - un.kb, kiters = nk * a.krep;
+      for (int it = 0; it < kiters; ++it) {
+        const int rep = it / nk, kt = un.kb + (it - rep * nk);
+        if (!mbar_wait(&empty[stage], phase ^ 1u, wc, 100 + stage)) { ok = false; break; }
+        uint8_t* sX = smem + stage * kPStageBytes;
+        uint8_t* sW = sX + kPXBytes;
+        const uint32_t sx = smem_u32(sX);
+#pragma unroll
+        for (int i = 0; i < kRowsPerThread; ++i) {
+          if (src[i] >= 0) {
+            const int c = rsub + 16 * i;
+            cp_async_16(sx + c * 128 + ((chunk ^ (c & 7)) << 4), bsrc + (size_t)src[i] * a.K + kt * kBK + chunk * 8);
+          }
+        }
+        cp_async_arrive_noinc(&rows_bar_base[stage]);
+        if (pt == 0) {
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kPWBytes);
+          const int d2 = a.a_dim2_rep ? rep : un.group;
+          const uint32_t fb = full_leader + stage * 8;
+          tma_load_3d_pair(sW, &wmap, fb, wcol, kt * kBK, d2, pol_w);
+          tma_load_3d_pair(sW + kPWBytes / 2, &wmap, fb, wcol + 64, kt * kBK, d2, pol_w);
+        }
+        if (++stage == kPStages) { stage = 0; phase ^= 1u; }
+      }
+    }
+    cp_async_wait_all();
+    if (!ok && pt == 0) {
+      // Aborted: weight tiles this SM requested may still be landing in its
+      // shared memory (their completion is counted on the leader); give them
+      // time to arrive before the block can exit.
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 50000ull) {
+      }
+    }
+  } else if (warp == kPCtlWarp) {
+    if (leader) {
+      // ---------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        const WaitCtx wc{a.status, abort_flag, a.timeout_ns, SITE_GEMM_MMA};
+        // A = token rows (K-major), B = weights (MN-major), M = 256 over the pair, N = 256.
+        const uint32_t idesc = idesc_bf16_f32(256, 256, false, true);
+        int stage = 0;
+        uint32_t phase = 0;
+        int acc_it = 0;
+        bool ok = true;
+        for (int u = pair; u < total && ok; u += npairs) {
+          const Unit un = decode_unit<kPNt>(a, ustart, ngroups, u);
+          const int buf = acc_it & 1;
+          const uint32_t apar = (acc_it >> 1) & 1;
+          if (!mbar_wait(&tempty[buf], apar ^ 1u, wc, 200 + buf)) break;
+          tc_fence_after();
+          const uint32_t d = tmem + buf * kPAccCols;
+          const int kiters = (un.ke - un.kb) * a.krep;
+          uint32_t acc = 0;
+          for (int it = 0; it < kiters; ++it) {
+            if (!mbar_wait(&full[stage], phase, wc, 300 + stage)) { ok = false; break; }
+            tc_fence_after();
+            fence_proxy_async_smem();
+            const uint32_t sx = smem_u32(smem + stage * kPStageBytes), sw = sx + kPXBytes;
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t ad = smem_desc_sw128(sx + kk * 32, 16, 1024);     // rows: +16 k = 32 B
+              const uint64_t bd = smem_desc_sw128(sw + kk * 2048, 8192, 1024); // weights: +16 k = 2048 B
+              mma_bf16_pair(d, ad, bd, idesc, acc);
+              acc = 1;
+            }
+            mma_commit_pair(&empty[stage]);
+            if (++stage == kPStages) { stage = 0; phase ^= 1u; }
+          }
+          if (!ok) break;
+          mma_commit_pair(&tfull[buf]);
+          ++acc_it;
+        }
+        mma_commit_pair_leader(mma_done);
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(mma_done, 0) && globaltimer_ns() - t0 < a.timeout_ns) {
+        }
+      }
+    } else if (lane == 0) {
+      // ---------------------------------------------------------- peer relay
+      // Forward "this SM's rows of stage s have landed" to the leader.
+      const WaitCtx wc{a.status, abort_flag, a.timeout_ns, SITE_GEMM_PRODUCER};
+      const uint32_t full_leader = map_to_rank(smem_u32(full), 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = pair; u < total && ok; u += npairs) {
+        const Unit un = decode_unit<kPNt>(a, ustart, ngroups, u);
+        const int kiters = (un.ke - un.kb) * a.krep;
+        for (int it = 0; it < kiters; ++it) {
+          if (!mbar_wait(&xfull[stage], phase, wc, 500 + stage)) { ok = false; break; }
+          fence_proxy_async_smem();
+          remote_arrive_relaxed(full_leader + stage * 8);
+          if (++stage == kPStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 0-7)
+    // Warp w reads TMEM lanes 32*(w%4).. = rows 32*(w%4).. of this SM's 128,
+    // and the column half (w/4): one row per thread, contiguous columns.
+    const WaitCtx wc{a.status, abort_flag, a.timeout_ns, SITE_GEMM_EPILOGUE};
+    const int quarter = warp & 3, half = warp >> 2;
+    const uint32_t tempty_leader = map_to_rank(smem_u32(tempty), 0);
+    int acc_it = 0;
+    for (int u = pair; u < total; u += npairs) {
+      const Unit un = decode_unit<kPNt>(a, ustart, ngroups, u);
+      const int buf = acc_it & 1;
+      const uint32_t apar = (acc_it >> 1) & 1;
+      if (!mbar_wait(&tfull[buf], apar, wc, 400 + buf)) break;
+      tc_fence_after();
+      const int my0 = (int)rank * kPRows;
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * kPAccCols;
+      const int row_in_unit = my0 + quarter * 32 + lane;
+      const bool row_ok = row_in_unit < un.rows;
+      const size_t grow = (size_t)(un.row0 + row_in_unit);
+      if (my0 + quarter * 32 < un.rows) {  // skip warps whose 32 rows are all padding
+        if (EPI == EPI_SWIGLU) {
+          // columns [half*64, half*64+64) of gate (TMEM 0..127) and of up (TMEM 128..255)
+          const int col0 = un.nb * a.out_col_stride + half * 64;
+          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + grow * a.ld_out + col0;
+#pragma unroll
+          for (int c = 0; c < 64; c += 32) {
+            float g[32], v[32];
+            const uint32_t tg = tbase + half * 64 + c, tu = tbase + 128 + half * 64 + c;
+            tmem_ld_4x16(tg, tg + 16, tu, tu + 16, g, g + 16, v, v + 16);
+            if (row_ok && col0 + c < a.n_valid) {
+#pragma unroll
+              for (int q = 0; q < 32; q += 8) {
+                st_global_v4(out + c + q, pack_bf16x2(silu_f(g[q]) * v[q], silu_f(g[q + 1]) * v[q + 1]),
+                             pack_bf16x2(silu_f(g[q + 2]) * v[q + 2], silu_f(g[q + 3]) * v[q + 3]),
+                             pack_bf16x2(silu_f(g[q + 4]) * v[q + 4], silu_f(g[q + 5]) * v[q + 5]),
+                             pack_bf16x2(silu_f(g[q + 6]) * v[q + 6], silu_f(g[q + 7]) * v[q + 7]));
+              }
+            }
+          }
+        } else {
+          // output columns [half*128, half*128+128) of the unit's 256
+          const int col0 = un.nb * a.out_col_stride + half * 128;
+          float* out = reinterpret_cast<float*>(a.out) + (size_t)un.ks * a.split_stride + grow * a.ld_out + col0;
+#pragma unroll
+          for (int c = 0; c < 128; c += 32) {
+            float v[32];
+            tmem_ld_2x16(tbase + half * 128 + c, tbase + half * 128 + c + 16, v, v + 16);
+            if (row_ok && col0 + c < a.n_valid) {
+#pragma unroll
+              for (int q = 0; q < 32; q += 4)
+                st_global_v4(out + c + q, __float_as_uint(v[q]), __float_as_uint(v[q + 1]),
+                             __float_as_uint(v[q + 2]), __float_as_uint(v[q + 3]));
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) remote_arrive(tempty_leader + buf * 8);
+      ++acc_it;
+    }
+  }
+
+  // Both SMs finish every access to each other's shared memory and barriers
+  // before TMEM is released and either block exits.
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == kPCtlWarp) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kPTmemCols);
+  }
+}
+
+template <int EPI>
+cudaError_t launch_pair(const CUtensorMap& wmap, const GemmArgs& a, int num_sms, cudaStream_t stream) {
+  auto kern = grouped_gemm_pair_kernel<EPI>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmemBytes);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kPThreads, 1, 1);
+  cfg.dynamicSmemBytes = kPSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // One pair per co-resident cluster slot (persistent).
+  cfg.gridDim = dim3(num_sms & ~1, 1, 1);
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) == cudaSuccess && clusters > 0 &&
+      2 * clusters < (int)cfg.gridDim.x)
+    cfg.gridDim = dim3(2 * clusters, 1, 1);
+  return cudaLaunchKernelEx(&cfg, kern, wmap, a);
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_gemm_pair(const CUtensorMap& wmap, const GemmArgs& a, int epilogue, int num_sms,
+                                     cudaStream_t stream) {
+  return epilogue == EPI_SWIGLU ? launch_pair<EPI_SWIGLU>(wmap, a, num_sms, stream)
+                                : launch_pair<EPI_STORE_F32>(wmap, a, num_sms, stream);
+}
+
+}  // namespace moe

@@ -45,6 +45,13 @@ enum Epilogue { EPI_SWIGLU = 0, EPI_STORE_F32 = 1 };
 // for units of 128 * that many columns.
 int gemm_tiles_per_unit(int tiles, int epilogue);
 
+// Large-row groups on SM pairs (grouped_gemm_pair.cu): 256 token rows per
+// unit, two 128-column weight tiles per unit (the same n_blocks/col_stride/
+// col1_off/out_col_stride as the single-SM kernel with two tiles per unit);
+// output columns must come in whole chunks of 32 (n_valid % 32 == 0).
+cudaError_t launch_grouped_gemm_pair(const CUtensorMap& wmap, const GemmArgs& a, int epilogue, int num_sms,
+                                     cudaStream_t stream);
+
 // tiles: MOE_TILES_SMALL or MOE_TILES_LARGE.
 cudaError_t launch_grouped_gemm(const CUtensorMap& wmap, const GemmArgs& a, int epilogue, int tiles,
                                 int num_sms, cudaStream_t stream);

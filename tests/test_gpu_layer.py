@@ -102,7 +102,7 @@ def test_permute_random_ids_large():
         np.testing.assert_array_equal(g.cpu().numpy().reshape(w.shape), w)
 
 
-@pytest.mark.parametrize("tiles", [moe.TILES_SMALL, moe.TILES_LARGE])
+@pytest.mark.parametrize("tiles", [moe.TILES_SMALL, moe.TILES_LARGE, moe.TILES_PAIR])
 @pytest.mark.parametrize("name", list(CASES))
 def test_grouped_swiglu_matches_oracle(name, tiles):
     cfg, inp, ref = case(name)
@@ -114,7 +114,7 @@ def test_grouped_swiglu_matches_oracle(name, tiles):
     assert_close_output(host_f64(h), ref["h"], "h")
 
 
-@pytest.mark.parametrize("tiles", [moe.TILES_SMALL, moe.TILES_LARGE])
+@pytest.mark.parametrize("tiles", [moe.TILES_SMALL, moe.TILES_LARGE, moe.TILES_PAIR])
 @pytest.mark.parametrize("name", list(CASES))
 def test_down_combine_matches_oracle(name, tiles):
     """Fed a synthetic h (not the GPU's): y = sum_j w o[inv_perm] + shared."""
@@ -143,7 +143,7 @@ def test_grouped_down_single_group():
 
 
 @pytest.mark.parametrize("router", [moe.ROUTER_FMA, moe.ROUTER_TC])
-@pytest.mark.parametrize("tiles", [moe.TILES_SMALL, moe.TILES_LARGE])
+@pytest.mark.parametrize("tiles", [moe.TILES_SMALL, moe.TILES_LARGE, moe.TILES_PAIR])
 @pytest.mark.parametrize("name", list(CASES))
 def test_forward_matches_oracle(name, tiles, router):
     cfg, inp, ref = case(name)
@@ -171,13 +171,13 @@ def test_forward_bitwise_deterministic():
     d = dev_inputs(inp)
     ws = workspace(cfg)
     ys = []
-    for _ in range(3):
+    for i in range(4):
         ys.append(moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws,
-                              tiles=moe.TILES_LARGE).cpu())
+                              tiles=moe.TILES_LARGE if i < 2 else moe.TILES_PAIR).cpu())
         moe.forward(d["x"][:7], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k,
                     moe.alloc_workspace(7, cfg.H, cfg.E, cfg.I, cfg.k))
     assert_ok(ws)
-    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[0], ys[2])
+    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[2], ys[3])
 
 
 def test_all_tokens_to_the_same_experts():
@@ -188,7 +188,7 @@ def test_all_tokens_to_the_same_experts():
     ref = oracle.layer_forward(inp.x, inp.w_router, inp.bias, inp.w_gate_up, inp.w_down, cfg.k)
     assert ref["counts"].tolist() == [300, 300, 0, 0, 0, 0, 0, 0]
     d = dev_inputs(inp)
-    for tiles in (moe.TILES_SMALL, moe.TILES_LARGE):
+    for tiles in (moe.TILES_SMALL, moe.TILES_LARGE, moe.TILES_PAIR):
         ws = workspace(cfg)
         y = moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws, tiles=tiles)
         assert_ok(ws)
