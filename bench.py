@@ -198,28 +198,54 @@ def recorded_traffic(workload):
 TILES = {"auto": 0, "small": 1, "large": 2, "pair": 3}
 
 
-def time_workload(cfg, d, ws, steps, warmup, rank, world, flush, moe, gpu_index, sample_clocks=True, tiles=0):
+def time_workload(cfg, d, ws, steps, warmup, rank, world, flush, moe, gpu_index, sample_clocks=True, tiles=0,
+                  graph=False):
+    """K timed steps (L2 flushed before each).  graph=True captures one layer
+    call in a CUDA graph and replays it per step (no host launch overhead);
+    otherwise every step is an eager library call."""
     import torch
     import torch.distributed as dist
     T = cfg.T
+    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
 
     def step(evs=None, info=None):
         return moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws,
-                           d["w_sh_gate_up"], d["w_sh_down"], stage_events=evs, info=info, tiles=tiles)
+                           d["w_sh_gate_up"], d["w_sh_down"], stage_events=evs, info=info, tiles=tiles, out=out)
+
+    def events(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for ev in evs:  # torch creates an event on its first record; the library re-records the same handle
+            ev.record()
+        return evs
 
     for _ in range(warmup):
         flush.zero_()
         step()
     torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(warmup):
+        step()
+    host_us = (time.perf_counter() - t0) / warmup * 1e6  # host time per eager call (enqueue only)
+    torch.cuda.synchronize()
     st = moe.device_status(ws)
     if st != 0:
         raise RuntimeError(f"device status {moe.STATUS.get(st, st)} after warm-up")
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(steps)]
-    for row in evs:  # torch creates an event on its first record; the library re-records the same handle
-        for ev in row:
-            ev.record()
-    torch.cuda.synchronize()
     info = {}
+    g = None
+    if graph:
+        # An event recorded while a stream is captured only orders work inside
+        # the graph (no timestamp at replay), so graph mode times whole steps.
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(None, info)
+        for _ in range(warmup):
+            flush.zero_()
+            g.replay()
+        torch.cuda.synchronize()
+        ends = [events(2) for _ in range(steps)]
+    else:
+        evs = [events(7) for _ in range(steps)]
+        torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -227,24 +253,34 @@ def time_workload(cfg, d, ws, steps, warmup, rank, world, flush, moe, gpu_index,
     if clk:
         clk.start()
         time.sleep(0.3)
+    stage_ms = []
     for i in range(steps):
         flush.zero_()  # L2 flush between steps, outside the timed events
-        step(evs[i], info)
+        if graph:
+            ends[i][0].record()
+            g.replay()
+            ends[i][1].record()
+        else:
+            step(evs[i], info)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = clk.stop() if clk else None
-    step_ms = [e[0].elapsed_time(e[6]) for e in evs]
-    stage_ms = [[e[j].elapsed_time(e[j + 1]) for j in range(6)] for e in evs]
+    if graph:
+        step_ms = [e[0].elapsed_time(e[1]) for e in ends]
+    else:
+        step_ms = [e[0].elapsed_time(e[6]) for e in evs]
+        stage_ms = [[e[j].elapsed_time(e[j + 1]) for j in range(6)] for e in evs]
     total_ms = sum(step_ms)
     if world > 1:
         t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
-    mean_stage = [statistics.mean(s[j] for s in stage_ms) for j in range(6)]
+    mean_stage = [statistics.mean(s[j] for s in stage_ms) for j in range(6)] if stage_ms else None
+    del g
     return dict(total_ms=total_ms, ms_per_step=total_ms / steps, value=T * world * steps / (total_ms / 1e3),
                 stage_ms=mean_stage, launches=info.get("launches", 0) * steps, clocks=clocks,
-                step_ms_median=statistics.median(step_ms))
+                step_ms_median=statistics.median(step_ms), host_us_per_call=host_us)
 
 
 def time_e2e(cfg, d, ws, steps, warmup, rank, world, moe, tiles=0):
@@ -404,10 +440,18 @@ def run_ours(args):
             wse = moe.alloc_workspace(ecfg.T, ecfg.H, ecfg.E, ecfg.I, ecfg.k, ecfg.I_s)
             eres = time_workload(ecfg, de, wse, args.steps, args.warmup, rank, world, flush, moe, gpu_index,
                                  sample_clocks=False, tiles=tiles)
+            gres = time_workload(ecfg, de, wse, args.steps, args.warmup, rank, world, flush, moe, gpu_index,
+                                 sample_clocks=False, tiles=tiles, graph=True)
             ecounts = moe.workspace_view(wse, ecfg.T, ecfg.H, ecfg.E, ecfg.I, ecfg.k, ecfg.I_s)["counts"]
             eacc = layer_accounting(ecfg, ecounts.cpu().numpy())
             extra[name] = {"value": round(eres["value"], 1), "unit": "tokens/s",
-                           "ms_per_step": round(eres["ms_per_step"], 4), **roof(ecfg, eres, eacc)}
+                           "ms_per_step": round(eres["ms_per_step"], 4),
+                           "host_us_per_call": round(eres["host_us_per_call"], 1),
+                           "graph": {"value": round(gres["value"], 1), "ms_per_step": round(gres["ms_per_step"], 4),
+                                     "layer_roofline_frac": round(
+                                         roof(ecfg, eres, eacc)["layer_roofline"]["t_roofline_ms"]
+                                         / gres["ms_per_step"], 4)},
+                           **roof(ecfg, eres, eacc)}
             del wse
 
     cpu = None
@@ -431,6 +475,7 @@ def run_ours(args):
                        "l2": "flushed (256 MiB write) before every timed step; expert weights "
                              f"{synth.expert_weight_bytes(cfg) / 1e9:.1f} GB > 126 MB L2"},
             **out_main,
+            "host_us_per_call": round(main["host_us_per_call"], 1),
             "e2e": {k: (round(v, 1) if isinstance(v, float) else v) for k, v in e2e.items()},
             "gpu_launches": main["launches"],
             "clocks": main["clocks"],

@@ -84,7 +84,38 @@ EncodeTiledFn encode_fn() {
 }
 
 // bf16 tensor [d2][d1][d0] (d0 contiguous), box 64 x 64 x 1, 128-byte swizzle.
+// A descriptor depends only on (address, extents), so the last few are
+// memoised: a steady stream of calls on the same weights skips the encode.
+struct MapCacheEntry {
+  const void* base;
+  uint64_t d0, d1, d2;
+  CUtensorMap map;
+};
+constexpr int kMapCache = 16;
+std::mutex g_map_mutex;
+MapCacheEntry g_map_cache[kMapCache];
+int g_map_next = 0;
+
+bool encode_weight_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2);
+
 bool make_weight_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2) {
+  {
+    std::lock_guard<std::mutex> lock(g_map_mutex);
+    for (const MapCacheEntry& e : g_map_cache) {
+      if (e.base == base && e.d0 == d0 && e.d1 == d1 && e.d2 == d2) {
+        *m = e.map;
+        return true;
+      }
+    }
+  }
+  if (!encode_weight_map(m, base, d0, d1, d2)) return false;
+  std::lock_guard<std::mutex> lock(g_map_mutex);
+  g_map_cache[g_map_next] = MapCacheEntry{base, d0, d1, d2, *m};
+  g_map_next = (g_map_next + 1) % kMapCache;
+  return true;
+}
+
+bool encode_weight_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {d0, d1, d2};

@@ -9,7 +9,8 @@
 // to bf16 once.  A fixed summation order makes y bitwise reproducible
 // run to run, whatever order the expert GEMM tiles finished in.
 //
-// Memory-bound: one block per token, float4 loads along H.
+// Memory-bound: a block per (token, 1024-column slice), one float4 per
+// thread, the k slot loads of a thread issued together.
 #include "kernels.h"
 
 namespace moe {
@@ -21,8 +22,8 @@ constexpr int kThreads = 256;
 __global__ void __launch_bounds__(kThreads) combine_kernel(const float* __restrict__ o, const float* __restrict__ w,
                                                          const int32_t* __restrict__ inv_perm,
                                                          const float* __restrict__ shared, int H, int k, int rows,
-                                                         __nv_bfloat16* __restrict__ y, DevStatus* st) {
-  const int t = blockIdx.x;
+                                                         __nv_bfloat16* __restrict__ y, DevStatus* st, int t0) {
+  const int t = t0 + blockIdx.y;
   __shared__ int32_t srow[64];
   __shared__ float sw[64];
   __shared__ int bad;
@@ -40,8 +41,9 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const float* __restri
   __syncthreads();
   if (bad) return;
   const int H4 = H >> 2;
-  for (int c = threadIdx.x; c < H4; c += blockDim.x) {
+  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < H4; c += gridDim.x * blockDim.x) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
     for (int j = 0; j < k; ++j) {
       const float4 v = __ldcs(reinterpret_cast<const float4*>(o + (size_t)srow[j] * H) + c);
       const float wj = sw[j];
@@ -71,9 +73,19 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const float* __restri
 cudaError_t launch_combine(const float* o, const float* topk_w, const int32_t* inv_perm, const float* shared, int T,
                            int H, int k, int rows, uint16_t* y, DevStatus* st, cudaStream_t s) {
   if (k > 64) return cudaErrorInvalidValue;
-  combine_kernel<<<T, kThreads, 0, s>>>(o, topk_w, inv_perm, shared, H, k, rows,
-                                        reinterpret_cast<__nv_bfloat16*>(y), st);
-  return cudaGetLastError();
+  // Few tokens: split each row over several blocks so every SM has work;
+  // many tokens: one block per token, each thread looping over its float4s.
+  const int slices_max = (H / 4 + kThreads - 1) / kThreads;
+  int slices = (2 * 148 + T - 1) / T;
+  slices = slices < 1 ? 1 : (slices > slices_max ? slices_max : slices);
+  for (int t0 = 0; t0 < T; t0 += 65535) {  // grid.y limit
+    const dim3 grid(slices, T - t0 < 65535 ? T - t0 : 65535);
+    combine_kernel<<<grid, kThreads, 0, s>>>(o, topk_w, inv_perm, shared, H, k, rows,
+                                             reinterpret_cast<__nv_bfloat16*>(y), st, t0);
+    const cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace moe

@@ -297,7 +297,10 @@ template <int NT, int ST, int MT, int EPI>
 cudaError_t launch_cfg(const CUtensorMap& wmap, const GemmArgs& a, int num_sms, cudaStream_t stream) {
   using C = Cfg<NT, ST, MT>;
   auto kern = grouped_gemm_kernel<NT, ST, MT, EPI>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  static std::atomic<int> configured[kMaxDevices];
+  cudaError_t err = once_per_device(configured, [&] {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  });
   if (err != cudaSuccess) return err;
   kern<<<num_sms, kThreads, C::SMEM_BYTES, stream>>>(wmap, a);
   return cudaGetLastError();

@@ -406,7 +406,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
 template <int EPI>
 cudaError_t launch_pair(const CUtensorMap& wmap, const GemmArgs& a, int num_sms, cudaStream_t stream) {
   auto kern = grouped_gemm_pair_kernel<EPI>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmemBytes);
+  static std::atomic<int> configured[kMaxDevices];
+  cudaError_t err = once_per_device(configured, [&] {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmemBytes);
+  });
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kPThreads, 1, 1);
@@ -419,12 +422,21 @@ cudaError_t launch_pair(const CUtensorMap& wmap, const GemmArgs& a, int num_sms,
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  // One pair per co-resident cluster slot (persistent).
+  // One pair per co-resident cluster slot (persistent); the slot count is
+  // queried once per device.
+  static std::atomic<int> queried[kMaxDevices];
+  static int slots[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
   cfg.gridDim = dim3(num_sms & ~1, 1, 1);
-  int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) == cudaSuccess && clusters > 0 &&
-      2 * clusters < (int)cfg.gridDim.x)
-    cfg.gridDim = dim3(2 * clusters, 1, 1);
+  if (dev >= 0 && dev < kMaxDevices) {
+    once_per_device(queried, [&] {
+      int clusters = 0;
+      slots[dev] = (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) == cudaSuccess) ? clusters : 0;
+      return cudaSuccess;
+    });
+    if (slots[dev] > 0 && 2 * slots[dev] < (int)cfg.gridDim.x) cfg.gridDim = dim3(2 * slots[dev], 1, 1);
+  }
   return cudaLaunchKernelEx(&cfg, kern, wmap, a);
 }
 

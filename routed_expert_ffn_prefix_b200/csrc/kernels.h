@@ -5,11 +5,28 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "common.cuh"
 
 namespace moe {
 
 constexpr int kMaxExperts = 1024;
+constexpr int kMaxDevices = 64;
+
+// Runs `setup` once per (call site, device): kernel attributes and occupancy
+// queries are per device and never change, so they stay off the per-call path.
+template <typename F>
+inline cudaError_t once_per_device(std::atomic<int>* done, F&& setup) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDevices) return setup();
+  if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  err = setup();
+  if (err == cudaSuccess) done[dev].store(1, std::memory_order_release);
+  return err;
+}
 
 // Arguments of the grouped GEMM (see grouped_gemm.cu).  "Rows" are token
 // rows (the MMA's N side); "columns" are weight columns (the MMA's M side).

@@ -21,6 +21,9 @@
 //               the same expert are ranked by __match_any_sync, so a slot's
 //               row = offsets[e] + earlier slots of e in earlier blocks, runs
 //               and lanes.
+// Up to 8192 slots (decode-sized batches) the three steps run in one block
+// of 32 warps instead (one launch): per-warp histograms in shared memory,
+// a block scan, and the same in-order warp walk.
 #include "kernels.h"
 
 namespace moe {
@@ -153,6 +156,85 @@ __global__ void __launch_bounds__(kScatterWarps * 32) scatter_kernel(const int32
   }
 }
 
+constexpr int kFusedWarps = 32;
+constexpr int kFusedMaxSlots = kFusedWarps * kRun;  // 8192
+
+// Whole permutation in one block (n <= kFusedMaxSlots): warp w owns slots
+// [w*kRun, (w+1)*kRun).
+__global__ void __launch_bounds__(kFusedWarps * 32) permute_fused_kernel(const int32_t* __restrict__ ids, int n, int E,
+                                                                       int k, int32_t* __restrict__ counts,
+                                                                       int32_t* __restrict__ offsets,
+                                                                       int32_t* __restrict__ sorted_ids,
+                                                                       int32_t* __restrict__ inv_perm, DevStatus* st) {
+  extern __shared__ int32_t wh[];  // [kFusedWarps][E] counts, then bases
+  __shared__ int32_t warp_sums[32];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  for (int i = tid; i < kFusedWarps * E; i += blockDim.x) wh[i] = 0;
+  __syncthreads();
+  const int s0 = w * kRun;
+  for (int i = lane; i < kRun; i += 32) {
+    const int s = s0 + i;
+    if (s < n) {
+      const int e = ids[s];
+      if (e < 0 || e >= E) raise_error(st, MOE_ERR_DEVICE_BOUNDS, SITE_PERMUTE_IDS, s);
+      else atomicAdd(&wh[w * E + e], 1);
+    }
+  }
+  __syncthreads();
+  // per expert (thread e): rows of e owned by earlier warps, and the total
+  int tot = 0;
+  if (tid < E) {
+    for (int j = 0; j < kFusedWarps; ++j) {
+      const int c = wh[j * E + tid];
+      wh[j * E + tid] = tot;
+      tot += c;
+    }
+    counts[tid] = tot;
+  }
+  // exclusive scan of the totals over experts (E <= 1024 = blockDim)
+  int incl = tot;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += o;
+  }
+  if (lane == 31) warp_sums[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int ws = warp_sums[lane];
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, ws, d);
+      if (lane >= d) ws += o;
+    }
+    warp_sums[lane] = ws;
+  }
+  __syncthreads();
+  const int excl = incl - tot + (w > 0 ? warp_sums[w - 1] : 0);
+  if (tid < E) {
+    offsets[tid] = excl;
+    if (tid == E - 1) offsets[E] = excl + tot;
+    for (int j = 0; j < kFusedWarps; ++j) wh[j * E + tid] += excl;
+  }
+  __syncthreads();
+  int* mine = wh + w * E;
+  for (int r = 0; r < kRun; r += 32) {
+    const int s = s0 + r + lane;
+    int e = s < n ? ids[s] : -1;
+    if (e >= E) e = -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    const int pos = e >= 0 ? mine[e] + rank : -1;
+    __syncwarp();
+    if (e >= 0 && rank == 0) mine[e] += __popc(peers);
+    __syncwarp();
+    if (e >= 0) {
+      sorted_ids[pos] = s / k;
+      inv_perm[s] = pos;
+    }
+  }
+}
+
 }  // namespace
 
 int permute_num_blocks(int T, int k) { return (T * k + kChunk - 1) / kChunk; }
@@ -161,6 +243,17 @@ cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* cou
                            int32_t* sorted_ids, int32_t* inv_perm, int32_t* block_hist, DevStatus* st,
                            cudaStream_t s) {
   const int n = T * k;
+  if (n <= kFusedMaxSlots) {
+    const size_t sh = (size_t)kFusedWarps * E * sizeof(int32_t);
+    static std::atomic<int> configured[kMaxDevices];
+    cudaError_t err = once_per_device(configured, [&] {
+      return cudaFuncSetAttribute(permute_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)((size_t)kFusedWarps * kMaxExperts * sizeof(int32_t)));
+    });
+    if (err != cudaSuccess) return err;
+    permute_fused_kernel<<<1, kFusedWarps * 32, sh, s>>>(ids, n, E, k, counts, offsets, sorted_ids, inv_perm, st);
+    return cudaGetLastError();
+  }
   const int nblk = permute_num_blocks(T, k);
   hist_kernel<<<nblk, 256, (size_t)E * sizeof(int32_t), s>>>(ids, n, E, block_hist, st);
   cudaError_t err = cudaGetLastError();

@@ -89,32 +89,54 @@ __global__ void __launch_bounds__(kFmaThreads) router_logits_fma_kernel(const __
 }
 
 constexpr int kTopkWarps = 8;
-constexpr int kPerLane = kMaxExperts / 32;
 
+// One warp per token; EPL = experts per lane (E <= 32 * EPL).  The K-split
+// partial slabs are summed in slab order; UNR slabs are loaded before any is
+// added so that UNR * EPL loads per lane are in flight at once.
+template <int EPL, int UNR>
 __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __restrict__ logits, int nsplit,
-                                                             size_t split_stride,
-                                                             const float* __restrict__ bias, int T, int E,
-                                                             int k, int32_t* __restrict__ ids,
+                                                             size_t split_stride, const float* __restrict__ bias,
+                                                             int T, int E, int k, int32_t* __restrict__ ids,
                                                              float* __restrict__ wout, DevStatus* st) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kTopkWarps + warp;
   if (t >= T) return;
   const float* row = logits + (size_t)t * E;
-  float v[kPerLane];
   const float NEG = -INFINITY;
+  float v[EPL];
 #pragma unroll
-  for (int i = 0; i < kPerLane; ++i) {
+  for (int i = 0; i < EPL; ++i) {
     const int e = lane + 32 * i;
-    if (e < E) {
-      float l = row[e];
-      for (int sp = 1; sp < nsplit; ++sp) l += row[sp * split_stride + e];  // K-split partials, in order
-      v[i] = l + (bias ? bias[e] : 0.f);
-    } else {
-      v[i] = NEG;
+    v[i] = e < E ? row[e] : 0.f;
+  }
+  int sp = 1;
+  for (; sp + UNR <= nsplit; sp += UNR) {
+    float p[UNR][EPL];
+#pragma unroll
+    for (int q = 0; q < UNR; ++q)
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        p[q][i] = e < E ? row[(size_t)(sp + q) * split_stride + e] : 0.f;
+      }
+#pragma unroll
+    for (int q = 0; q < UNR; ++q)
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) v[i] += p[q][i];
+  }
+  for (; sp < nsplit; ++sp) {
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E) v[i] += row[(size_t)sp * split_stride + e];
     }
   }
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = e < E ? v[i] + (bias ? bias[e] : 0.f) : NEG;
+  }
   uint32_t taken = 0;
-  const int nper = (E + 31) / 32;
   float lead = 0.f, sum = 0.f;
   int32_t* idrow = ids + (size_t)t * k;
   float* wrow = wout + (size_t)t * k;
@@ -123,9 +145,9 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
     float bv = NEG;
     int bi = 0x7fffffff;
 #pragma unroll
-    for (int i = 0; i < kPerLane; ++i) {
+    for (int i = 0; i < EPL; ++i) {
       const int e = lane + 32 * i;
-      if (i < nper && e < E && !(taken >> i & 1u)) {
+      if (e < E && !(taken >> i & 1u)) {
         if (v[i] > bv || (v[i] == bv && e < bi)) { bv = v[i]; bi = e; }
       }
     }
@@ -154,6 +176,14 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
   for (int j = lane; j < k; j += 32) wrow[j] = wrow[j] * inv;
 }
 
+template <int EPL, int UNR>
+cudaError_t launch_topk_t(const float* logits, int nsplit, size_t split_stride, const float* bias, int T, int E,
+                          int k, int32_t* ids, float* w, DevStatus* st, cudaStream_t s) {
+  topk_kernel<EPL, UNR><<<(T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, s>>>(logits, nsplit, split_stride,
+                                                                                      bias, T, E, k, ids, w, st);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_router_split(const float* w, int H, int E, uint16_t* planes, cudaStream_t s) {
@@ -171,9 +201,12 @@ cudaError_t launch_router_logits_fma(const uint16_t* x, const float* w, int T, i
 
 cudaError_t launch_topk(const float* logits, int nsplit, size_t split_stride, const float* bias, int T, int E, int k,
                         int32_t* ids, float* w, DevStatus* st, cudaStream_t s) {
-  topk_kernel<<<(T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, s>>>(logits, nsplit, split_stride, bias, T, E,
-                                                                            k, ids, w, st);
-  return cudaGetLastError();
+  if (E <= 32) return launch_topk_t<1, 8>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
+  if (E <= 64) return launch_topk_t<2, 8>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
+  if (E <= 128) return launch_topk_t<4, 8>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
+  if (E <= 256) return launch_topk_t<8, 4>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
+  if (E <= 512) return launch_topk_t<16, 4>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
+  return launch_topk_t<32, 2>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
 }
 
 }  // namespace moe

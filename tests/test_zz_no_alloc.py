@@ -2,7 +2,9 @@
 device memory at call time (its scratch is an array built into the
 library).  Called through the C ABI and compared, bit for bit, with the
 workspace-based moe_permute on two calls in a row; the second call has a
-different shape so stale scratch from the first would show."""
+different shape so stale scratch from the first would show.  Batches of up
+to 8192 slots are permuted inside one block without any scratch, so the
+calls use 32,768 and 16,384 slots, which go through the scratch array."""
 import ctypes
 
 import numpy as np
@@ -32,7 +34,7 @@ def test_noalloc_permute_matches_workspace_permute_twice():
     fn = _noalloc()
     rng = np.random.default_rng(11)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    for T, E, k in [(512, 512, 10), (300, 16, 3)]:
+    for T, E, k in [(4096, 256, 8), (2048, 512, 8)]:
         ids = torch.from_numpy(_ids(rng, T, E, k)).cuda()
         ws = moe.alloc_workspace(T, 256, E, 128, k)
         want = moe.permute(ids, E, ws)
