@@ -348,3 +348,20 @@ def test_zipf_bias_makes_expert_zero_hottest():
     ids, _ = om.topk_route(om.router_logits(inp.x, inp.w_router, inp.bias), cfg.k)
     counts = np.bincount(ids.reshape(-1), minlength=cfg.E)
     assert counts.argmax() == 0 and counts[0] > 0.5 * cfg.T
+
+
+def test_oracle_matches_frozen_tiny_regression():
+    """Guards against unintended changes to the oracle's arithmetic (the
+    fixture is written by tests/golden/make_golden.py from the oracle)."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "tiny_oracle_regression.npz")
+    want = np.load(path)
+    cfg = synth.CONFIGS["tiny"]
+    inp = synth.make_inputs(cfg)
+    oracle.enforce_logit_gap(inp)
+    np.testing.assert_array_equal(inp.x, want["x"])
+    got = om.layer_forward(inp.x, inp.w_router, inp.bias, inp.w_gate_up, inp.w_down, cfg.k)
+    for key in ("ids", "offsets", "sorted_token_ids"):
+        np.testing.assert_array_equal(got[key], want[key])
+    np.testing.assert_allclose(got["w"], want["w"], rtol=1e-13)
+    np.testing.assert_allclose(got["y"], want["y"], rtol=1e-12, atol=1e-15)
