@@ -51,6 +51,22 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def reduce_max(value, device):
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(tokens_per_rank, world, steps, max_total_ms):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time (weak scaling)."""
+    return tokens_per_rank * world * steps / (max_total_ms / 1e3)
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -271,14 +287,10 @@ def time_workload(cfg, d, ws, steps, warmup, rank, world, flush, moe, gpu_index,
     else:
         step_ms = [e[0].elapsed_time(e[6]) for e in evs]
         stage_ms = [[e[j].elapsed_time(e[j + 1]) for j in range(6)] for e in evs]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max(sum(step_ms), "cuda")
     mean_stage = [statistics.mean(s[j] for s in stage_ms) for j in range(6)] if stage_ms else None
     del g
-    return dict(total_ms=total_ms, ms_per_step=total_ms / steps, value=T * world * steps / (total_ms / 1e3),
+    return dict(total_ms=total_ms, ms_per_step=total_ms / steps, value=throughput(T, world, steps, total_ms),
                 stage_ms=mean_stage, launches=info.get("launches", 0) * steps, clocks=clocks,
                 step_ms_median=statistics.median(step_ms), host_us_per_call=host_us)
 
@@ -310,12 +322,8 @@ def time_e2e(cfg, d, ws, steps, warmup, rank, world, moe, tiles=0):
         step()
     e.record()
     torch.cuda.synchronize()
-    ms = s.elapsed_time(e)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": cfg.T * world * steps / (ms / 1e3), "unit": "tokens/s",
+    ms = reduce_max(s.elapsed_time(e), "cuda")
+    return {"value": throughput(cfg.T, world, steps, ms), "unit": "tokens/s",
             "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2,
             "ms_per_step": ms / steps}
 

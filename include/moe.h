@@ -72,7 +72,7 @@ typedef enum moe_status {
 /* Tile policy of the grouped expert GEMMs (moe_forward_ex / grouped calls). */
 enum {
   MOE_TILES_AUTO = 0,   /* chosen from the mean rows per expert, T*k/E */
-  MOE_TILES_SMALL = 1,  /* <= 64 token rows per tile pass, 5-stage ring: decode */
+  MOE_TILES_SMALL = 1,  /* <= 128 token rows per tile pass, 4-stage ring: decode */
   MOE_TILES_LARGE = 2,  /* <= 256 token rows per tile pass, 3-stage ring: prefill */
   MOE_TILES_PAIR = 3    /* 256-row tiles on SM pairs (2-SM tcgen05 MMA, 6-stage ring); never chosen by AUTO */
 };

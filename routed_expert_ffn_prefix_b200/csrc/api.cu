@@ -26,7 +26,7 @@ inline int resolve_router(int impl, int E) {
 
 inline int router_tiles(int T) { return T >= 2048 ? MOE_TILES_LARGE : MOE_TILES_SMALL; }
 inline int router_splits(int T, int H, int E) {
-  const int nt = router_tiles(T) == MOE_TILES_LARGE ? 256 : 64;
+  const int nt = router_tiles(T) == MOE_TILES_LARGE ? 256 : 128;
   const int cols = 128 * gemm_tiles_per_unit(router_tiles(T), EPI_STORE_F32);
   const int base = ((T + nt - 1) / nt) * ((E + cols - 1) / cols);
   int s = (296 + base - 1) / base;
@@ -187,7 +187,7 @@ inline Tp* at(void* ws, size_t off) {
 int choose_tiles(int policy, long long rows, int groups) {
   if (policy == MOE_TILES_SMALL || policy == MOE_TILES_LARGE || policy == MOE_TILES_PAIR) return policy;
   // mean rows per group: small groups stream weights under few rows
-  return rows > 48ll * groups ? MOE_TILES_LARGE : MOE_TILES_SMALL;
+  return rows > 64ll * groups ? MOE_TILES_LARGE : MOE_TILES_SMALL;
 }
 
 // ---------------------------------------------------------------- stage launchers (no checks)

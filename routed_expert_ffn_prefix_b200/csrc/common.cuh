@@ -131,6 +131,12 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   return p;
 }
 
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 __device__ __forceinline__ uint64_t policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
@@ -142,8 +148,9 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
 }
 
 // ---------------------------------------------------------------- cp.async
-__device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
+__device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void* src, uint64_t policy) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src), "l"(policy)
+               : "memory");
 }
 
 // Arrive on `bar` once all cp.async issued so far by this thread have
@@ -207,20 +214,28 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout):
+// Shared-memory matrix descriptor (sm_100 layout):
 //   bits 0-13 start>>4, 16-29 leading byte offset>>4, 32-45 stride byte
-//   offset>>4, 46-47 version (1), 61-63 layout (2 = SWIZZLE_128B).
-// K-major operand: rows of 128 B, SBO = byte distance between 8-row groups.
+//   offset>>4, 46-47 version (1), 61-63 layout (2 = SWIZZLE_128B, 4 = SWIZZLE_64B).
+// K-major operand: rows of 128 B (64 B for the 64-byte swizzle), SBO = byte
+// distance between 8-row groups.
 // MN-major operand: LBO = distance between 64-element MN blocks, SBO =
 // distance between 8-row K groups.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
   d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
   d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
+  d |= (uint64_t)layout << 61;
   return d;
+}
+
+constexpr uint32_t kLayoutSw128 = 2;  // 128-byte swizzle
+constexpr uint32_t kLayoutSw64 = 4;   // 64-byte swizzle
+
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return smem_desc(saddr, lbo, sbo, kLayoutSw128);
 }
 
 // Two 16-column loads (32 lanes x 32 bit each) from TMEM plus the wait, in

@@ -16,6 +16,7 @@ constexpr int kBK = 64;  // k per pipeline stage (one 128-byte swizzle row of bf
 
 struct Unit {
   int group, nb, row0, rows, ks, kb, ke;  // ks: K split; [kb, ke): its k-steps (of kBK)
+  int passes;                             // row passes of this group (units re-streaming the same weights)
 };
 
 __device__ __forceinline__ int group_rows_begin(const GemmArgs& a, int g) {
@@ -45,6 +46,7 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, const int* ustart
   r.ks = rem - pass * S;
   r.row0 = b + pass * NT;
   r.rows = min(NT, e - r.row0);
+  r.passes = passes;
   const int nkt = a.K / kBK;
   r.kb = r.ks * nkt / S;
   r.ke = (r.ks + 1) * nkt / S;

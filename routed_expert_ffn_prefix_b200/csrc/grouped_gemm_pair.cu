@@ -205,7 +205,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int pt = tid - kPEpiWarps * 32;
     const int chunk = pt & 7, rsub = pt >> 3;
     constexpr int kRowsPerThread = kPRows / (kPProdThreads / 8);
+    // Weight tiles are streamed past L2 (evict-first): keeping them (even for
+    // groups with several row passes) measured slower, because it displaces
+    // the token rows, which every column block of the group reads again.
     const uint64_t pol_w = policy_evict_first();
+    const uint64_t pol_rows = a.rows_evict_last ? policy_evict_last() : policy_evict_normal();
     const __nv_bfloat16* bsrc = reinterpret_cast<const __nv_bfloat16*>(a.b_src);
     uint64_t* rows_bar_base = leader ? full : xfull;
     const uint32_t full_leader = map_to_rank(smem_u32(full), 0);
@@ -242,7 +246,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
         for (int i = 0; i < kRowsPerThread; ++i) {
           if (src[i] >= 0) {
             const int c = rsub + 16 * i;
-            cp_async_16(sx + c * 128 + ((chunk ^ (c & 7)) << 4), bsrc + (size_t)src[i] * a.K + kt * kBK + chunk * 8);
+            cp_async_16(sx + c * 128 + ((chunk ^ (c & 7)) << 4), bsrc + (size_t)src[i] * a.K + kt * kBK + chunk * 8,
+                        pol_rows);
           }
         }
         cp_async_arrive_noinc(&rows_bar_base[stage]);

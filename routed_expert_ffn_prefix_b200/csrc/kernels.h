@@ -49,6 +49,7 @@ struct GemmArgs {
   int out_col1_off;    // store epilogue: second tile's output columns offset
   int n_valid;         // output columns < n_valid are written
   int rows_cap;        // offsets[groups] may not exceed this (rows of out / row_index)
+  int rows_evict_last; // token-row gathers keep their lines in L2 (evict-last hint) instead of normal
   int k_splits;        // K range split across this many work units (store epilogue only)
   size_t split_stride; // elements between the partial-result slabs of consecutive K splits
   DevStatus* status;
