@@ -40,7 +40,9 @@
  *   - Workspace: caller-allocated device memory of at least
  *     moe_workspace_size() bytes for the layer's shapes; every call takes
  *     the same workspace (each stage uses its own region of it).  Calls
- *     that share a workspace must be stream-ordered.
+ *     that share a workspace must be stream-ordered.  Its status block
+ *     (offset 0) must be cleared once, with moe_clear_device_status(),
+ *     before the workspace is first used.
  *   - Errors in the arguments are found on the host before anything is
  *     enqueued: the call returns the status and launches nothing.
  *     Errors found on the device (a bounds check on routing metadata, a
@@ -81,8 +83,13 @@ enum {
 enum {
   MOE_ROUTER_AUTO = 0,
   MOE_ROUTER_FMA = 1,   /* fp32 CUDA-core dot products */
-  MOE_ROUTER_TC = 2     /* fp32 W split into three bf16 terms, tcgen05 MMA, fp32 accumulate */
+  MOE_ROUTER_TC = 2,    /* fp32 W split into three bf16 terms, tcgen05 MMA, fp32 accumulate */
+  MOE_ROUTER_SMALL = 3  /* T <= 16, E % 4 == 0: fp32 CUDA-core dot products with H split over
+                           ~148 blocks; the last block sums the partials, selects the top-k and
+                           (in moe_forward) builds the permutation -- one launch */
 };
+/* MOE_ROUTER_AUTO picks SMALL when T <= 16 and E % 4 == 0, else TC when
+ * E % 8 == 0, else FMA. */
 
 /* Human-readable name of a status code (static storage). */
 const char *moe_status_string(int status);
@@ -95,10 +102,12 @@ int moe_abi_version(void);
  *   topk_ids [T,k] i32, topk_w [T,k] f32, counts [E] i32, offsets [E+1] i32,
  *   sorted_token_ids [T*k] i32, inv_perm [T,k] i32, h [T*k, I] bf16,
  *   o [T*k, H] f32, h_shared [T, I_s] bf16, o_shared [T, H] f32,
- *   logits [T, E] f32, router_split [3, H, E] bf16, block_hist (permute). */
+ *   logits [S, T, E] f32 (S router partial slabs), router_split [3, H, E]
+ *   bf16, block_hist (permute), split: K-split partial slabs of the expert
+ *   GEMMs when few tokens leave SMs idle (f32; 0 bytes when unused). */
 typedef struct moe_workspace_layout {
   size_t status, topk_ids, topk_w, counts, offsets, sorted_token_ids, inv_perm;
-  size_t h, o, h_shared, o_shared, logits, router_split, block_hist;
+  size_t h, o, h_shared, o_shared, logits, router_split, block_hist, split;
   size_t total;
 } moe_workspace_layout_t;
 
@@ -112,7 +121,8 @@ moe_status_t moe_workspace_size(int T, int H, int E, int I, int k, int I_s, size
  * *out receives MOE_OK or the first error a kernel recorded. */
 moe_status_t moe_get_device_status(const void *workspace, void *stream, int32_t *out);
 
-/* Resets the device status word to MOE_OK (stream-ordered). */
+/* Resets the workspace status block (stream-ordered): the status word to
+ * MOE_OK and the block counter the few-token router keeps beside it. */
 moe_status_t moe_clear_device_status(void *workspace, void *stream);
 
 /* Route: topk_ids [T,k] i32 and topk_w [T,k] f32 from x [T,H] bf16,
@@ -195,7 +205,11 @@ moe_status_t moe_down_combine(const uint16_t *h, const uint16_t *w_down,
 
 /* The whole layer: y [T,H] bf16.  W_sh_gate_up [H, 2 I_s] and W_sh_down
  * [I_s, H] describe the optional shared expert (both NULL and I_s = 0 for
- * none).  Intermediates stay in the workspace (moe_workspace_layout). */
+ * none).  Intermediates stay in the workspace (moe_workspace_layout).
+ * When T*k is so small that the expert GEMMs have fewer work units than
+ * the GPU has SMs, their K range is split and the partial slabs are summed
+ * in a fixed order (gate/up before SwiGLU, down inside the combine); y is
+ * bitwise reproducible for given shapes either way. */
 moe_status_t moe_forward(const uint16_t *x, const float *w_router, const float *bias,
                          const uint16_t *w_gate_up, const uint16_t *w_down,
                          const uint16_t *w_sh_gate_up, const uint16_t *w_sh_down, int I_s,
@@ -211,7 +225,8 @@ typedef struct moe_forward_options {
    * by the caller) is recorded on the stream at stage boundary i:
    * 0 before routing, 1 after routing, 2 after the permutation, 3 after the
    * shared expert, 4 after the gate/up GEMM, 5 after the down GEMM, 6 after
-   * the combine. */
+   * the combine.  With MOE_ROUTER_SMALL routing and permutation are one
+   * kernel (events 1 and 2 are recorded together after it). */
   void *stage_events[7];
   /* Output: the number of kernels this call enqueued. */
   int launches;

@@ -17,10 +17,12 @@ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 // the K range (H) is split so that about two work units land on each of the
 // 148 SMs.  A function of the shapes only, so the workspace layout and the
 // launch always agree.
-// MOE_ROUTER_AUTO: tensor cores whenever the 16-byte row pitch of the split
-// planes allows it (E % 8 == 0), else fp32 CUDA cores.
-inline int resolve_router(int impl, int E) {
+// MOE_ROUTER_AUTO: a few tokens -> the one-launch split-H router; else tensor
+// cores whenever the 16-byte row pitch of the split planes allows it
+// (E % 8 == 0), else fp32 CUDA cores.
+inline int resolve_router(int impl, int T, int E) {
   if (impl != MOE_ROUTER_AUTO) return impl;
+  if (T <= kSmallRouterT && E % 4 == 0) return MOE_ROUTER_SMALL;
   return E % 8 == 0 ? MOE_ROUTER_TC : MOE_ROUTER_FMA;
 }
 
@@ -35,6 +37,39 @@ inline int router_splits(int T, int H, int E) {
   if (s > 32) s = 32;
   return s < 1 ? 1 : s;
 }
+// Router partial slabs the logits region must hold.
+inline int router_slabs(int T, int H, int E) {
+  int s = router_splits(T, H, E);
+  if (fma_router_splits(T, H) > s) s = fma_router_splits(T, H);
+  if (T <= kSmallRouterT) {
+    const int ss = small_router_slabs(H, E);
+    if (ss > s) s = ss;
+  }
+  return s;
+}
+
+// K splits of the two expert GEMMs (SMALL tiles only).  When even the upper
+// bound on work units, min(E, T*k) + T*k/128 row passes times the column
+// blocks, leaves SMs idle, each unit's K range is split so that about two
+// units land on each of the 148 SMs; every slice keeps >= 4 k-steps of 64.
+// A function of the shapes only, like the workspace layout.
+struct SplitPlan {
+  int gate_up, down;
+};
+inline int split_for(long long units, int nkt) {
+  if (units >= 148) return 1;
+  long long s = 296 / units;
+  if (s > nkt / 4) s = nkt / 4;
+  if (s > 8) s = 8;
+  return s < 1 ? 1 : (int)s;
+}
+inline SplitPlan split_plan(int T, int H, int E, int I, int k, int tiles) {
+  if (tiles != MOE_TILES_SMALL || H <= 0 || I <= 0) return {1, 1};
+  const long long rows = (long long)T * k;
+  const long long passes = (rows < E ? rows : E) + rows / 128;
+  return {split_for(passes * (I / 128), H / 64), split_for(passes * (H / 256), I / 64)};
+}
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // ---------------------------------------------------------------- workspace
@@ -55,12 +90,17 @@ moe_workspace_layout_t make_layout(int T, int H, int E, int I, int k, int I_s) {
   L.sorted_token_ids = take(tk * 4);
   L.inv_perm = take(tk * 4);
   L.block_hist = take((size_t)permute_num_blocks(T, k) * E * 4);
-  L.logits = take((size_t)(H > 0 ? router_splits(T, H, E) : 1) * T * E * 4);
+  L.logits = take((size_t)(H > 0 ? router_slabs(T, H, E) : 1) * T * E * 4);
   L.router_split = take((size_t)3 * H * E * 2);
   L.h = take(tk * I * 2);
   L.o = take(tk * H * 4);
   L.h_shared = take((size_t)T * I_s * 2);
   L.o_shared = take(I_s > 0 ? (size_t)T * H * 4 : 0);
+  // Sized for SMALL tiles, the only policy that splits K.
+  const SplitPlan sp = split_plan(T, H, E, I, k, MOE_TILES_SMALL);
+  const size_t gu = sp.gate_up > 1 ? (size_t)sp.gate_up * tk * 2 * I : 0;
+  const size_t dn = sp.down > 1 ? (size_t)sp.down * tk * H : 0;
+  L.split = take((gu > dn ? gu : dn) * 4);
   L.total = off;
   return L;
 }
@@ -185,18 +225,31 @@ inline Tp* at(void* ws, size_t off) {
 }
 
 int choose_tiles(int policy, long long rows, int groups) {
-  if (policy == MOE_TILES_SMALL || policy == MOE_TILES_LARGE || policy == MOE_TILES_PAIR) return policy;
+  if (policy != MOE_TILES_AUTO) return policy;
   // mean rows per group: small groups stream weights under few rows
   return rows > 64ll * groups ? MOE_TILES_LARGE : MOE_TILES_SMALL;
 }
 
 // ---------------------------------------------------------------- stage launchers (no checks)
+// perm: permutation outputs for the one-launch router (nullptr: routing only)
+struct PermOut {
+  int32_t *counts, *offsets, *sorted_ids, *inv_perm;
+};
+
 moe_status_t run_route(const uint16_t* x, const float* w_router, const float* bias, int T, int H, int E, int k,
                        int32_t* ids, float* w, int impl, void* ws, const moe_workspace_layout_t& L,
-                       const DeviceInfo& dev, cudaStream_t s) {
+                       const DeviceInfo& dev, cudaStream_t s, const PermOut* perm = nullptr) {
   DevStatus* st = status_of(ws);
   float* logits = at<float>(ws, L.logits);
-  impl = resolve_router(impl, E);
+  impl = resolve_router(impl, T, E);
+  if (impl == MOE_ROUTER_SMALL) {
+    if (T > kSmallRouterT) return MOE_ERR_INVALID_ARG;
+    if (E % 4 != 0) return MOE_ERR_ALIGNMENT;
+    return cuda_status(launch_router_small(x, w_router, bias, T, H, E, k, logits, &st->arrivals, ids, w,
+                                           perm ? perm->counts : nullptr, perm ? perm->offsets : nullptr,
+                                           perm ? perm->sorted_ids : nullptr, perm ? perm->inv_perm : nullptr, st,
+                                           s));
+  }
   int nsplit = 1;
   if (impl == MOE_ROUTER_TC) {
     if (E % 8 != 0) return MOE_ERR_ALIGNMENT;
@@ -232,13 +285,17 @@ moe_status_t run_route(const uint16_t* x, const float* w_router, const float* bi
     MOE_TRY(cuda_status(launch_grouped_gemm(map, a, EPI_STORE_F32, router_tiles(T), dev.num_sms, s)));
   } else {
     MOE_TRY(cuda_status(launch_router_logits_fma(x, w_router, T, H, E, logits, s)));
+    nsplit = fma_router_splits(T, H);
   }
   return cuda_status(launch_topk(logits, nsplit, (size_t)T * E, bias, T, E, k, ids, w, st, s));
 }
 
+// nsplit > 1: K-split into partial slabs [nsplit][rows][2I] f32 at `partials`
+// (gate columns [0, I), up [I, 2I)), then one reduce + SwiGLU pass into h.
 moe_status_t run_swiglu(const uint16_t* x, int src_rows, const uint16_t* w_gate_up, const int32_t* offsets,
                         const int32_t* row_index, int rows, int H, int E, int I, int tiles, uint16_t* h,
-                        DevStatus* st, const DeviceInfo& dev, cudaStream_t s) {
+                        DevStatus* st, const DeviceInfo& dev, cudaStream_t s, int nsplit = 1,
+                        float* partials = nullptr) {
   CUtensorMap map;
   if (!make_weight_map(&map, w_gate_up, 2ull * I, (uint64_t)H, (uint64_t)E)) return MOE_ERR_CUDA;
   GemmArgs a{};
@@ -264,12 +321,24 @@ moe_status_t run_swiglu(const uint16_t* x, int src_rows, const uint16_t* w_gate_
   a.split_stride = 0;
   a.status = st;
   a.timeout_ns = kDefaultTimeoutNs;
+  if (nsplit > 1) {
+    a.out = partials;
+    a.ld_out = 2 * I;
+    a.out_col1_off = I;
+    a.n_valid = 2 * I;
+    a.k_splits = nsplit;
+    a.split_stride = (size_t)rows * 2 * I;
+    MOE_TRY(cuda_status(launch_grouped_gemm(map, a, EPI_STORE_F32, tiles, dev.num_sms, s)));
+    return cuda_status(launch_swiglu_reduce(partials, nsplit, a.split_stride, rows, I, h, s));
+  }
   if (tiles == MOE_TILES_PAIR) return cuda_status(launch_grouped_gemm_pair(map, a, EPI_SWIGLU, dev.num_sms, s));
   return cuda_status(launch_grouped_gemm(map, a, EPI_SWIGLU, tiles, dev.num_sms, s));
 }
 
+// nsplit > 1: K-split into partial slabs [nsplit][rows][H] at o.
 moe_status_t run_down(const uint16_t* h, const uint16_t* w_down, const int32_t* offsets, int rows, int H, int E,
-                      int I, int tiles, float* o, DevStatus* st, const DeviceInfo& dev, cudaStream_t s) {
+                      int I, int tiles, float* o, DevStatus* st, const DeviceInfo& dev, cudaStream_t s,
+                      int nsplit = 1) {
   CUtensorMap map;
   if (!make_weight_map(&map, w_down, (uint64_t)H, (uint64_t)I, (uint64_t)E)) return MOE_ERR_CUDA;
   const int cols = 128 * gemm_tiles_per_unit(tiles, EPI_STORE_F32);  // output columns per work unit
@@ -292,8 +361,8 @@ moe_status_t run_down(const uint16_t* h, const uint16_t* w_down, const int32_t* 
   a.out_col1_off = 128;
   a.n_valid = H;
   a.rows_cap = rows;
-  a.k_splits = 1;
-  a.split_stride = 0;
+  a.k_splits = nsplit;
+  a.split_stride = nsplit > 1 ? (size_t)rows * H : 0;
   a.status = st;
   a.timeout_ns = kDefaultTimeoutNs;
   if (tiles == MOE_TILES_PAIR) return cuda_status(launch_grouped_gemm_pair(map, a, EPI_STORE_F32, dev.num_sms, s));
@@ -357,7 +426,7 @@ moe_status_t moe_route_ex(const uint16_t* x, const float* w_router, const float*
                           size_t workspace_bytes, void* stream) {
   if (!all_nonnull(x, w_router, topk_ids, topk_w)) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_shapes(T, H, E, 0, k, false));
-  if (router_impl < MOE_ROUTER_AUTO || router_impl > MOE_ROUTER_TC) return MOE_ERR_INVALID_ARG;
+  if (router_impl < MOE_ROUTER_AUTO || router_impl > MOE_ROUTER_SMALL) return MOE_ERR_INVALID_ARG;
   if (!all_aligned(x, w_router, topk_ids, topk_w) || (bias && !aligned16(bias))) return MOE_ERR_ALIGNMENT;
   const moe_workspace_layout_t L = make_layout(T, H, E, 0, k, 0);
   MOE_TRY(check_ws(workspace, workspace_bytes, L.h));
@@ -439,7 +508,7 @@ moe_status_t moe_down_combine(const uint16_t* h, const uint16_t* w_down, const f
   float* o = at<float>(workspace, L.o);
   DevStatus* st = status_of(workspace);
   MOE_TRY(run_down(h, w_down, offsets, rows, H, E, I, choose_tiles(tile_policy, rows, E), o, st, dev, s));
-  return cuda_status(launch_combine(o, topk_w, inv_perm, shared_out, T, H, k, rows, y, st, s));
+  return cuda_status(launch_combine(o, topk_w, inv_perm, shared_out, T, H, k, rows, 1, 0, y, st, s));
 }
 
 moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const float* bias, const uint16_t* w_gate_up,
@@ -457,7 +526,7 @@ moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const floa
   const int tile_policy = options ? options->tile_policy : MOE_TILES_AUTO;
   const int router_impl = options ? options->router_impl : MOE_ROUTER_AUTO;
   if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_PAIR) return MOE_ERR_INVALID_ARG;
-  if (router_impl < MOE_ROUTER_AUTO || router_impl > MOE_ROUTER_TC) return MOE_ERR_INVALID_ARG;
+  if (router_impl < MOE_ROUTER_AUTO || router_impl > MOE_ROUTER_SMALL) return MOE_ERR_INVALID_ARG;
   if (!all_aligned(x, w_router, w_gate_up, w_down, y) || (bias && !aligned16(bias))) return MOE_ERR_ALIGNMENT;
   const moe_workspace_layout_t L = make_layout(T, H, E, I, k, shared ? I_s : 0);
   MOE_TRY(check_ws(workspace, workspace_bytes, L.total));
@@ -482,16 +551,25 @@ moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const floa
     return MOE_OK;
   };
   int launches = 0;
-  const int ri = resolve_router(router_impl, E);
+  const int ri = resolve_router(router_impl, T, E);
   MOE_TRY(mark(0));
-  MOE_TRY(run_route(x, w_router, bias, T, H, E, k, ids, tw, ri, ws, L, dev, s));
-  launches += ri == MOE_ROUTER_TC ? 3 : 2;
-  MOE_TRY(mark(1));
-  MOE_TRY(cuda_status(
-      launch_permute(ids, T, E, k, counts, offs, sids, inv, at<int32_t>(ws, L.block_hist), st, s)));
-  launches += 3;
+  if (ri == MOE_ROUTER_SMALL) {
+    const PermOut perm{counts, offs, sids, inv};
+    MOE_TRY(run_route(x, w_router, bias, T, H, E, k, ids, tw, ri, ws, L, dev, s, &perm));
+    launches += 1;
+    MOE_TRY(mark(1));
+  } else {
+    MOE_TRY(run_route(x, w_router, bias, T, H, E, k, ids, tw, ri, ws, L, dev, s));
+    launches += ri == MOE_ROUTER_TC ? 3 : 2;
+    MOE_TRY(mark(1));
+    MOE_TRY(cuda_status(
+        launch_permute(ids, T, E, k, counts, offs, sids, inv, at<int32_t>(ws, L.block_hist), st, s)));
+    launches += rows <= 8192 ? 1 : 3;
+  }
   MOE_TRY(mark(2));
   const int tiles = choose_tiles(tile_policy, rows, E);
+  const SplitPlan sp = split_plan(T, H, E, I, k, tiles);
+  float* split = at<float>(ws, L.split);
   float* o_sh = nullptr;
   if (shared) {
     uint16_t* h_sh = at<uint16_t>(ws, L.h_shared);
@@ -502,13 +580,14 @@ moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const floa
     launches += 2;
   }
   MOE_TRY(mark(3));
-  MOE_TRY(run_swiglu(x, T, w_gate_up, offs, sids, rows, H, E, I, tiles, h, st, dev, s));
-  launches += 1;
+  MOE_TRY(run_swiglu(x, T, w_gate_up, offs, sids, rows, H, E, I, tiles, h, st, dev, s, sp.gate_up, split));
+  launches += sp.gate_up > 1 ? 2 : 1;
   MOE_TRY(mark(4));
-  MOE_TRY(run_down(h, w_down, offs, rows, H, E, I, tiles, o, st, dev, s));
+  float* od = sp.down > 1 ? split : o;
+  MOE_TRY(run_down(h, w_down, offs, rows, H, E, I, tiles, od, st, dev, s, sp.down));
   launches += 1;
   MOE_TRY(mark(5));
-  MOE_TRY(cuda_status(launch_combine(o, tw, inv, o_sh, T, H, k, rows, y, st, s)));
+  MOE_TRY(cuda_status(launch_combine(od, tw, inv, o_sh, T, H, k, rows, sp.down, (size_t)rows * H, y, st, s)));
   launches += 1;
   MOE_TRY(mark(6));
   if (options) options->launches = launches;

@@ -11,7 +11,7 @@
 //
 // Memory-bound: a block per (token, 1024-column slice), one float4 per
 // thread, the k slot loads of a thread issued together.
-#include "kernels.h"
+#include "gemm_units.cuh"
 
 namespace moe {
 
@@ -22,6 +22,7 @@ constexpr int kThreads = 256;
 __global__ void __launch_bounds__(kThreads) combine_kernel(const float* __restrict__ o, const float* __restrict__ w,
                                                          const int32_t* __restrict__ inv_perm,
                                                          const float* __restrict__ shared, int H, int k, int rows,
+                                                         int nsplit, size_t split_stride,
                                                          __nv_bfloat16* __restrict__ y, DevStatus* st, int t0) {
   const int t = t0 + blockIdx.y;
   __shared__ int32_t srow[64];
@@ -45,7 +46,14 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const float* __restri
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 8
     for (int j = 0; j < k; ++j) {
-      const float4 v = __ldcs(reinterpret_cast<const float4*>(o + (size_t)srow[j] * H) + c);
+      float4 v = __ldcs(reinterpret_cast<const float4*>(o + (size_t)srow[j] * H) + c);
+      for (int sp = 1; sp < nsplit; ++sp) {  // K-split partial slabs of the down GEMM, in slab order
+        const float4 p = __ldcs(reinterpret_cast<const float4*>(o + sp * split_stride + (size_t)srow[j] * H) + c);
+        v.x += p.x;
+        v.y += p.y;
+        v.z += p.z;
+        v.w += p.w;
+      }
       const float wj = sw[j];
       acc.x = fmaf(wj, v.x, acc.x);
       acc.y = fmaf(wj, v.y, acc.y);
@@ -68,10 +76,48 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const float* __restri
   }
 }
 
+// h[r, i] = bf16(silu(g) * u) with g, u the sums (in slab order) of the K-split
+// partial gate/up slabs P[s][r][0..2I) written by the grouped GEMM's store
+// epilogue (gate in columns [0, I), up in [I, 2I)).
+__global__ void __launch_bounds__(kThreads) swiglu_reduce_kernel(const float* __restrict__ p, int nsplit,
+                                                               size_t split_stride, int rows, int I,
+                                                               __nv_bfloat16* __restrict__ h) {
+  const int I4 = I >> 2;
+  const long long n = (long long)rows * I4;
+  for (long long q = blockIdx.x * (long long)blockDim.x + threadIdx.x; q < n; q += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(q / I4), c = (int)(q - (long long)r * I4);
+    const float* row = p + (size_t)r * 2 * I;
+    float4 g = reinterpret_cast<const float4*>(row)[c];
+    float4 u = reinterpret_cast<const float4*>(row + I)[c];
+    for (int sp = 1; sp < nsplit; ++sp) {
+      const float4 g2 = reinterpret_cast<const float4*>(row + sp * split_stride)[c];
+      const float4 u2 = reinterpret_cast<const float4*>(row + sp * split_stride + I)[c];
+      g.x += g2.x; g.y += g2.y; g.z += g2.z; g.w += g2.w;
+      u.x += u2.x; u.y += u2.y; u.z += u2.z; u.w += u2.w;
+    }
+    __nv_bfloat162 lo = __floats2bfloat162_rn(silu_f(g.x) * u.x, silu_f(g.y) * u.y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(silu_f(g.z) * u.z, silu_f(g.w) * u.w);
+    uint2 packed;
+    packed.x = *reinterpret_cast<uint32_t*>(&lo);
+    packed.y = *reinterpret_cast<uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(h + (size_t)r * I)[c] = packed;
+  }
+}
+
 }  // namespace
 
+cudaError_t launch_swiglu_reduce(const float* partials, int nsplit, size_t split_stride, int rows, int I, uint16_t* h,
+                                 cudaStream_t s) {
+  const long long n = (long long)rows * (I / 4);
+  const int blocks = (int)((n + kThreads - 1) / kThreads < 4096 ? (n + kThreads - 1) / kThreads : 4096);
+  swiglu_reduce_kernel<<<blocks, kThreads, 0, s>>>(partials, nsplit, split_stride, rows, I,
+                                                   reinterpret_cast<__nv_bfloat16*>(h));
+  return cudaGetLastError();
+}
+
 cudaError_t launch_combine(const float* o, const float* topk_w, const int32_t* inv_perm, const float* shared, int T,
-                           int H, int k, int rows, uint16_t* y, DevStatus* st, cudaStream_t s) {
+                           int H, int k, int rows, int nsplit, size_t split_stride, uint16_t* y, DevStatus* st,
+                           cudaStream_t s) {
   if (k > 64) return cudaErrorInvalidValue;
   // Few tokens: split each row over several blocks so every SM has work;
   // many tokens: one block per token, each thread looping over its float4s.
@@ -80,7 +126,7 @@ cudaError_t launch_combine(const float* o, const float* topk_w, const int32_t* i
   slices = slices < 1 ? 1 : (slices > slices_max ? slices_max : slices);
   for (int t0 = 0; t0 < T; t0 += 65535) {  // grid.y limit
     const dim3 grid(slices, T - t0 < 65535 ? T - t0 : 65535);
-    combine_kernel<<<grid, kThreads, 0, s>>>(o, topk_w, inv_perm, shared, H, k, rows,
+    combine_kernel<<<grid, kThreads, 0, s>>>(o, topk_w, inv_perm, shared, H, k, rows, nsplit, split_stride,
                                              reinterpret_cast<__nv_bfloat16*>(y), st, t0);
     const cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;

@@ -19,7 +19,7 @@ struct DevStatus {
   int32_t code;
   int32_t site;
   int32_t aux;
-  int32_t pad;
+  uint32_t arrivals;  // block counter of the few-token router: zero between its launches
 };
 
 // Where an error was raised (DevStatus::site).

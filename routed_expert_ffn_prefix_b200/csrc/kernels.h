@@ -76,6 +76,8 @@ cudaError_t launch_grouped_gemm(const CUtensorMap& wmap, const GemmArgs& a, int 
 
 // Router.
 cudaError_t launch_router_split(const float* w, int H, int E, uint16_t* planes, cudaStream_t s);
+// fp32 CUDA-core logits into fma_router_splits(T, H) partial slabs [T, E].
+int fma_router_splits(int T, int H);
 cudaError_t launch_router_logits_fma(const uint16_t* x, const float* w, int T, int H, int E, float* logits,
                                      cudaStream_t s);
 // logits: nsplit partial slabs of [T, E], split_stride elements apart, summed in slab order.
@@ -89,8 +91,27 @@ cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* cou
                            cudaStream_t s);
 
 // Combine.
+// o: nsplit partial slabs [rows, H] (split_stride elements apart) summed in slab order.
 cudaError_t launch_combine(const float* o, const float* topk_w, const int32_t* inv_perm, const float* shared,
-                           int T, int H, int k, int rows, uint16_t* y, DevStatus* st, cudaStream_t s);
+                           int T, int H, int k, int rows, int nsplit, size_t split_stride, uint16_t* y, DevStatus* st,
+                           cudaStream_t s);
+
+// h = bf16(silu(sum_s gate_s) * sum_s up_s) from K-split partial slabs [rows, 2I].
+cudaError_t launch_swiglu_reduce(const float* partials, int nsplit, size_t split_stride, int rows, int I, uint16_t* h,
+                                 cudaStream_t s);
+
+// Router for a few tokens (T <= kSmallRouterT, E % 4 == 0): fp32 logits with
+// H split over blocks; the last block to finish sums the partial slabs
+// (small_router_slabs(H, E) of them, [slab][T][E] in `partial`) in slab
+// order, selects the top-k and, if counts != nullptr, writes the
+// permutation (counts, offsets, sorted_ids, inv_perm) as launch_permute
+// would.  *arrivals must be zero on entry and is zero again on exit.
+constexpr int kSmallRouterT = 16;
+int small_router_slabs(int H, int E);
+cudaError_t launch_router_small(const uint16_t* x, const float* w, const float* bias, int T, int H, int E, int k,
+                                float* partial, unsigned int* arrivals, int32_t* ids, float* wout, int32_t* counts,
+                                int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm, DevStatus* st,
+                                cudaStream_t s);
 
 cudaError_t launch_selftest_timeout(DevStatus* st, uint64_t timeout_ns, cudaStream_t s);
 

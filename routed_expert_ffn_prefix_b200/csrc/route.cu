@@ -44,27 +44,33 @@ constexpr int kFmaHc = 256;    // h per shared-memory chunk
 constexpr int kFmaThreads = 256;
 constexpr int kFmaEPer = kMaxExperts / kFmaThreads;  // experts per thread (max)
 
+// Block (tb, sy): tokens [16 tb, 16 tb + 16), the sy-th of gridDim.y slices of
+// H (whole 256-row chunks), written to partial slab sy of `logits`.
 __global__ void __launch_bounds__(kFmaThreads) router_logits_fma_kernel(const __nv_bfloat16* __restrict__ x,
                                                                         const float* __restrict__ w, int T,
                                                                         int H, int E,
                                                                         float* __restrict__ logits) {
   __shared__ float xs[kFmaTok][kFmaHc];
   const int t0 = blockIdx.x * kFmaTok;
+  const int nch = (H + kFmaHc - 1) / kFmaHc;
+  const int hb = (int)((long long)blockIdx.y * nch / gridDim.y) * kFmaHc;
+  const int he = min(H, (int)((long long)(blockIdx.y + 1) * nch / gridDim.y) * kFmaHc);
+  logits += (size_t)blockIdx.y * T * E;
   const int tid = threadIdx.x;
   float acc[kFmaTok][kFmaEPer];
 #pragma unroll
   for (int i = 0; i < kFmaTok; ++i)
 #pragma unroll
     for (int j = 0; j < kFmaEPer; ++j) acc[i][j] = 0.f;
-  for (int h0 = 0; h0 < H; h0 += kFmaHc) {
+  for (int h0 = hb; h0 < he; h0 += kFmaHc) {
     __syncthreads();
     for (int i = tid; i < kFmaTok * kFmaHc; i += kFmaThreads) {
       const int r = i / kFmaHc, c = i - r * kFmaHc;
       const int t = t0 + r;
-      xs[r][c] = (t < T && h0 + c < H) ? __bfloat162float(x[(size_t)t * H + h0 + c]) : 0.f;
+      xs[r][c] = (t < T && h0 + c < he) ? __bfloat162float(x[(size_t)t * H + h0 + c]) : 0.f;
     }
     __syncthreads();
-    const int hn = min(kFmaHc, H - h0);
+    const int hn = min(kFmaHc, he - h0);
     for (int hh = 0; hh < hn; ++hh) {
       const float* wrow = w + (size_t)(h0 + hh) * E;
 #pragma unroll
@@ -86,6 +92,73 @@ __global__ void __launch_bounds__(kFmaThreads) router_logits_fma_kernel(const __
       if (e < E) logits[(size_t)t * E + e] = acc[i][j];
     }
   }
+}
+
+// Top-k of one token by one warp: lane L holds the logits of experts
+// L + 32 i in v (entries >= E ignored).  k rounds of a warp arg-max (larger
+// logit first, ties to the lower expert id; NaN logits are never chosen),
+// then w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0) over the k selected
+// logits.  Each round takes the lane's best by a pairwise tree over its EPL
+// entries (log2 EPL dependent steps) and the warp's best by 5 shuffles.
+// sel, if given, receives the k ids too (shared memory of the caller).
+constexpr int kNoExpert = 0x7fffffff;
+
+__device__ __forceinline__ bool topk_better(float av, int ai, float bv, int bi) {
+  return av > bv || (av == bv && ai < bi);
+}
+
+template <int EPL>
+__device__ __forceinline__ void warp_topk(const float (&vin)[EPL], int E, int k, int t, int32_t* idrow, float* wrow,
+                                          int32_t* sel, DevStatus* st) {
+  const int lane = threadIdx.x & 31;
+  float v[EPL];
+  int id[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    const bool ok = e < E && !isnan(vin[i]);
+    v[i] = ok ? vin[i] : -INFINITY;
+    id[i] = ok ? e : kNoExpert;
+  }
+  float lead = 0.f, sum = 0.f;
+  for (int j = 0; j < k; ++j) {
+    float tv[EPL];
+    int ti[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) { tv[i] = v[i]; ti[i] = id[i]; }
+#pragma unroll
+    for (int w = 1; w < EPL; w <<= 1)
+#pragma unroll
+      for (int i = 0; i + w < EPL; i += 2 * w)
+        if (topk_better(tv[i + w], ti[i + w], tv[i], ti[i])) { tv[i] = tv[i + w]; ti[i] = ti[i + w]; }
+    float bv = tv[0];
+    int bi = ti[0];
+#pragma unroll
+    for (int d = 16; d >= 1; d >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, d);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, d);
+      if (topk_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+    }
+    if (bi == kNoExpert) {  // no candidate left: the logits were NaN
+      if (lane == 0) raise_error(st, MOE_ERR_DEVICE_BOUNDS, SITE_TOPK, t);
+      bi = 0;
+      bv = lead;
+    }
+#pragma unroll
+    for (int i = 0; i < EPL; ++i)
+      if (id[i] == bi) { v[i] = -INFINITY; id[i] = kNoExpert; }
+    if (j == 0) lead = bv;
+    const float z = expf(bv - lead);
+    sum += z;
+    if (lane == 0) {
+      idrow[j] = bi;
+      wrow[j] = z;
+      if (sel) sel[j] = bi;
+    }
+  }
+  __syncwarp();
+  const float inv = 1.0f / sum;
+  for (int j = lane; j < k; j += 32) wrow[j] = wrow[j] * inv;
 }
 
 constexpr int kTopkWarps = 8;
@@ -136,44 +209,7 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
     const int e = lane + 32 * i;
     v[i] = e < E ? v[i] + (bias ? bias[e] : 0.f) : NEG;
   }
-  uint32_t taken = 0;
-  float lead = 0.f, sum = 0.f;
-  int32_t* idrow = ids + (size_t)t * k;
-  float* wrow = wout + (size_t)t * k;
-  for (int j = 0; j < k; ++j) {
-    // lane-local best among untaken entries: larger value, then lower index
-    float bv = NEG;
-    int bi = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !(taken >> i & 1u)) {
-        if (v[i] > bv || (v[i] == bv && e < bi)) { bv = v[i]; bi = e; }
-      }
-    }
-#pragma unroll
-    for (int d = 16; d >= 1; d >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, d);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, d);
-      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-    }
-    if (bi == 0x7fffffff) {  // no finite candidate: logits were NaN
-      if (lane == 0) raise_error(st, MOE_ERR_DEVICE_BOUNDS, SITE_TOPK, t);
-      bi = 0;
-      bv = lead;
-    }
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    if (j == 0) lead = bv;
-    const float z = expf(bv - lead);
-    sum += z;
-    if (lane == 0) {
-      idrow[j] = bi;
-      wrow[j] = z;
-    }
-  }
-  __syncwarp();
-  const float inv = 1.0f / sum;
-  for (int j = lane; j < k; j += 32) wrow[j] = wrow[j] * inv;
+  warp_topk<EPL>(v, E, k, t, ids + (size_t)t * k, wout + (size_t)t * k, nullptr, st);
 }
 
 template <int EPL, int UNR>
@@ -184,6 +220,217 @@ cudaError_t launch_topk_t(const float* logits, int nsplit, size_t split_stride, 
   return cudaGetLastError();
 }
 
+
+// ---------------------------------------------------------------- few tokens
+// For T <= kSmallRouterT the logits are a matrix-vector product whose cost is
+// reading W_router (H x E fp32) once, so the work is spread over ~148 blocks:
+// block (cs, hy) owns W columns [8 cs, 8 cs + 8) (one 32-byte sector per
+// row) and rows [hy * chunk, (hy + 1) * chunk).  Each thread streams its rows
+// as float4s (all issued before any is used), multiplies them by the bf16 x
+// staged in shared memory and the block reduces over its rows in a fixed
+// order into partial slab hy.  The last block to arrive (a counter in the
+// workspace status block) sums the slabs in slab order, selects the top-k per
+// token and, when asked, builds the expert-contiguous permutation of the T*k
+// slots (stable: slot order inside each expert) -- routing and permutation in
+// one launch.
+constexpr int kSmallThreads = 256;
+constexpr int kSmallCols = 8;
+constexpr int kSmallPass = 128;  // rows per block pass: 8 warps x 16
+constexpr int kSmallIters = 8;   // passes per block: chunk <= 1024 rows
+constexpr int kSmallMaxSlots = kSmallRouterT * 64;
+
+struct SmallGrid {
+  int ncs, hs, chunk;
+};
+
+inline SmallGrid small_grid(int H, int E) {
+  SmallGrid g;
+  g.ncs = (E + kSmallCols - 1) / kSmallCols;
+  int hs = 148 / g.ncs;
+  const int hs_min = (H + kSmallPass * kSmallIters - 1) / (kSmallPass * kSmallIters);
+  if (hs < hs_min) hs = hs_min;
+  if (hs < 1) hs = 1;
+  g.chunk = (((H + hs - 1) / hs) + 15) & ~15;
+  g.hs = (H + g.chunk - 1) / g.chunk;
+  return g;
+}
+
+template <int TT, int EPL>
+__global__ void __launch_bounds__(kSmallThreads) router_small_kernel(
+    const __nv_bfloat16* __restrict__ x, const float* __restrict__ w, const float* __restrict__ bias, int T, int H,
+    int E, int k, int chunk, int hs, float* __restrict__ partial, unsigned int* arrivals, int32_t* __restrict__ ids,
+    float* __restrict__ wout, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ sorted_ids, int32_t* __restrict__ inv_perm, DevStatus* st) {
+  __shared__ __align__(16) __nv_bfloat16 xs[TT][kSmallPass * kSmallIters];
+  __shared__ float red[kSmallThreads / 32][TT][kSmallCols];
+  __shared__ int32_t sel[kSmallMaxSlots];
+  __shared__ int32_t cnt[kMaxExperts];
+  __shared__ int32_t warp_sums[kSmallThreads / 32];
+  __shared__ int is_last;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cs = blockIdx.x, hy = blockIdx.y;
+  const int h0 = hy * chunk, h1 = min(H, h0 + chunk);
+  const int q = lane & 1, r = lane >> 1;
+  const int c0 = cs * kSmallCols + q * 4;
+  const bool cval = c0 < E;  // E % 4 == 0: a quad is all in or all out
+
+  float4 wr[kSmallIters];
+#pragma unroll
+  for (int i = 0; i < kSmallIters; ++i) {
+    const int h = h0 + warp * 16 + r + kSmallPass * i;
+    wr[i] = (cval && h < h1) ? __ldcs(reinterpret_cast<const float4*>(w + (size_t)h * E + c0))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  // x rows [h0, h1) of every token, zero beyond T and h1
+  constexpr int kVec = kSmallPass * kSmallIters / 8;  // 16-byte vectors per staged row
+  for (int i = tid; i < TT * kVec; i += kSmallThreads) {
+    const int t = i / kVec, v = i - t * kVec, h = h0 + v * 8;
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (t < T && h < h1) val = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H + h));
+    reinterpret_cast<uint4*>(&xs[t][0])[v] = val;
+  }
+  __syncthreads();
+  float acc[TT][4];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+#pragma unroll
+  for (int i = 0; i < kSmallIters; ++i) {
+    const int hl = warp * 16 + r + kSmallPass * i;
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+      const float xv = __bfloat162float(xs[t][hl]);
+      acc[t][0] = fmaf(xv, wr[i].x, acc[t][0]);
+      acc[t][1] = fmaf(xv, wr[i].y, acc[t][1]);
+      acc[t][2] = fmaf(xv, wr[i].z, acc[t][2]);
+      acc[t][3] = fmaf(xv, wr[i].w, acc[t][3]);
+    }
+  }
+  // rows of a warp (lane bits 1..4), then the 8 warps in order
+#pragma unroll
+  for (int d = 2; d < 32; d <<= 1)
+#pragma unroll
+    for (int t = 0; t < TT; ++t)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[t][j] += __shfl_xor_sync(0xffffffffu, acc[t][j], d);
+  if (r == 0) {
+#pragma unroll
+    for (int t = 0; t < TT; ++t)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) red[warp][t][q * 4 + j] = acc[t][j];
+  }
+  __syncthreads();
+  if (tid < TT * kSmallCols) {
+    const int t = tid / kSmallCols, c = tid - t * kSmallCols;
+    float sum = 0.f;
+#pragma unroll
+    for (int v = 0; v < kSmallThreads / 32; ++v) sum += red[v][t][c];
+    const int e = cs * kSmallCols + c;
+    if (t < T && e < E) partial[((size_t)hy * T + t) * E + e] = sum;
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) is_last = atomicAdd(arrivals, 1u) == gridDim.x * gridDim.y - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+
+  // ---- last block: slab sum in slab order, bias, top-k (one warp per token)
+  for (int t = warp; t < T; t += kSmallThreads / 32) {
+    float v[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) v[i] = 0.f;
+    for (int sp = 0; sp < hs; ++sp) {
+      const float* slab = partial + ((size_t)sp * T + t) * E;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) v[i] += __ldcg(slab + e);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      v[i] = e < E ? v[i] + (bias ? bias[e] : 0.f) : -INFINITY;
+    }
+    warp_topk<EPL>(v, E, k, t, ids + (size_t)t * k, wout + (size_t)t * k, sel + t * k, st);
+  }
+  if (counts != nullptr) {
+    // ---- permutation of the n = T*k slots, stable counting sort by expert
+    const int n = T * k;
+    for (int e = tid; e < E; e += kSmallThreads) cnt[e] = 0;
+    __syncthreads();
+    for (int s = tid; s < n; s += kSmallThreads) atomicAdd(&cnt[sel[s]], 1);
+    __syncthreads();
+    constexpr int EPT = kMaxExperts / kSmallThreads;  // experts per thread in the scan
+    int loc[EPT], tot = 0;
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      const int e = tid * EPT + j;
+      loc[j] = e < E ? cnt[e] : 0;
+      tot += loc[j];
+    }
+    int incl = tot;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += o;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    int base = incl - tot;
+    for (int v = 0; v < warp; ++v) base += warp_sums[v];
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      const int e = tid * EPT + j;
+      if (e < E) {
+        counts[e] = loc[j];
+        offsets[e] = base;
+        cnt[e] = base;  // running position of expert e
+      }
+      base += loc[j];
+    }
+    if (tid == 0) offsets[E] = n;
+    __syncthreads();
+    if (warp == 0) {
+      for (int s0 = 0; s0 < n; s0 += 32) {
+        const int s = s0 + lane;
+        const int e = s < n ? sel[s] : -1;
+        const uint32_t peers = __match_any_sync(0xffffffffu, e);
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        const int pos = e >= 0 ? cnt[e] + rank : -1;
+        __syncwarp();
+        if (e >= 0 && rank == 0) cnt[e] += __popc(peers);
+        __syncwarp();
+        if (e >= 0) {
+          sorted_ids[pos] = s / k;
+          inv_perm[s] = pos;
+        }
+      }
+    }
+  }
+  if (tid == 0) *arrivals = 0u;  // every block has arrived: ready for the next launch
+}
+
+template <int TT, int EPL>
+cudaError_t launch_router_small_t(const uint16_t* x, const float* w, const float* bias, int T, int H, int E, int k,
+                                  float* partial, unsigned int* arrivals, int32_t* ids, float* wout,
+                                  int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
+                                  DevStatus* st, cudaStream_t s) {
+  const SmallGrid g = small_grid(H, E);
+  router_small_kernel<TT, EPL><<<dim3(g.ncs, g.hs), kSmallThreads, 0, s>>>(
+      reinterpret_cast<const __nv_bfloat16*>(x), w, bias, T, H, E, k, g.chunk, g.hs, partial, arrivals, ids, wout,
+      counts, offsets, sorted_ids, inv_perm, st);
+  return cudaGetLastError();
+}
+
+// accumulators for 1, 4 or 16 tokens
+template <int EPL, typename... A>
+cudaError_t launch_router_small_e(int T, A... args) {
+  if (T == 1) return launch_router_small_t<1, EPL>(args...);
+  if (T <= 4) return launch_router_small_t<4, EPL>(args...);
+  return launch_router_small_t<kSmallRouterT, EPL>(args...);
+}
+
 }  // namespace
 
 cudaError_t launch_router_split(const float* w, int H, int E, uint16_t* planes, cudaStream_t s) {
@@ -192,9 +439,19 @@ cudaError_t launch_router_split(const float* w, int H, int E, uint16_t* planes, 
   return cudaGetLastError();
 }
 
+int fma_router_splits(int T, int H) {
+  const int tb = (T + kFmaTok - 1) / kFmaTok;
+  int sp = 148 / tb;
+  const int nch = (H + kFmaHc - 1) / kFmaHc;
+  if (sp > nch) sp = nch;
+  if (sp > 32) sp = 32;
+  return sp < 1 ? 1 : sp;
+}
+
 cudaError_t launch_router_logits_fma(const uint16_t* x, const float* w, int T, int H, int E, float* logits,
                                      cudaStream_t s) {
-  router_logits_fma_kernel<<<(T + kFmaTok - 1) / kFmaTok, kFmaThreads, 0, s>>>(
+  const dim3 grid((T + kFmaTok - 1) / kFmaTok, fma_router_splits(T, H));
+  router_logits_fma_kernel<<<grid, kFmaThreads, 0, s>>>(
       reinterpret_cast<const __nv_bfloat16*>(x), w, T, H, E, logits);
   return cudaGetLastError();
 }
@@ -207,6 +464,25 @@ cudaError_t launch_topk(const float* logits, int nsplit, size_t split_stride, co
   if (E <= 256) return launch_topk_t<8, 4>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
   if (E <= 512) return launch_topk_t<16, 4>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
   return launch_topk_t<32, 2>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
+}
+
+int small_router_slabs(int H, int E) { return small_grid(H, E).hs; }
+
+cudaError_t launch_router_small(const uint16_t* x, const float* w, const float* bias, int T, int H, int E, int k,
+                                float* partial, unsigned int* arrivals, int32_t* ids, float* wout, int32_t* counts,
+                                int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm, DevStatus* st,
+                                cudaStream_t s) {
+  if (T < 1 || T > kSmallRouterT || E % 4 != 0 || k > 64) return cudaErrorInvalidValue;
+  if (E <= 64) return launch_router_small_e<2>(T, x, w, bias, T, H, E, k, partial, arrivals, ids, wout, counts,
+                                                offsets, sorted_ids, inv_perm, st, s);
+  if (E <= 128) return launch_router_small_e<4>(T, x, w, bias, T, H, E, k, partial, arrivals, ids, wout, counts,
+                                                 offsets, sorted_ids, inv_perm, st, s);
+  if (E <= 256) return launch_router_small_e<8>(T, x, w, bias, T, H, E, k, partial, arrivals, ids, wout, counts,
+                                                 offsets, sorted_ids, inv_perm, st, s);
+  if (E <= 512) return launch_router_small_e<16>(T, x, w, bias, T, H, E, k, partial, arrivals, ids, wout, counts,
+                                                  offsets, sorted_ids, inv_perm, st, s);
+  return launch_router_small_e<32>(T, x, w, bias, T, H, E, k, partial, arrivals, ids, wout, counts, offsets,
+                                   sorted_ids, inv_perm, st, s);
 }
 
 }  // namespace moe

@@ -1,8 +1,8 @@
 """GPU parity of every stage and of the whole layer against the CPU oracle,
 at sizes the oracle finishes in seconds: several tiles per expert, ragged
 per-expert row counts, empty experts, one token, k = E, a shared expert,
-experts with more rows than one tile pass, and both tile policies and both
-router implementations.  Routing (ids, counts, offsets, permutation) must
+experts with more rows than one tile pass, every tile policy, every router
+implementation and the K-split of the expert GEMMs for a few tokens.  Routing (ids, counts, offsets, permutation) must
 match bit for bit; floating-point outputs within the layer's tolerance."""
 import numpy as np
 import pytest
@@ -26,6 +26,10 @@ CASES = {
         Config("one_token", T=1, H=512, E=16, I=256, k=4),
         Config("sparse", T=5, H=256, E=64, I=128, k=2),            # most experts empty
         Config("wide", T=96, H=1024, E=32, I=384, k=6, I_s=128),   # I not a power of two
+        # few tokens: the one-launch router and K-split expert GEMMs
+        Config("decode_split", T=1, H=1024, E=64, I=512, k=8),      # gate/up 4 K slices, down 2
+        Config("few_e20", T=12, H=512, E=20, I=256, k=5),           # E % 8 != 0: ragged column slice
+        Config("three_shared", T=3, H=768, E=32, I=128, k=4, I_s=128),
     ]
 }
 
@@ -61,12 +65,18 @@ def assert_ok(ws):
     assert st == 0, moe.STATUS.get(st, st)
 
 
-@pytest.mark.parametrize("impl", [moe.ROUTER_FMA, moe.ROUTER_TC])
+def router_skip(cfg, impl):
+    if impl == moe.ROUTER_TC and cfg.E % 8:
+        pytest.skip("tensor-core router needs E % 8 == 0")
+    if impl == moe.ROUTER_SMALL and (cfg.T > 16 or cfg.E % 4):
+        pytest.skip("few-token router needs T <= 16 and E % 4 == 0")
+
+
+@pytest.mark.parametrize("impl", [moe.ROUTER_FMA, moe.ROUTER_TC, moe.ROUTER_SMALL])
 @pytest.mark.parametrize("name", list(CASES))
 def test_route_matches_oracle(name, impl):
     cfg, inp, ref = case(name)
-    if impl == moe.ROUTER_TC and cfg.E % 8:
-        pytest.skip("tensor-core router needs E % 8 == 0")
+    router_skip(cfg, impl)
     d = dev_inputs(inp)
     ws = workspace(cfg)
     ids, w = moe.route(d["x"], d["w_router"], d["bias"], cfg.k, ws, impl=impl)
@@ -142,13 +152,12 @@ def test_grouped_down_single_group():
     assert_close_output(host_f64(o), want, "o")
 
 
-@pytest.mark.parametrize("router", [moe.ROUTER_FMA, moe.ROUTER_TC])
+@pytest.mark.parametrize("router", [moe.ROUTER_FMA, moe.ROUTER_TC, moe.ROUTER_SMALL])
 @pytest.mark.parametrize("tiles", [moe.TILES_SMALL, moe.TILES_LARGE, moe.TILES_PAIR])
 @pytest.mark.parametrize("name", list(CASES))
 def test_forward_matches_oracle(name, tiles, router):
     cfg, inp, ref = case(name)
-    if router == moe.ROUTER_TC and cfg.E % 8:
-        pytest.skip("tensor-core router needs E % 8 == 0")
+    router_skip(cfg, router)
     d = dev_inputs(inp)
     ws = workspace(cfg)
     y = moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws,
@@ -178,6 +187,43 @@ def test_forward_bitwise_deterministic():
                     moe.alloc_workspace(7, cfg.H, cfg.E, cfg.I, cfg.k))
     assert_ok(ws)
     assert torch.equal(ys[0], ys[1]) and torch.equal(ys[2], ys[3])
+
+
+def test_few_token_router_repeated_calls():
+    """The one-launch router's last-block counter returns to zero after each
+    launch: back-to-back calls (also through the whole layer) stay correct
+    and leave the workspace's status block all zero."""
+    import torch
+    for name in ("decode_split", "few_e20", "three_shared"):
+        cfg, inp, ref = case(name)
+        d = dev_inputs(inp)
+        ws = workspace(cfg)
+        for _ in range(3):
+            ids, w = moe.route(d["x"], d["w_router"], d["bias"], cfg.k, ws, impl=moe.ROUTER_SMALL)
+            np.testing.assert_array_equal(ids.cpu().numpy(), ref["ids"])
+            y = moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws,
+                            d["w_sh_gate_up"], d["w_sh_down"])
+            assert_close_output(host_f64(y), ref["y"])
+        torch.cuda.synchronize()
+        assert ws[:16].view(torch.int32).cpu().tolist() == [0, 0, 0, 0]
+
+
+def test_split_k_forward_bitwise_deterministic():
+    """K-split partial slabs are summed in slab order: repeated runs give
+    identical bits, and the layout reserves the slabs."""
+    import torch
+    cfg, inp, ref = case("decode_split")
+    lay = moe.workspace_layout(cfg.T, cfg.H, cfg.E, cfg.I, cfg.k, 0)
+    assert lay["total"] - lay["split"] >= 4 * 4 * cfg.T * cfg.k * 2 * cfg.I  # 4 gate/up slices
+    d = dev_inputs(inp)
+    ws = workspace(cfg)
+    info = {}
+    ys = [moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws,
+                      info=info).cpu() for _ in range(3)]
+    assert_ok(ws)
+    assert info["launches"] == 5  # route+permute, gate/up, SwiGLU reduce, down, combine
+    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2])
+    assert_close_output(host_f64(ys[0]), ref["y"])
 
 
 def test_all_tokens_to_the_same_experts():
