@@ -73,10 +73,11 @@ typedef enum moe_status {
 
 /* Tile policy of the grouped expert GEMMs (moe_forward_ex / grouped calls). */
 enum {
-  MOE_TILES_AUTO = 0,   /* chosen from the mean rows per expert, T*k/E */
+  MOE_TILES_AUTO = 0,   /* chosen from the mean rows per expert, T*k/E: SMALL up to 64, else PAIR */
   MOE_TILES_SMALL = 1,  /* <= 128 token rows per tile pass, 4-stage ring: decode */
   MOE_TILES_LARGE = 2,  /* <= 256 token rows per tile pass, 3-stage ring: prefill */
-  MOE_TILES_PAIR = 3    /* 256-row tiles on SM pairs (2-SM tcgen05 MMA, 6-stage ring); never chosen by AUTO */
+  MOE_TILES_PAIR = 3    /* SM pairs (2-SM tcgen05 MMA): 256 weight columns per MMA, 128 per SM; <= 256
+                           token rows per pass, half gathered by each SM; 4-stage ring: prefill */
 };
 
 /* Router logits implementation. */
@@ -101,7 +102,8 @@ int moe_abi_version(void);
  * after moe_forward; all 256-byte aligned).  Regions:
  *   topk_ids [T,k] i32, topk_w [T,k] f32, counts [E] i32, offsets [E+1] i32,
  *   sorted_token_ids [T*k] i32, inv_perm [T,k] i32, h [T*k, I] bf16,
- *   o [T*k, H] f32, h_shared [T, I_s] bf16, o_shared [T, H] f32,
+ *   o [T*k, H] bf16 (expert outputs, permuted order), h_shared [T, I_s] bf16,
+ *   o_shared [T, H] f32,
  *   logits [S, T, E] f32 (S router partial slabs), router_split [3, H, E]
  *   bf16, block_hist (permute), split: K-split partial slabs of the expert
  *   GEMMs when few tokens leave SMs idle (f32; 0 bytes when unused). */
@@ -193,9 +195,10 @@ moe_status_t moe_grouped_down(const uint16_t *h, const uint16_t *w_down, const i
 /* Down GEMM + weighted combine: y [T,H] bf16 from h [T*k, I] bf16 (permuted
  * order), W_down [E, I, H] bf16, topk_w [T,k] f32, inv_perm [T,k] i32,
  * offsets [E+1] i32 and an optional shared-expert output shared_out [T,H]
- * f32 (NULL for none), added after the k routed terms.  The k terms of a
- * token are summed in slot order j = 0..k-1 in fp32, so y is bitwise
- * reproducible. */
+ * f32 (NULL for none), added after the k routed terms.  Each expert output
+ * row is accumulated in fp32 and stored as bf16 (the layer's activation
+ * type); the k terms of a token are summed in slot order j = 0..k-1 in
+ * fp32, so y is bitwise reproducible. */
 moe_status_t moe_down_combine(const uint16_t *h, const uint16_t *w_down,
                               const float *topk_w, const int32_t *inv_perm,
                               const int32_t *offsets, const float *shared_out,

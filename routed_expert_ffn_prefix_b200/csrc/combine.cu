@@ -3,14 +3,16 @@
 // The Qwen 3.5-397B-on-Ironwood page (sec. 7.2) un-permutes the [T*k, H]
 // expert outputs and gather-reduces them per token; the Ling-2.6-1T /
 // SGLang-JAX page fuses scatter, expert FFN and gather ("Fused MoE V2").
-// Here each token's k expert rows are read through inv_perm and summed in
+// Here each token's k expert rows (bf16, or fp32 K-split partial slabs that
+// are first summed in slab order) are read through inv_perm and summed in
 // slot order j = 0..k-1 in fp32 (w_j * o_j, one fused multiply-add per
 // term), the shared-expert row (weight 1) is added last, and y is rounded
 // to bf16 once.  A fixed summation order makes y bitwise reproducible
 // run to run, whatever order the expert GEMM tiles finished in.
 //
-// Memory-bound: a block per (token, 1024-column slice), one float4 per
-// thread, the k slot loads of a thread issued together.
+// Memory-bound: a block per (token, column slice), one 16-byte vector of a
+// row per thread and slot (8 bf16 or 4 fp32 columns), the k slot loads of a
+// thread issued together.
 #include "gemm_units.cuh"
 
 namespace moe {
@@ -19,11 +21,40 @@ namespace {
 
 constexpr int kThreads = 256;
 
-__global__ void __launch_bounds__(kThreads) combine_kernel(const float* __restrict__ o, const float* __restrict__ w,
+// V consecutive columns of an expert output row in one 16-byte load, widened
+// to fp32: 4 fp32 columns or 8 bf16 columns.
+template <typename OT>
+struct Vec;
+template <>
+struct Vec<float> {
+  static constexpr int V = 4;
+  static __device__ __forceinline__ void load(const float* p, float (&v)[4]) {
+    const float4 q = __ldcs(reinterpret_cast<const float4*>(p));
+    v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+  }
+};
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int V = 8;
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 q = __ldcs(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
+  }
+};
+
+template <typename OT>
+__global__ void __launch_bounds__(kThreads) combine_kernel(const OT* __restrict__ o, const float* __restrict__ w,
                                                          const int32_t* __restrict__ inv_perm,
                                                          const float* __restrict__ shared, int H, int k, int rows,
                                                          int nsplit, size_t split_stride,
                                                          __nv_bfloat16* __restrict__ y, DevStatus* st, int t0) {
+  constexpr int V = Vec<OT>::V;
   const int t = t0 + blockIdx.y;
   __shared__ int32_t srow[64];
   __shared__ float sw[64];
@@ -41,38 +72,46 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const float* __restri
   }
   __syncthreads();
   if (bad) return;
-  const int H4 = H >> 2;
-  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < H4; c += gridDim.x * blockDim.x) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int HV = H / V;
+  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < HV; c += gridDim.x * blockDim.x) {
+    float acc[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) acc[i] = 0.f;
 #pragma unroll 8
     for (int j = 0; j < k; ++j) {
-      float4 v = __ldcs(reinterpret_cast<const float4*>(o + (size_t)srow[j] * H) + c);
+      float v[V];
+      Vec<OT>::load(o + (size_t)srow[j] * H + V * c, v);
       for (int sp = 1; sp < nsplit; ++sp) {  // K-split partial slabs of the down GEMM, in slab order
-        const float4 p = __ldcs(reinterpret_cast<const float4*>(o + sp * split_stride + (size_t)srow[j] * H) + c);
-        v.x += p.x;
-        v.y += p.y;
-        v.z += p.z;
-        v.w += p.w;
+        float p[V];
+        Vec<OT>::load(o + sp * split_stride + (size_t)srow[j] * H + V * c, p);
+#pragma unroll
+        for (int i = 0; i < V; ++i) v[i] += p[i];
       }
       const float wj = sw[j];
-      acc.x = fmaf(wj, v.x, acc.x);
-      acc.y = fmaf(wj, v.y, acc.y);
-      acc.z = fmaf(wj, v.z, acc.z);
-      acc.w = fmaf(wj, v.w, acc.w);
+#pragma unroll
+      for (int i = 0; i < V; ++i) acc[i] = fmaf(wj, v[i], acc[i]);
     }
     if (shared) {
-      const float4 s = __ldcs(reinterpret_cast<const float4*>(shared + (size_t)t * H) + c);
-      acc.x += s.x;
-      acc.y += s.y;
-      acc.z += s.z;
-      acc.w += s.w;
+#pragma unroll
+      for (int q = 0; q < V; q += 4) {
+        const float4 sv = __ldcs(reinterpret_cast<const float4*>(shared + (size_t)t * H + V * c + q));
+        acc[q] += sv.x;
+        acc[q + 1] += sv.y;
+        acc[q + 2] += sv.z;
+        acc[q + 3] += sv.w;
+      }
     }
-    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-    uint2 packed;
-    packed.x = *reinterpret_cast<uint32_t*>(&lo);
-    packed.y = *reinterpret_cast<uint32_t*>(&hi);
-    reinterpret_cast<uint2*>(y + (size_t)t * H)[c] = packed;
+    uint32_t packed[V / 2];
+#pragma unroll
+    for (int i = 0; i < V / 2; ++i) {
+      __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+      packed[i] = *reinterpret_cast<uint32_t*>(&b2);
+    }
+    if constexpr (V == 8) {
+      reinterpret_cast<uint4*>(y + (size_t)t * H)[c] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    } else {
+      reinterpret_cast<uint2*>(y + (size_t)t * H)[c] = make_uint2(packed[0], packed[1]);
+    }
   }
 }
 
@@ -115,23 +154,40 @@ cudaError_t launch_swiglu_reduce(const float* partials, int nsplit, size_t split
   return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const float* o, const float* topk_w, const int32_t* inv_perm, const float* shared, int T,
-                           int H, int k, int rows, int nsplit, size_t split_stride, uint16_t* y, DevStatus* st,
-                           cudaStream_t s) {
+namespace {
+
+template <typename OT>
+cudaError_t launch_combine_t(const OT* o, const float* topk_w, const int32_t* inv_perm, const float* shared, int T,
+                             int H, int k, int rows, int nsplit, size_t split_stride, uint16_t* y, DevStatus* st,
+                             cudaStream_t s) {
   if (k > 64) return cudaErrorInvalidValue;
   // Few tokens: split each row over several blocks so every SM has work;
-  // many tokens: one block per token, each thread looping over its float4s.
-  const int slices_max = (H / 4 + kThreads - 1) / kThreads;
+  // many tokens: one block per token, each thread looping over its vectors.
+  const int slices_max = (H / Vec<OT>::V + kThreads - 1) / kThreads;
   int slices = (2 * 148 + T - 1) / T;
   slices = slices < 1 ? 1 : (slices > slices_max ? slices_max : slices);
   for (int t0 = 0; t0 < T; t0 += 65535) {  // grid.y limit
     const dim3 grid(slices, T - t0 < 65535 ? T - t0 : 65535);
-    combine_kernel<<<grid, kThreads, 0, s>>>(o, topk_w, inv_perm, shared, H, k, rows, nsplit, split_stride,
-                                             reinterpret_cast<__nv_bfloat16*>(y), st, t0);
+    combine_kernel<OT><<<grid, kThreads, 0, s>>>(o, topk_w, inv_perm, shared, H, k, rows, nsplit, split_stride,
+                                                 reinterpret_cast<__nv_bfloat16*>(y), st, t0);
     const cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
   return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const float* o, const float* topk_w, const int32_t* inv_perm, const float* shared, int T,
+                           int H, int k, int rows, int nsplit, size_t split_stride, uint16_t* y, DevStatus* st,
+                           cudaStream_t s) {
+  return launch_combine_t(o, topk_w, inv_perm, shared, T, H, k, rows, nsplit, split_stride, y, st, s);
+}
+
+cudaError_t launch_combine_bf16(const uint16_t* o, const float* topk_w, const int32_t* inv_perm, const float* shared,
+                                int T, int H, int k, int rows, uint16_t* y, DevStatus* st, cudaStream_t s) {
+  return launch_combine_t(reinterpret_cast<const __nv_bfloat16*>(o), topk_w, inv_perm, shared, T, H, k, rows, 1, 0, y,
+                          st, s);
 }
 
 }  // namespace moe

@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 out[(size_t)(un.row0 + c0 + j) * a.ld_out + col] = __float2bfloat16_rn(silu_f(g[j]) * v[j]);
             }
           }
-        } else {
+        } else if (EPI == EPI_STORE_F32) {
           float* out = reinterpret_cast<float*>(a.out) + (size_t)un.ks * a.split_stride;
 #pragma unroll
           for (int t = 0; t < MT; ++t) {
@@ -294,6 +294,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
                 if (j < nr) out[(size_t)(un.row0 + c0 + j) * a.ld_out + ct] = v[j];
+              }
+            }
+          }
+        } else {
+          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+#pragma unroll
+          for (int t = 0; t < MT; ++t) {
+            float v[32];
+            tmem_ld_2x16(tbase + t * NT + c0, tbase + t * NT + c0 + 16, v, v + 16);
+            const int ct = col + t * a.out_col1_off;
+            if (ct < a.n_valid) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                if (j < nr) out[(size_t)(un.row0 + c0 + j) * a.ld_out + ct] = __float2bfloat16_rn(v[j]);
               }
             }
           }
@@ -337,13 +351,19 @@ int gemm_tiles_per_unit(int tiles, int epilogue) {
 cudaError_t launch_grouped_gemm(const CUtensorMap& wmap, const GemmArgs& a, int epilogue, int tiles, int num_sms,
                                 cudaStream_t stream) {
   if (tiles == MOE_TILES_LARGE) {
-    return epilogue == EPI_SWIGLU ? launch_cfg<256, 3, 2, EPI_SWIGLU>(wmap, a, num_sms, stream)
-                                  : launch_cfg<256, 3, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
+    switch (epilogue) {
+      case EPI_SWIGLU: return launch_cfg<256, 3, 2, EPI_SWIGLU>(wmap, a, num_sms, stream);
+      case EPI_STORE_F32: return launch_cfg<256, 3, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
+      default: return launch_cfg<256, 3, 2, EPI_STORE_BF16>(wmap, a, num_sms, stream);
+    }
   }
   // Small groups (decode): 128-row passes, 4 stages -- measured ~5% faster
   // than 64-row passes with 5 stages at 1-30 rows per expert.
-  return epilogue == EPI_SWIGLU ? launch_cfg<128, 4, 2, EPI_SWIGLU>(wmap, a, num_sms, stream)
-                                : launch_cfg<128, 4, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
+  switch (epilogue) {
+    case EPI_SWIGLU: return launch_cfg<128, 4, 2, EPI_SWIGLU>(wmap, a, num_sms, stream);
+    case EPI_STORE_F32: return launch_cfg<128, 4, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
+    default: return launch_cfg<128, 4, 2, EPI_STORE_BF16>(wmap, a, num_sms, stream);
+  }
 }
 
 }  // namespace moe

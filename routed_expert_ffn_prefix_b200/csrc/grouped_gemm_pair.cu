@@ -1,26 +1,21 @@
 // grouped_gemm_pair.cu -- grouped expert GEMM on SM pairs (tcgen05 cta_group::2).
 //
-// A variant of the grouped GEMM for groups that fill 256-row tiles
-// (grouped_gemm.cu has the design notes shared by both; this one is selected
-// with MOE_TILES_PAIR).  Here the token rows are the MMA's M side and one MMA
-// spans two SMs of a cluster (M = 256: 128 rows in each SM's TMEM), with
-// N = 256 weight columns of which each SM loads half.  The MMA work per
-// weight byte is fixed at the full 256 rows, so groups with fewer rows pay
-// for padding; measured on 512 experts x ~160 rows it is slower than the
-// single-SM kernel, which adapts N to the rows.
+// The variant of the grouped GEMM selected with MOE_TILES_PAIR
+// (grouped_gemm.cu has the design notes shared by both).  Same orientation
+// as the single-SM kernel -- weight columns are the MMA's M side, the
+// expert's token rows its N side -- but one MMA spans the two SMs of a
+// cluster: M = 256 weight columns (128 in each SM's TMEM lanes), N = the
+// unit's rows rounded up to 16 (<= 256), of which each SM gathers half.
 //
-//   * gate/up: N = [128 gate | 128 up] columns of the same 128 intermediate
-//     units, so each thread of the epilogue holds gate and up for its row in
-//     its own TMEM lane: SwiGLU is thread-local and each thread writes 64
-//     contiguous bytes of h per 32-column chunk (16-byte vector stores);
-//   * down: N = 256 adjacent output columns, fp32 rows stored likewise.
+// Why: at prefill sizes (~160 rows per expert) the single-SM kernel is paced
+// by the gathered token rows (32 KB per 64-deep stage at 256 rows) and only
+// three stages fit in shared memory.  Here each SM stages 32 KB of weights
+// (its 128 columns of the two tiles) but only 16 KB of rows, so four stages
+// fit, and every SM still streams each weight byte once per 256-row pass.
 //
-// Per SM and pipeline stage: 128 gathered token rows (16 KB, cp.async,
-// 128-byte swizzle, K-major) + half of the weight tile (16 KB, TMA, MN-major)
-// = 32 KB, so six stages fit, and the accumulator (256 TMEM columns) is
-// double-buffered: the weight stream from HBM never waits for an epilogue.
-// Each SM streams a disjoint half of every weight tile exactly once per
-// 256-row pass.
+//   * gate/up: the two tiles are the gate and the up columns of the same 256
+//     intermediate units (128 per SM), so SwiGLU stays thread-local;
+//   * down: the two tiles are 2 x 256 adjacent output columns.
 //
 // Synchronisation (cluster of 2; rank 0 = leader issues every MMA):
 //   full[s]  (leader): 128 cp.async arrivals of the leader's rows, the
@@ -30,13 +25,13 @@
 //   xfull[s] (peer):   the peer's 128 cp.async arrivals; the peer's relay
 //            thread waits on it, fences the writes into the async proxy and
 //            arrives on the leader's full[s].
-//   empty[s], tfull[b] (both): arrived by the leader's commits, multicast to
+//   empty[s], tfull (both): arrived by the leader's commits, multicast to
 //            both SMs of the pair.
-//   tempty[b] (leader): one arrival per epilogue warp of both SMs.
+//   tempty (leader): one arrival per epilogue warp of both SMs.
 // Every wait is bounded; both SMs meet at a cluster barrier before TMEM is
 // released and the blocks exit.
 //
-// Warp roles (320 threads): warps 0-7 epilogue, warps 8-11 producers
+// Warp roles (416 threads): warps 0-7 epilogue, warps 8-11 producers
 // (cp.async rows; thread 0 also issues the weight TMA), warp 12: TMEM
 // allocation, MMA issue (leader) or completion relay (peer).
 #include "gemm_units.cuh"
@@ -45,21 +40,23 @@ namespace moe {
 
 namespace {
 
-constexpr int kPNt = 256;       // token rows per pair unit (128 per SM)
-constexpr int kPRows = 128;     // token rows per SM
-constexpr int kPStages = 6;
+constexpr int kPNt = 256;        // token rows per pair unit (N <= 256, half per SM)
+constexpr int kPRowsMax = kPNt / 2;
+constexpr int kPStages = 4;
 constexpr int kPEpiWarps = 8;
 constexpr int kPProdWarps = 4;
 constexpr int kPCtlWarp = kPEpiWarps + kPProdWarps;
 constexpr int kPThreads = (kPCtlWarp + 1) * 32;
 constexpr int kPProdThreads = kPProdWarps * 32;
-constexpr int kPXBytes = kPRows * kBK * 2;   // 16 KB of rows per stage
-constexpr int kPWBytes = 128 * kBK * 2;      // 16 KB: this SM's half of the weight tile
-constexpr int kPStageBytes = kPXBytes + kPWBytes;
-constexpr int kPAccCols = 256;
-constexpr int kPTmemCols = 512;              // two accumulator buffers
+constexpr int kPBoxBytes = 64 * kBK * 2;         // 8 KB: one 64-column TMA box of weights
+constexpr int kPATileBytes = 2 * kPBoxBytes;     // 16 KB: this SM's 128 columns of one tile
+constexpr int kPABytes = 2 * kPATileBytes;       // 32 KB: both tiles
+constexpr int kPBBytes = kPRowsMax * kBK * 2;    // 16 KB: this SM's half of the token rows
+constexpr int kPStageBytes = kPABytes + kPBBytes;
+constexpr int kPTmemCols = 512;                  // two tiles x 256 columns, one buffer
 constexpr int kPSmemBytes = kPStages * kPStageBytes + 512 + 4 * (kMaxExperts + 1) + 1024;
 static_assert(kPSmemBytes <= 232448, "shared memory budget");
+static_assert(kPStageBytes % 1024 == 0, "stages must keep 1024-byte swizzle alignment");
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -142,15 +139,6 @@ __device__ __forceinline__ void mma_commit_pair_leader(uint64_t* bar) {
       : "memory");
 }
 
-__device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
 template <int EPI>
 __global__ void __launch_bounds__(kPThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap wmap, const GemmArgs a) {
@@ -160,8 +148,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
   uint64_t* xfull = full + kPStages;
   uint64_t* empty = xfull + kPStages;
   uint64_t* tfull = empty + kPStages;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* mma_done = tempty + 2;
+  uint64_t* tempty = tfull + 1;
+  uint64_t* mma_done = tempty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* total_units = abort_flag + 1;
@@ -179,10 +167,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
       mbar_init(xfull + s, kPProdThreads);     // peer rows
       mbar_init(empty + s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(tfull + b, 1);
-      mbar_init(tempty + b, 2 * kPEpiWarps);
-    }
+    mbar_init(tfull, 1);
+    mbar_init(tempty, 2 * kPEpiWarps);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -201,13 +187,13 @@ __global__ void __launch_bounds__(kPThreads, 1)
 
   if (warp >= kPEpiWarps && warp < kPCtlWarp) {
     // ------------------------------------------------------------ producers
+    // This SM gathers rows [rank * nh, rank * nh + nh) of the unit (nh = N/2)
+    // and loads its 128 weight columns of both tiles.
     const WaitCtx wc{a.status, abort_flag, a.timeout_ns, SITE_GEMM_PRODUCER};
     const int pt = tid - kPEpiWarps * 32;
     const int chunk = pt & 7, rsub = pt >> 3;
-    constexpr int kRowsPerThread = kPRows / (kPProdThreads / 8);
-    // Weight tiles are streamed past L2 (evict-first): keeping them (even for
-    // groups with several row passes) measured slower, because it displaces
-    // the token rows, which every column block of the group reads again.
+    constexpr int kRowsPerThread = kPRowsMax / (kPProdThreads / 8);
+    // Weight tiles are streamed past L2 (evict-first), as in the single-SM kernel.
     const uint64_t pol_w = policy_evict_first();
     const uint64_t pol_rows = a.rows_evict_last ? policy_evict_last() : policy_evict_normal();
     const __nv_bfloat16* bsrc = reinterpret_cast<const __nv_bfloat16*>(a.b_src);
@@ -218,14 +204,15 @@ __global__ void __launch_bounds__(kPThreads, 1)
     bool ok = true;
     for (int u = pair; u < total && ok; u += npairs) {
       const Unit un = decode_unit<kPNt>(a, ustart, ngroups, u);
-      const int my0 = (int)rank * kPRows;  // this SM's first row of the unit
+      const int nh = ((un.rows + 15) & ~15) >> 1;
+      const int my0 = (int)rank * nh;
       int src[kRowsPerThread];
 #pragma unroll
       for (int i = 0; i < kRowsPerThread; ++i) {
-        const int c = my0 + rsub + 16 * i;
+        const int c = rsub + 16 * i;
         int sr = -1;
-        if (c < un.rows) {
-          const int r = un.row0 + c;
+        if (c < nh && my0 + c < un.rows) {
+          const int r = un.row0 + my0 + c;
           sr = a.row_index ? __ldg(a.row_index + r) : r;
           if (sr < 0 || sr >= a.src_rows) {
             raise_error(a.status, MOE_ERR_DEVICE_BOUNDS, SITE_GEMM_GATHER, r);
@@ -234,29 +221,32 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
         src[i] = sr;
       }
-      const int wcol = un.nb * a.col_stride + (int)rank * a.col1_off;  // this SM's weight-column half
+      const int wcol = un.nb * a.col_stride + (int)rank * 128;  // this SM's 128 columns of tile 0
       const int nk = un.ke - un.kb, kiters = nk * a.krep;
       for (int it = 0; it < kiters; ++it) {
         const int rep = it / nk, kt = un.kb + (it - rep * nk);
         if (!mbar_wait(&empty[stage], phase ^ 1u, wc, 100 + stage)) { ok = false; break; }
-        uint8_t* sX = smem + stage * kPStageBytes;
-        uint8_t* sW = sX + kPXBytes;
-        const uint32_t sx = smem_u32(sX);
+        uint8_t* sA = smem + stage * kPStageBytes;
+        const uint32_t sb = smem_u32(sA + kPABytes);
 #pragma unroll
         for (int i = 0; i < kRowsPerThread; ++i) {
           if (src[i] >= 0) {
             const int c = rsub + 16 * i;
-            cp_async_16(sx + c * 128 + ((chunk ^ (c & 7)) << 4), bsrc + (size_t)src[i] * a.K + kt * kBK + chunk * 8,
+            cp_async_16(sb + c * 128 + ((chunk ^ (c & 7)) << 4), bsrc + (size_t)src[i] * a.K + kt * kBK + chunk * 8,
                         pol_rows);
           }
         }
         cp_async_arrive_noinc(&rows_bar_base[stage]);
         if (pt == 0) {
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kPWBytes);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kPABytes);
           const int d2 = a.a_dim2_rep ? rep : un.group;
           const uint32_t fb = full_leader + stage * 8;
-          tma_load_3d_pair(sW, &wmap, fb, wcol, kt * kBK, d2, pol_w);
-          tma_load_3d_pair(sW + kPWBytes / 2, &wmap, fb, wcol + 64, kt * kBK, d2, pol_w);
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const int c = wcol + t * a.col1_off;
+            tma_load_3d_pair(sA + t * kPATileBytes, &wmap, fb, c, kt * kBK, d2, pol_w);
+            tma_load_3d_pair(sA + t * kPATileBytes + kPBoxBytes, &wmap, fb, c + 64, kt * kBK, d2, pol_w);
+          }
         }
         if (++stage == kPStages) { stage = 0; phase ^= 1u; }
       }
@@ -275,38 +265,40 @@ __global__ void __launch_bounds__(kPThreads, 1)
       // ---------------------------------------------------------- MMA issuer
       if (lane == 0) {
         const WaitCtx wc{a.status, abort_flag, a.timeout_ns, SITE_GEMM_MMA};
-        // A = token rows (K-major), B = weights (MN-major), M = 256 over the pair, N = 256.
-        const uint32_t idesc = idesc_bf16_f32(256, 256, false, true);
         int stage = 0;
         uint32_t phase = 0;
         int acc_it = 0;
         bool ok = true;
         for (int u = pair; u < total && ok; u += npairs) {
           const Unit un = decode_unit<kPNt>(a, ustart, ngroups, u);
-          const int buf = acc_it & 1;
-          const uint32_t apar = (acc_it >> 1) & 1;
-          if (!mbar_wait(&tempty[buf], apar ^ 1u, wc, 200 + buf)) break;
+          if (!mbar_wait(tempty, (acc_it & 1) ^ 1u, wc, 200)) break;
           tc_fence_after();
-          const uint32_t d = tmem + buf * kPAccCols;
+          // A = weights (MN-major), M = 256 over the pair; B = rows (K-major), N = rows rounded to 16.
+          const int N = (un.rows + 15) & ~15;
+          const uint32_t idesc = idesc_bf16_f32(256, N, /*A MN-major*/ true, /*B K-major*/ false);
           const int kiters = (un.ke - un.kb) * a.krep;
           uint32_t acc = 0;
           for (int it = 0; it < kiters; ++it) {
             if (!mbar_wait(&full[stage], phase, wc, 300 + stage)) { ok = false; break; }
             tc_fence_after();
             fence_proxy_async_smem();
-            const uint32_t sx = smem_u32(smem + stage * kPStageBytes), sw = sx + kPXBytes;
+            const uint32_t sa = smem_u32(smem + stage * kPStageBytes), sb = sa + kPABytes;
 #pragma unroll
             for (int kk = 0; kk < kBK / 16; ++kk) {
-              const uint64_t ad = smem_desc_sw128(sx + kk * 32, 16, 1024);     // rows: +16 k = 32 B
-              const uint64_t bd = smem_desc_sw128(sw + kk * 2048, 8192, 1024); // weights: +16 k = 2048 B
-              mma_bf16_pair(d, ad, bd, idesc, acc);
+              const uint64_t bd = smem_desc(sb + kk * 32, 16, 1024, kLayoutSw128);  // rows: +16 k = 32 B
+#pragma unroll
+              for (int t = 0; t < 2; ++t) {
+                // weights: +16 k = two 8-row groups = 2048 B; 64-column halves one box apart
+                const uint64_t ad = smem_desc_sw128(sa + t * kPATileBytes + kk * 2048, kPBoxBytes, 1024);
+                mma_bf16_pair(tmem + t * kPNt, ad, bd, idesc, acc);
+              }
               acc = 1;
             }
             mma_commit_pair(&empty[stage]);
             if (++stage == kPStages) { stage = 0; phase ^= 1u; }
           }
           if (!ok) break;
-          mma_commit_pair(&tfull[buf]);
+          mma_commit_pair(tfull);
           ++acc_it;
         }
         mma_commit_pair_leader(mma_done);
@@ -336,63 +328,57 @@ __global__ void __launch_bounds__(kPThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue (warps 0-7)
-    // Warp w reads TMEM lanes 32*(w%4).. = rows 32*(w%4).. of this SM's 128,
-    // and the column half (w/4): one row per thread, contiguous columns.
+    // Warp w reads TMEM lanes 32*(w%4).. = this SM's weight columns
+    // 32*(w%4).. (one column per thread) and the 32-row chunks
+    // c0 = 32*(w/4) + 64*j of the unit's rows (TMEM column = row).
     const WaitCtx wc{a.status, abort_flag, a.timeout_ns, SITE_GEMM_EPILOGUE};
     const int quarter = warp & 3, half = warp >> 2;
     const uint32_t tempty_leader = map_to_rank(smem_u32(tempty), 0);
     int acc_it = 0;
     for (int u = pair; u < total; u += npairs) {
       const Unit un = decode_unit<kPNt>(a, ustart, ngroups, u);
-      const int buf = acc_it & 1;
-      const uint32_t apar = (acc_it >> 1) & 1;
-      if (!mbar_wait(&tfull[buf], apar, wc, 400 + buf)) break;
+      if (!mbar_wait(tfull, acc_it & 1, wc, 400)) break;
       tc_fence_after();
-      const int my0 = (int)rank * kPRows;
-      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * kPAccCols;
-      const int row_in_unit = my0 + quarter * 32 + lane;
-      const bool row_ok = row_in_unit < un.rows;
-      const size_t grow = (size_t)(un.row0 + row_in_unit);
-      if (my0 + quarter * 32 < un.rows) {  // skip warps whose 32 rows are all padding
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16);
+      const int col = un.nb * a.out_col_stride + (int)rank * 128 + quarter * 32 + lane;
+      for (int c0 = half * 32; c0 < un.rows; c0 += 64) {
+        const int nr = min(32, un.rows - c0);
         if (EPI == EPI_SWIGLU) {
-          // columns [half*64, half*64+64) of gate (TMEM 0..127) and of up (TMEM 128..255)
-          const int col0 = un.nb * a.out_col_stride + half * 64;
-          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + grow * a.ld_out + col0;
+          float g[32], v[32];
+          tmem_ld_4x16(tbase + c0, tbase + c0 + 16, tbase + kPNt + c0, tbase + kPNt + c0 + 16, g, g + 16, v, v + 16);
+          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+          if (col < a.n_valid) {
 #pragma unroll
-          for (int c = 0; c < 64; c += 32) {
-            float g[32], v[32];
-            const uint32_t tg = tbase + half * 64 + c, tu = tbase + 128 + half * 64 + c;
-            tmem_ld_4x16(tg, tg + 16, tu, tu + 16, g, g + 16, v, v + 16);
-            if (row_ok && col0 + c < a.n_valid) {
-#pragma unroll
-              for (int q = 0; q < 32; q += 8) {
-                st_global_v4(out + c + q, pack_bf16x2(silu_f(g[q]) * v[q], silu_f(g[q + 1]) * v[q + 1]),
-                             pack_bf16x2(silu_f(g[q + 2]) * v[q + 2], silu_f(g[q + 3]) * v[q + 3]),
-                             pack_bf16x2(silu_f(g[q + 4]) * v[q + 4], silu_f(g[q + 5]) * v[q + 5]),
-                             pack_bf16x2(silu_f(g[q + 6]) * v[q + 6], silu_f(g[q + 7]) * v[q + 7]));
-              }
+            for (int j = 0; j < 32; ++j) {
+              if (j < nr)
+                out[(size_t)(un.row0 + c0 + j) * a.ld_out + col] = __float2bfloat16_rn(silu_f(g[j]) * v[j]);
             }
           }
         } else {
-          // output columns [half*128, half*128+128) of the unit's 256
-          const int col0 = un.nb * a.out_col_stride + half * 128;
-          float* out = reinterpret_cast<float*>(a.out) + (size_t)un.ks * a.split_stride + grow * a.ld_out + col0;
 #pragma unroll
-          for (int c = 0; c < 128; c += 32) {
+          for (int t = 0; t < 2; ++t) {
             float v[32];
-            tmem_ld_2x16(tbase + half * 128 + c, tbase + half * 128 + c + 16, v, v + 16);
-            if (row_ok && col0 + c < a.n_valid) {
+            tmem_ld_2x16(tbase + t * kPNt + c0, tbase + t * kPNt + c0 + 16, v, v + 16);
+            const int ct = col + t * a.out_col1_off;
+            if (ct < a.n_valid) {
+              if (EPI == EPI_STORE_F32) {
+                float* out = reinterpret_cast<float*>(a.out) + (size_t)un.ks * a.split_stride;
 #pragma unroll
-              for (int q = 0; q < 32; q += 4)
-                st_global_v4(out + c + q, __float_as_uint(v[q]), __float_as_uint(v[q + 1]),
-                             __float_as_uint(v[q + 2]), __float_as_uint(v[q + 3]));
+                for (int j = 0; j < 32; ++j)
+                  if (j < nr) out[(size_t)(un.row0 + c0 + j) * a.ld_out + ct] = v[j];
+              } else {
+                __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (j < nr) out[(size_t)(un.row0 + c0 + j) * a.ld_out + ct] = __float2bfloat16_rn(v[j]);
+              }
             }
           }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) remote_arrive(tempty_leader + buf * 8);
+      if (lane == 0) remote_arrive(tempty_leader);
       ++acc_it;
     }
   }
@@ -449,8 +435,11 @@ cudaError_t launch_pair(const CUtensorMap& wmap, const GemmArgs& a, int num_sms,
 
 cudaError_t launch_grouped_gemm_pair(const CUtensorMap& wmap, const GemmArgs& a, int epilogue, int num_sms,
                                      cudaStream_t stream) {
-  return epilogue == EPI_SWIGLU ? launch_pair<EPI_SWIGLU>(wmap, a, num_sms, stream)
-                                : launch_pair<EPI_STORE_F32>(wmap, a, num_sms, stream);
+  switch (epilogue) {
+    case EPI_SWIGLU: return launch_pair<EPI_SWIGLU>(wmap, a, num_sms, stream);
+    case EPI_STORE_F32: return launch_pair<EPI_STORE_F32>(wmap, a, num_sms, stream);
+    default: return launch_pair<EPI_STORE_BF16>(wmap, a, num_sms, stream);
+  }
 }
 
 }  // namespace moe
