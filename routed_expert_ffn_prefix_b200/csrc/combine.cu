@@ -56,6 +56,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const OT* __restrict_
                                                          __nv_bfloat16* __restrict__ y, DevStatus* st, int t0) {
   constexpr int V = Vec<OT>::V;
   const int t = t0 + blockIdx.y;
+  pdl_enter();
   __shared__ int32_t srow[64];
   __shared__ float sw[64];
   __shared__ int bad;
@@ -77,19 +78,37 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const OT* __restrict_
     float acc[V];
 #pragma unroll
     for (int i = 0; i < V; ++i) acc[i] = 0.f;
-#pragma unroll 8
-    for (int j = 0; j < k; ++j) {
-      float v[V];
-      Vec<OT>::load(o + (size_t)srow[j] * H + V * c, v);
-      for (int sp = 1; sp < nsplit; ++sp) {  // K-split partial slabs of the down GEMM, in slab order
-        float p[V];
-        Vec<OT>::load(o + sp * split_stride + (size_t)srow[j] * H + V * c, p);
+    if (nsplit == 1) {
+      // k independent row loads in flight together, then the slot-order sum
+      int j = 0;
+      for (; j + 8 <= k; j += 8) {
+        float v[8][V];
 #pragma unroll
-        for (int i = 0; i < V; ++i) v[i] += p[i];
+        for (int q = 0; q < 8; ++q) Vec<OT>::load(o + (size_t)srow[j + q] * H + V * c, v[q]);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+#pragma unroll
+          for (int i = 0; i < V; ++i) acc[i] = fmaf(sw[j + q], v[q][i], acc[i]);
       }
-      const float wj = sw[j];
+      for (; j < k; ++j) {
+        float v[V];
+        Vec<OT>::load(o + (size_t)srow[j] * H + V * c, v);
 #pragma unroll
-      for (int i = 0; i < V; ++i) acc[i] = fmaf(wj, v[i], acc[i]);
+        for (int i = 0; i < V; ++i) acc[i] = fmaf(sw[j], v[i], acc[i]);
+      }
+    } else {
+      for (int j = 0; j < k; ++j) {
+        float v[V];
+        Vec<OT>::load(o + (size_t)srow[j] * H + V * c, v);
+        for (int sp = 1; sp < nsplit; ++sp) {  // K-split partial slabs of the down GEMM, in slab order
+          float p[V];
+          Vec<OT>::load(o + sp * split_stride + (size_t)srow[j] * H + V * c, p);
+#pragma unroll
+          for (int i = 0; i < V; ++i) v[i] += p[i];
+        }
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] = fmaf(sw[j], v[i], acc[i]);
+      }
     }
     if (shared) {
 #pragma unroll
@@ -121,6 +140,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const OT* __restrict_
 __global__ void __launch_bounds__(kThreads) swiglu_reduce_kernel(const float* __restrict__ p, int nsplit,
                                                                size_t split_stride, int rows, int I,
                                                                __nv_bfloat16* __restrict__ h) {
+  pdl_enter();
   const int I4 = I >> 2;
   const long long n = (long long)rows * I4;
   for (long long q = blockIdx.x * (long long)blockDim.x + threadIdx.x; q < n; q += (long long)gridDim.x * blockDim.x) {
@@ -149,9 +169,8 @@ cudaError_t launch_swiglu_reduce(const float* partials, int nsplit, size_t split
                                  cudaStream_t s) {
   const long long n = (long long)rows * (I / 4);
   const int blocks = (int)((n + kThreads - 1) / kThreads < 4096 ? (n + kThreads - 1) / kThreads : 4096);
-  swiglu_reduce_kernel<<<blocks, kThreads, 0, s>>>(partials, nsplit, split_stride, rows, I,
-                                                   reinterpret_cast<__nv_bfloat16*>(h));
-  return cudaGetLastError();
+  return launch_pdl(swiglu_reduce_kernel, dim3(blocks), dim3(kThreads), 0, s, partials, nsplit, split_stride, rows, I,
+                    reinterpret_cast<__nv_bfloat16*>(h));
 }
 
 namespace {
@@ -168,9 +187,8 @@ cudaError_t launch_combine_t(const OT* o, const float* topk_w, const int32_t* in
   slices = slices < 1 ? 1 : (slices > slices_max ? slices_max : slices);
   for (int t0 = 0; t0 < T; t0 += 65535) {  // grid.y limit
     const dim3 grid(slices, T - t0 < 65535 ? T - t0 : 65535);
-    combine_kernel<OT><<<grid, kThreads, 0, s>>>(o, topk_w, inv_perm, shared, H, k, rows, nsplit, split_stride,
-                                                 reinterpret_cast<__nv_bfloat16*>(y), st, t0);
-    const cudaError_t err = cudaGetLastError();
+    const cudaError_t err = launch_pdl(combine_kernel<OT>, grid, dim3(kThreads), 0, s, o, topk_w, inv_perm, shared, H,
+                                       k, rows, nsplit, split_stride, reinterpret_cast<__nv_bfloat16*>(y), st, t0);
     if (err != cudaSuccess) return err;
   }
   return cudaSuccess;

@@ -40,23 +40,31 @@ namespace moe {
 
 namespace {
 
-constexpr int kPNt = 256;        // token rows per pair unit (N <= 256, half per SM)
-constexpr int kPRowsMax = kPNt / 2;
-constexpr int kPStages = 4;
 constexpr int kPEpiWarps = 8;
 constexpr int kPProdWarps = 4;
 constexpr int kPCtlWarp = kPEpiWarps + kPProdWarps;
 constexpr int kPThreads = (kPCtlWarp + 1) * 32;
 constexpr int kPProdThreads = kPProdWarps * 32;
-constexpr int kPBoxBytes = 64 * kBK * 2;         // 8 KB: one 64-column TMA box of weights
-constexpr int kPATileBytes = 2 * kPBoxBytes;     // 16 KB: this SM's 128 columns of one tile
-constexpr int kPABytes = 2 * kPATileBytes;       // 32 KB: both tiles
-constexpr int kPBBytes = kPRowsMax * kBK * 2;    // 16 KB: this SM's half of the token rows
-constexpr int kPStageBytes = kPABytes + kPBBytes;
-constexpr int kPTmemCols = 512;                  // two tiles x 256 columns, one buffer
-constexpr int kPSmemBytes = kPStages * kPStageBytes + 512 + 4 * (kMaxExperts + 1) + 1024;
-static_assert(kPSmemBytes <= 232448, "shared memory budget");
-static_assert(kPStageBytes % 1024 == 0, "stages must keep 1024-byte swizzle alignment");
+constexpr int kPBoxBytes = 64 * kBK * 2;  // 8 KB: one 64-column TMA box of weights
+constexpr int kPATileBytes = 2 * kPBoxBytes;  // 16 KB: this SM's 128 columns of one tile
+
+// NT: rows per pass (N <= NT, NT/2 gathered per SM); ST: pipeline stages;
+// MT: MMA tiles per unit (gate + up, or 1-2 output blocks of 256 columns).
+template <int NT, int ST, int MT>
+struct PCfg {
+  static constexpr int ROWS = NT / 2;
+  static constexpr int A_BYTES = MT * kPATileBytes;
+  static constexpr int B_BYTES = ROWS * kBK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int NBUF = (2 * MT * NT <= 512) ? 2 : 1;  // accumulators double-buffered if they fit
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int SMEM_BYTES = ST * STAGE_BYTES + 512 + 4 * (kMaxExperts + 1) + 1024;
+  static_assert(NT % 32 == 0 && NT >= 32 && NT <= 256, "row pass must be 32..256, multiple of 32");
+  static_assert(MT == 1 || MT == 2, "one or two MMA tiles per unit");
+  static_assert(MT * NT * NBUF <= TMEM_COLS, "accumulators must fit in TMEM");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte swizzle alignment");
+};
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -139,21 +147,23 @@ __device__ __forceinline__ void mma_commit_pair_leader(uint64_t* bar) {
       : "memory");
 }
 
-template <int EPI>
+template <int NT, int ST, int MT, int EPI>
 __global__ void __launch_bounds__(kPThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap wmap, const GemmArgs a) {
+  using C = PCfg<NT, ST, MT>;
+  static_assert(EPI != EPI_SWIGLU || MT == 2, "SwiGLU needs the gate and the up tile");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPStages * kPStageBytes);
-  uint64_t* xfull = full + kPStages;
-  uint64_t* empty = xfull + kPStages;
-  uint64_t* tfull = empty + kPStages;
-  uint64_t* tempty = tfull + 1;
-  uint64_t* mma_done = tempty + 1;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * C::STAGE_BYTES);
+  uint64_t* xfull = full + ST;
+  uint64_t* empty = xfull + ST;
+  uint64_t* tfull = empty + ST;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* total_units = abort_flag + 1;
-  int* ustart = reinterpret_cast<int*>(smem + kPStages * kPStageBytes + 512);
+  int* ustart = reinterpret_cast<int*>(smem + ST * C::STAGE_BYTES + 512);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_rank();
@@ -162,23 +172,26 @@ __global__ void __launch_bounds__(kPThreads, 1)
   const int ngroups = a.offsets ? a.groups : 1;
 
   if (tid == 0) {
-    for (int s = 0; s < kPStages; ++s) {
+    for (int s = 0; s < ST; ++s) {
       mbar_init(full + s, kPProdThreads + 2);  // leader rows + leader expect_tx + peer relay
       mbar_init(xfull + s, kPProdThreads);     // peer rows
       mbar_init(empty + s, 1);
     }
-    mbar_init(tfull, 1);
-    mbar_init(tempty, 2 * kPEpiWarps);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull + b, 1);
+      mbar_init(tempty + b, 2 * kPEpiWarps);
+    }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) build_unit_prefix<kPNt>(a, ngroups, ustart, total_units);
   if (warp == kPCtlWarp) {
-    tmem_alloc_pair(tmem_slot, kPTmemCols);
+    tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
     tmem_relinquish_pair();
   }
   if (warp == kPEpiWarps && lane == 0) prefetch_tmap(&wmap);
+  pdl_enter();  // offsets, rows and outputs belong to the kernels before this one
+  if (warp == 0) build_unit_prefix<NT>(a, ngroups, ustart, total_units);
   tc_fence_before();
   cluster_sync();  // barriers of both SMs initialised before any remote arrive
   tc_fence_after();
@@ -192,7 +205,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const WaitCtx wc{a.status, abort_flag, a.timeout_ns, SITE_GEMM_PRODUCER};
     const int pt = tid - kPEpiWarps * 32;
     const int chunk = pt & 7, rsub = pt >> 3;
-    constexpr int kRowsPerThread = kPRowsMax / (kPProdThreads / 8);
+    constexpr int kRowsPerThread = C::ROWS / (kPProdThreads / 8);
     // Weight tiles are streamed past L2 (evict-first), as in the single-SM kernel.
     const uint64_t pol_w = policy_evict_first();
     const uint64_t pol_rows = a.rows_evict_last ? policy_evict_last() : policy_evict_normal();
@@ -203,7 +216,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     uint32_t phase = 0;
     bool ok = true;
     for (int u = pair; u < total && ok; u += npairs) {
-      const Unit un = decode_unit<kPNt>(a, ustart, ngroups, u);
+      const Unit un = decode_unit<NT>(a, ustart, ngroups, u);
       const int nh = ((un.rows + 15) & ~15) >> 1;
       const int my0 = (int)rank * nh;
       int src[kRowsPerThread];
@@ -226,8 +239,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
       for (int it = 0; it < kiters; ++it) {
         const int rep = it / nk, kt = un.kb + (it - rep * nk);
         if (!mbar_wait(&empty[stage], phase ^ 1u, wc, 100 + stage)) { ok = false; break; }
-        uint8_t* sA = smem + stage * kPStageBytes;
-        const uint32_t sb = smem_u32(sA + kPABytes);
+        uint8_t* sA = smem + stage * C::STAGE_BYTES;
+        const uint32_t sb = smem_u32(sA + C::A_BYTES);
 #pragma unroll
         for (int i = 0; i < kRowsPerThread; ++i) {
           if (src[i] >= 0) {
@@ -238,17 +251,17 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
         cp_async_arrive_noinc(&rows_bar_base[stage]);
         if (pt == 0) {
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kPABytes);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::A_BYTES);
           const int d2 = a.a_dim2_rep ? rep : un.group;
           const uint32_t fb = full_leader + stage * 8;
 #pragma unroll
-          for (int t = 0; t < 2; ++t) {
+          for (int t = 0; t < MT; ++t) {
             const int c = wcol + t * a.col1_off;
             tma_load_3d_pair(sA + t * kPATileBytes, &wmap, fb, c, kt * kBK, d2, pol_w);
             tma_load_3d_pair(sA + t * kPATileBytes + kPBoxBytes, &wmap, fb, c + 64, kt * kBK, d2, pol_w);
           }
         }
-        if (++stage == kPStages) { stage = 0; phase ^= 1u; }
+        if (++stage == ST) { stage = 0; phase ^= 1u; }
       }
     }
     cp_async_wait_all();
@@ -270,9 +283,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
         int acc_it = 0;
         bool ok = true;
         for (int u = pair; u < total && ok; u += npairs) {
-          const Unit un = decode_unit<kPNt>(a, ustart, ngroups, u);
-          if (!mbar_wait(tempty, (acc_it & 1) ^ 1u, wc, 200)) break;
+          const Unit un = decode_unit<NT>(a, ustart, ngroups, u);
+          const int buf = C::NBUF == 2 ? (acc_it & 1) : 0;
+          const uint32_t apar = C::NBUF == 2 ? ((acc_it >> 1) & 1) : (acc_it & 1);
+          if (!mbar_wait(&tempty[buf], apar ^ 1u, wc, 200 + buf)) break;
           tc_fence_after();
+          const uint32_t d0 = tmem + buf * MT * NT;
           // A = weights (MN-major), M = 256 over the pair; B = rows (K-major), N = rows rounded to 16.
           const int N = (un.rows + 15) & ~15;
           const uint32_t idesc = idesc_bf16_f32(256, N, /*A MN-major*/ true, /*B K-major*/ false);
@@ -282,23 +298,23 @@ __global__ void __launch_bounds__(kPThreads, 1)
             if (!mbar_wait(&full[stage], phase, wc, 300 + stage)) { ok = false; break; }
             tc_fence_after();
             fence_proxy_async_smem();
-            const uint32_t sa = smem_u32(smem + stage * kPStageBytes), sb = sa + kPABytes;
+            const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES), sb = sa + C::A_BYTES;
 #pragma unroll
             for (int kk = 0; kk < kBK / 16; ++kk) {
               const uint64_t bd = smem_desc(sb + kk * 32, 16, 1024, kLayoutSw128);  // rows: +16 k = 32 B
 #pragma unroll
-              for (int t = 0; t < 2; ++t) {
+              for (int t = 0; t < MT; ++t) {
                 // weights: +16 k = two 8-row groups = 2048 B; 64-column halves one box apart
                 const uint64_t ad = smem_desc_sw128(sa + t * kPATileBytes + kk * 2048, kPBoxBytes, 1024);
-                mma_bf16_pair(tmem + t * kPNt, ad, bd, idesc, acc);
+                mma_bf16_pair(d0 + t * NT, ad, bd, idesc, acc);
               }
               acc = 1;
             }
             mma_commit_pair(&empty[stage]);
-            if (++stage == kPStages) { stage = 0; phase ^= 1u; }
+            if (++stage == ST) { stage = 0; phase ^= 1u; }
           }
           if (!ok) break;
-          mma_commit_pair(tfull);
+          mma_commit_pair(&tfull[buf]);
           ++acc_it;
         }
         mma_commit_pair_leader(mma_done);
@@ -315,13 +331,13 @@ __global__ void __launch_bounds__(kPThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int u = pair; u < total && ok; u += npairs) {
-        const Unit un = decode_unit<kPNt>(a, ustart, ngroups, u);
+        const Unit un = decode_unit<NT>(a, ustart, ngroups, u);
         const int kiters = (un.ke - un.kb) * a.krep;
         for (int it = 0; it < kiters; ++it) {
           if (!mbar_wait(&xfull[stage], phase, wc, 500 + stage)) { ok = false; break; }
           fence_proxy_async_smem();
           remote_arrive_relaxed(full_leader + stage * 8);
-          if (++stage == kPStages) { stage = 0; phase ^= 1u; }
+          if (++stage == ST) { stage = 0; phase ^= 1u; }
         }
       }
     }
@@ -336,16 +352,18 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const uint32_t tempty_leader = map_to_rank(smem_u32(tempty), 0);
     int acc_it = 0;
     for (int u = pair; u < total; u += npairs) {
-      const Unit un = decode_unit<kPNt>(a, ustart, ngroups, u);
-      if (!mbar_wait(tfull, acc_it & 1, wc, 400)) break;
+      const Unit un = decode_unit<NT>(a, ustart, ngroups, u);
+      const int buf = C::NBUF == 2 ? (acc_it & 1) : 0;
+      const uint32_t apar = C::NBUF == 2 ? ((acc_it >> 1) & 1) : (acc_it & 1);
+      if (!mbar_wait(&tfull[buf], apar, wc, 400 + buf)) break;
       tc_fence_after();
-      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16);
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * MT * NT;
       const int col = un.nb * a.out_col_stride + (int)rank * 128 + quarter * 32 + lane;
       for (int c0 = half * 32; c0 < un.rows; c0 += 64) {
         const int nr = min(32, un.rows - c0);
         if (EPI == EPI_SWIGLU) {
           float g[32], v[32];
-          tmem_ld_4x16(tbase + c0, tbase + c0 + 16, tbase + kPNt + c0, tbase + kPNt + c0 + 16, g, g + 16, v, v + 16);
+          tmem_ld_4x16(tbase + c0, tbase + c0 + 16, tbase + NT + c0, tbase + NT + c0 + 16, g, g + 16, v, v + 16);
           __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
           if (col < a.n_valid) {
 #pragma unroll
@@ -356,9 +374,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
           }
         } else {
 #pragma unroll
-          for (int t = 0; t < 2; ++t) {
+          for (int t = 0; t < MT; ++t) {
             float v[32];
-            tmem_ld_2x16(tbase + t * kPNt + c0, tbase + t * kPNt + c0 + 16, v, v + 16);
+            tmem_ld_2x16(tbase + t * NT + c0, tbase + t * NT + c0 + 16, v, v + 16);
             const int ct = col + t * a.out_col1_off;
             if (ct < a.n_valid) {
               if (EPI == EPI_STORE_F32) {
@@ -378,7 +396,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) remote_arrive(tempty_leader);
+      if (lane == 0) remote_arrive(tempty_leader + buf * 8);
       ++acc_it;
     }
   }
@@ -390,21 +408,22 @@ __global__ void __launch_bounds__(kPThreads, 1)
   cluster_sync();
   if (warp == kPCtlWarp) {
     tc_fence_after();
-    tmem_dealloc_pair(tmem, kPTmemCols);
+    tmem_dealloc_pair(tmem, C::TMEM_COLS);
   }
 }
 
-template <int EPI>
+template <int NT, int ST, int MT, int EPI>
 cudaError_t launch_pair(const CUtensorMap& wmap, const GemmArgs& a, int num_sms, cudaStream_t stream) {
-  auto kern = grouped_gemm_pair_kernel<EPI>;
+  using C = PCfg<NT, ST, MT>;
+  auto kern = grouped_gemm_pair_kernel<NT, ST, MT, EPI>;
   static std::atomic<int> configured[kMaxDevices];
   cudaError_t err = once_per_device(configured, [&] {
-    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmemBytes);
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kPThreads, 1, 1);
-  cfg.dynamicSmemBytes = kPSmemBytes;
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -428,6 +447,11 @@ cudaError_t launch_pair(const CUtensorMap& wmap, const GemmArgs& a, int num_sms,
     });
     if (slots[dev] > 0 && 2 * slots[dev] < (int)cfg.gridDim.x) cfg.gridDim = dim3(2 * slots[dev], 1, 1);
   }
+  cudaLaunchAttribute attr_pdl[2] = {attr[0], {}};
+  attr_pdl[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr_pdl[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr_pdl;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, wmap, a);
 }
 
@@ -436,9 +460,14 @@ cudaError_t launch_pair(const CUtensorMap& wmap, const GemmArgs& a, int num_sms,
 cudaError_t launch_grouped_gemm_pair(const CUtensorMap& wmap, const GemmArgs& a, int epilogue, int num_sms,
                                      cudaStream_t stream) {
   switch (epilogue) {
-    case EPI_SWIGLU: return launch_pair<EPI_SWIGLU>(wmap, a, num_sms, stream);
-    case EPI_STORE_F32: return launch_pair<EPI_STORE_F32>(wmap, a, num_sms, stream);
-    default: return launch_pair<EPI_STORE_BF16>(wmap, a, num_sms, stream);
+    // 256-row passes, 4 stages.  Measured alternatives on the 8192-token
+    // prefill shape: 192-row passes with 5 stages (gate/up 1.56 vs 1.54 ms;
+    // down 0.99 vs 1.04 ms in isolation but 6% slower on Zipf-skewed routing,
+    // where hot experts need more passes), one 256-column tile per unit with a
+    // double-buffered accumulator (down 1.05 ms).
+    case EPI_SWIGLU: return launch_pair<256, 4, 2, EPI_SWIGLU>(wmap, a, num_sms, stream);
+    case EPI_STORE_F32: return launch_pair<256, 4, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
+    default: return launch_pair<256, 4, 2, EPI_STORE_BF16>(wmap, a, num_sms, stream);
   }
 }
 
