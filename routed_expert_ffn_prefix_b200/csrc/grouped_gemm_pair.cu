@@ -460,11 +460,14 @@ cudaError_t launch_pair(const CUtensorMap& wmap, const GemmArgs& a, int num_sms,
 cudaError_t launch_grouped_gemm_pair(const CUtensorMap& wmap, const GemmArgs& a, int epilogue, int num_sms,
                                      cudaStream_t stream) {
   switch (epilogue) {
-    // 256-row passes, 4 stages.  Measured alternatives on the 8192-token
-    // prefill shape: 192-row passes with 5 stages (gate/up 1.56 vs 1.54 ms;
-    // down 0.99 vs 1.04 ms in isolation but 6% slower on Zipf-skewed routing,
-    // where hot experts need more passes), one 256-column tile per unit with a
-    // double-buffered accumulator (down 1.05 ms).
+    // 256-row passes, 4 stages.  Measured alternatives (isolated kernel, in
+    // one process; 8192-token prefill shape / Zipf-skewed 4096-token shape):
+    //   gate/up 256/4: 1.58 / 3.58 ms; 192/5: 1.62 / 3.73 ms; 128/5: 2.56 / 4.52 ms
+    //   down    256/4: 1.12 / 2.07 ms; 192/5: 0.98 / 2.11 ms; 128/5: 1.45 / 2.33 ms
+    // but inside the layer, where h was just written and partly sits in L2,
+    // the 192/5 down GEMM measured slower (1.11 vs 1.07 ms; 2.32 vs 2.24 ms).
+    // One 256-column tile per unit with a double-buffered accumulator: down
+    // 1.03 / 2.35 ms.
     case EPI_SWIGLU: return launch_pair<256, 4, 2, EPI_SWIGLU>(wmap, a, num_sms, stream);
     case EPI_STORE_F32: return launch_pair<256, 4, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
     default: return launch_pair<256, 4, 2, EPI_STORE_BF16>(wmap, a, num_sms, stream);

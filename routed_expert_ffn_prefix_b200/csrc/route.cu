@@ -109,7 +109,14 @@ __device__ __forceinline__ bool topk_better(float av, int ai, float bv, int bi) 
   return av > bv || (av == bv && ai < bi);
 }
 
-template <int EPL>
+// Expert held in entry i of a lane's EPL logits: scalar layout e = lane + 32 i;
+// quad layout (16-byte loads, E % 4 == 0) e = 128 (i / 4) + 4 lane + i % 4.
+template <bool QUAD>
+__device__ __forceinline__ int entry_expert(int lane, int i) {
+  return QUAD ? 128 * (i >> 2) + 4 * lane + (i & 3) : lane + 32 * i;
+}
+
+template <int EPL, bool QUAD = false>
 __device__ __forceinline__ void warp_topk(const float (&vin)[EPL], int E, int k, int t, int32_t* idrow, float* wrow,
                                           int32_t* sel, DevStatus* st) {
   const int lane = threadIdx.x & 31;
@@ -117,7 +124,7 @@ __device__ __forceinline__ void warp_topk(const float (&vin)[EPL], int E, int k,
   int id[EPL];
 #pragma unroll
   for (int i = 0; i < EPL; ++i) {
-    const int e = lane + 32 * i;
+    const int e = entry_expert<QUAD>(lane, i);
     const bool ok = e < E && !isnan(vin[i]);
     v[i] = ok ? vin[i] : -INFINITY;
     id[i] = ok ? e : kNoExpert;
@@ -165,10 +172,32 @@ __device__ __forceinline__ void warp_topk(const float (&vin)[EPL], int E, int k,
 
 constexpr int kTopkWarps = 8;
 
+// The EPL logits of one token held by a lane (entry layout of entry_expert).
+template <int EPL, bool QUAD>
+__device__ __forceinline__ void load_logits(const float* __restrict__ row, int E, int lane, float (&v)[EPL]) {
+  if constexpr (QUAD) {
+#pragma unroll
+    for (int q = 0; q < EPL / 4; ++q) {
+      const int e0 = 128 * q + 4 * lane;
+      const float4 f = e0 < E ? *reinterpret_cast<const float4*>(row + e0) : make_float4(0.f, 0.f, 0.f, 0.f);
+      v[4 * q] = f.x;
+      v[4 * q + 1] = f.y;
+      v[4 * q + 2] = f.z;
+      v[4 * q + 3] = f.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      v[i] = e < E ? row[e] : 0.f;
+    }
+  }
+}
+
 // One warp per token; EPL = experts per lane (E <= 32 * EPL).  The K-split
 // partial slabs are summed in slab order; UNR slabs are loaded before any is
-// added so that UNR * EPL loads per lane are in flight at once.
-template <int EPL, int UNR>
+// added so that UNR * EPL values per lane are in flight at once.
+template <int EPL, int UNR, bool QUAD>
 __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __restrict__ logits, int nsplit,
                                                              size_t split_stride, const float* __restrict__ bias,
                                                              int T, int E, int k, int32_t* __restrict__ ids,
@@ -178,47 +207,36 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
   const int t = blockIdx.x * kTopkWarps + warp;
   if (t >= T) return;
   const float* row = logits + (size_t)t * E;
-  const float NEG = -INFINITY;
   float v[EPL];
-#pragma unroll
-  for (int i = 0; i < EPL; ++i) {
-    const int e = lane + 32 * i;
-    v[i] = e < E ? row[e] : 0.f;
-  }
+  load_logits<EPL, QUAD>(row, E, lane, v);
   int sp = 1;
   for (; sp + UNR <= nsplit; sp += UNR) {
     float p[UNR][EPL];
 #pragma unroll
-    for (int q = 0; q < UNR; ++q)
-#pragma unroll
-      for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        p[q][i] = e < E ? row[(size_t)(sp + q) * split_stride + e] : 0.f;
-      }
+    for (int q = 0; q < UNR; ++q) load_logits<EPL, QUAD>(row + (size_t)(sp + q) * split_stride, E, lane, p[q]);
 #pragma unroll
     for (int q = 0; q < UNR; ++q)
 #pragma unroll
       for (int i = 0; i < EPL; ++i) v[i] += p[q][i];
   }
   for (; sp < nsplit; ++sp) {
+    float p[EPL];
+    load_logits<EPL, QUAD>(row + (size_t)sp * split_stride, E, lane, p);
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E) v[i] += row[(size_t)sp * split_stride + e];
-    }
+    for (int i = 0; i < EPL; ++i) v[i] += p[i];
   }
 #pragma unroll
   for (int i = 0; i < EPL; ++i) {
-    const int e = lane + 32 * i;
-    v[i] = e < E ? v[i] + (bias ? bias[e] : 0.f) : NEG;
+    const int e = entry_expert<QUAD>(lane, i);
+    v[i] = e < E ? v[i] + (bias ? bias[e] : 0.f) : -INFINITY;
   }
-  warp_topk<EPL>(v, E, k, t, ids + (size_t)t * k, wout + (size_t)t * k, nullptr, st);
+  warp_topk<EPL, QUAD>(v, E, k, t, ids + (size_t)t * k, wout + (size_t)t * k, nullptr, st);
 }
 
-template <int EPL, int UNR>
+template <int EPL, int UNR, bool QUAD = false>
 cudaError_t launch_topk_t(const float* logits, int nsplit, size_t split_stride, const float* bias, int T, int E,
                           int k, int32_t* ids, float* w, DevStatus* st, cudaStream_t s) {
-  return launch_pdl(topk_kernel<EPL, UNR>, dim3((T + kTopkWarps - 1) / kTopkWarps), dim3(kTopkWarps * 32), 0, s,
+  return launch_pdl(topk_kernel<EPL, UNR, QUAD>, dim3((T + kTopkWarps - 1) / kTopkWarps), dim3(kTopkWarps * 32), 0, s,
                     logits, nsplit, split_stride, bias, T, E, k, ids, w, st);
 }
 
@@ -460,6 +478,13 @@ cudaError_t launch_topk(const float* logits, int nsplit, size_t split_stride, co
                         int32_t* ids, float* w, DevStatus* st, cudaStream_t s) {
   if (E <= 32) return launch_topk_t<1, 8>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
   if (E <= 64) return launch_topk_t<2, 8>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
+  // E % 4 == 0 (and 16-byte aligned rows): each lane loads 4 experts per 16-byte load
+  if (E % 4 == 0) {
+    if (E <= 128) return launch_topk_t<4, 8, true>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
+    if (E <= 256) return launch_topk_t<8, 4, true>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
+    if (E <= 512) return launch_topk_t<16, 4, true>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
+    return launch_topk_t<32, 2, true>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
+  }
   if (E <= 128) return launch_topk_t<4, 8>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
   if (E <= 256) return launch_topk_t<8, 4>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
   if (E <= 512) return launch_topk_t<16, 4>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
