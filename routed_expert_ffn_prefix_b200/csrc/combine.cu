@@ -56,7 +56,6 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const OT* __restrict_
                                                          __nv_bfloat16* __restrict__ y, DevStatus* st, int t0) {
   constexpr int V = Vec<OT>::V;
   const int t = t0 + blockIdx.y;
-  pdl_enter();
   __shared__ int32_t srow[64];
   __shared__ float sw[64];
   __shared__ int bad;
@@ -140,7 +139,6 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const OT* __restrict_
 __global__ void __launch_bounds__(kThreads) swiglu_reduce_kernel(const float* __restrict__ p, int nsplit,
                                                                size_t split_stride, int rows, int I,
                                                                __nv_bfloat16* __restrict__ h) {
-  pdl_enter();
   const int I4 = I >> 2;
   const long long n = (long long)rows * I4;
   for (long long q = blockIdx.x * (long long)blockDim.x + threadIdx.x; q < n; q += (long long)gridDim.x * blockDim.x) {
@@ -169,8 +167,8 @@ cudaError_t launch_swiglu_reduce(const float* partials, int nsplit, size_t split
                                  cudaStream_t s) {
   const long long n = (long long)rows * (I / 4);
   const int blocks = (int)((n + kThreads - 1) / kThreads < 4096 ? (n + kThreads - 1) / kThreads : 4096);
-  return launch_pdl(swiglu_reduce_kernel, dim3(blocks), dim3(kThreads), 0, s, partials, nsplit, split_stride, rows, I,
-                    reinterpret_cast<__nv_bfloat16*>(h));
+  return launch_kernel(swiglu_reduce_kernel, dim3(blocks), dim3(kThreads), 0, s, partials, nsplit, split_stride,
+                       rows, I, reinterpret_cast<__nv_bfloat16*>(h));
 }
 
 namespace {
@@ -187,8 +185,9 @@ cudaError_t launch_combine_t(const OT* o, const float* topk_w, const int32_t* in
   slices = slices < 1 ? 1 : (slices > slices_max ? slices_max : slices);
   for (int t0 = 0; t0 < T; t0 += 65535) {  // grid.y limit
     const dim3 grid(slices, T - t0 < 65535 ? T - t0 : 65535);
-    const cudaError_t err = launch_pdl(combine_kernel<OT>, grid, dim3(kThreads), 0, s, o, topk_w, inv_perm, shared, H,
-                                       k, rows, nsplit, split_stride, reinterpret_cast<__nv_bfloat16*>(y), st, t0);
+    const cudaError_t err =
+        launch_kernel(combine_kernel<OT>, grid, dim3(kThreads), 0, s, o, topk_w, inv_perm, shared, H, k, rows, nsplit,
+                      split_stride, reinterpret_cast<__nv_bfloat16*>(y), st, t0);
     if (err != cudaSuccess) return err;
   }
   return cudaSuccess;

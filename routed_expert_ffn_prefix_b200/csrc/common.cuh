@@ -54,18 +54,6 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// ---------------------------------------------------------------- programmatic dependent launch
-// Every kernel of the layer is launched with programmatic stream
-// serialisation (launch_pdl in kernels.h), so it may be scheduled while the
-// kernel before it in the stream is still running.  It first does only work
-// that reads nothing another kernel writes (barrier init, TMEM allocation,
-// descriptor prefetch), then pdl_enter(): wait until the previous grid has
-// completed and its writes are visible, and let the next kernel be scheduled.
-__device__ __forceinline__ void pdl_enter() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

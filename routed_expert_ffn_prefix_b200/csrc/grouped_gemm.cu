@@ -120,7 +120,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   if (warp == kEpiWarps && lane == 0) prefetch_tmap(&wmap);
-  pdl_enter();  // offsets, rows and outputs belong to the kernels before this one
   if (warp == 0) build_unit_prefix<NT>(a, ngroups, ustart, total_units);
   tc_fence_before();
   __syncthreads();
@@ -337,7 +336,7 @@ cudaError_t launch_cfg(const CUtensorMap& wmap, const GemmArgs& a, int num_sms, 
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (err != cudaSuccess) return err;
-  return launch_pdl(kern, dim3(num_sms), dim3(kThreads), C::SMEM_BYTES, stream, wmap, a);
+  return launch_kernel(kern, dim3(num_sms), dim3(kThreads), C::SMEM_BYTES, stream, wmap, a);
 }
 
 }  // namespace

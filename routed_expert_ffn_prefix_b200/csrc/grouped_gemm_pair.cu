@@ -190,7 +190,6 @@ __global__ void __launch_bounds__(kPThreads, 1)
     tmem_relinquish_pair();
   }
   if (warp == kPEpiWarps && lane == 0) prefetch_tmap(&wmap);
-  pdl_enter();  // offsets, rows and outputs belong to the kernels before this one
   if (warp == 0) build_unit_prefix<NT>(a, ngroups, ustart, total_units);
   tc_fence_before();
   cluster_sync();  // barriers of both SMs initialised before any remote arrive
@@ -447,11 +446,6 @@ cudaError_t launch_pair(const CUtensorMap& wmap, const GemmArgs& a, int num_sms,
     });
     if (slots[dev] > 0 && 2 * slots[dev] < (int)cfg.gridDim.x) cfg.gridDim = dim3(2 * slots[dev], 1, 1);
   }
-  cudaLaunchAttribute attr_pdl[2] = {attr[0], {}};
-  attr_pdl[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr_pdl[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr_pdl;
-  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, wmap, a);
 }
 

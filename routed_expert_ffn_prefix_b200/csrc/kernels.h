@@ -28,23 +28,15 @@ inline cudaError_t once_per_device(std::atomic<int>* done, F&& setup) {
   return err;
 }
 
-// Launches `kern` with programmatic stream serialisation: it may start while
-// the previous kernel in the stream finishes (the kernel calls pdl_enter()
-// before touching memory other kernels write).  With no PDL-capable
-// predecessor the attribute has no effect.
+// Launches `kern` on stream s (checked arguments, one call form for all kernels).
 template <typename... KArgs, typename... Args>
-inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                              Args... args) {
+inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                 Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 

@@ -38,7 +38,6 @@ __global__ void hist_kernel(const int32_t* __restrict__ ids, int n, int E, int32
                             DevStatus* st) {
   extern __shared__ int32_t h[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
-  pdl_enter();
   __syncthreads();
   const int s0 = blockIdx.x * kChunk;
   for (int i = threadIdx.x; i < kChunk; i += blockDim.x) {
@@ -62,7 +61,6 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ block_
   __shared__ int32_t tot[kMaxExperts];
   __shared__ int32_t warp_sums[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  pdl_enter();
   // block_hist[b][e] <- rows of expert e in blocks < b.  One thread per
   // expert walks its column; consecutive threads read consecutive experts
   // (coalesced) and each batch of 8 loads is issued before any is used.
@@ -122,7 +120,6 @@ __global__ void __launch_bounds__(kScatterWarps * 32) scatter_kernel(const int32
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int s0 = blockIdx.x * kChunk + w * kRun;
   for (int i = tid; i < kScatterWarps * E; i += blockDim.x) base[i] = 0;
-  pdl_enter();
   __syncthreads();
   for (int i = lane; i < kRun; i += 32) {
     const int s = s0 + i;
@@ -173,7 +170,6 @@ __global__ void __launch_bounds__(kFusedWarps * 32) permute_fused_kernel(const i
   __shared__ int32_t warp_sums[32];
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   for (int i = tid; i < kFusedWarps * E; i += blockDim.x) wh[i] = 0;
-  pdl_enter();
   __syncthreads();
   const int s0 = w * kRun;
   for (int i = lane; i < kRun; i += 32) {
@@ -255,17 +251,18 @@ cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* cou
                                   (int)((size_t)kFusedWarps * kMaxExperts * sizeof(int32_t)));
     });
     if (err != cudaSuccess) return err;
-    return launch_pdl(permute_fused_kernel, dim3(1), dim3(kFusedWarps * 32), sh, s, ids, n, E, k, counts, offsets,
-                      sorted_ids, inv_perm, st);
+    return launch_kernel(permute_fused_kernel, dim3(1), dim3(kFusedWarps * 32), sh, s, ids, n, E, k, counts, offsets,
+                         sorted_ids, inv_perm, st);
   }
   const int nblk = permute_num_blocks(T, k);
-  cudaError_t err = launch_pdl(hist_kernel, dim3(nblk), dim3(256), (size_t)E * sizeof(int32_t), s, ids, n, E,
-                               block_hist, st);
+  cudaError_t err = launch_kernel(hist_kernel, dim3(nblk), dim3(256), (size_t)E * sizeof(int32_t), s, ids, n, E,
+                                  block_hist, st);
   if (err != cudaSuccess) return err;
-  err = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, s, block_hist, nblk, E, counts, offsets);
+  err = launch_kernel(scan_kernel, dim3(1), dim3(1024), 0, s, block_hist, nblk, E, counts, offsets);
   if (err != cudaSuccess) return err;
-  return launch_pdl(scatter_kernel, dim3(nblk), dim3(kScatterWarps * 32), (size_t)kScatterWarps * E * sizeof(int32_t),
-                    s, ids, n, E, k, block_hist, offsets, sorted_ids, inv_perm);
+  return launch_kernel(scatter_kernel, dim3(nblk), dim3(kScatterWarps * 32),
+                       (size_t)kScatterWarps * E * sizeof(int32_t), s, ids, n, E, k, block_hist, offsets, sorted_ids,
+                       inv_perm);
 }
 
 }  // namespace moe

@@ -26,7 +26,6 @@ namespace moe {
 namespace {
 
 __global__ void router_split_kernel(const float* __restrict__ w, int n, uint16_t* __restrict__ planes) {
-  pdl_enter();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
     const float v = w[i];
     const __nv_bfloat16 p0 = __float2bfloat16_rn(v);
@@ -51,7 +50,6 @@ __global__ void __launch_bounds__(kFmaThreads) router_logits_fma_kernel(const __
                                                                         const float* __restrict__ w, int T,
                                                                         int H, int E,
                                                                         float* __restrict__ logits) {
-  pdl_enter();
   __shared__ float xs[kFmaTok][kFmaHc];
   const int t0 = blockIdx.x * kFmaTok;
   const int nch = (H + kFmaHc - 1) / kFmaHc;
@@ -202,7 +200,6 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
                                                              size_t split_stride, const float* __restrict__ bias,
                                                              int T, int E, int k, int32_t* __restrict__ ids,
                                                              float* __restrict__ wout, DevStatus* st) {
-  pdl_enter();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kTopkWarps + warp;
   if (t >= T) return;
@@ -236,8 +233,8 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
 template <int EPL, int UNR, bool QUAD = false>
 cudaError_t launch_topk_t(const float* logits, int nsplit, size_t split_stride, const float* bias, int T, int E,
                           int k, int32_t* ids, float* w, DevStatus* st, cudaStream_t s) {
-  return launch_pdl(topk_kernel<EPL, UNR, QUAD>, dim3((T + kTopkWarps - 1) / kTopkWarps), dim3(kTopkWarps * 32), 0, s,
-                    logits, nsplit, split_stride, bias, T, E, k, ids, w, st);
+  return launch_kernel(topk_kernel<EPL, UNR, QUAD>, dim3((T + kTopkWarps - 1) / kTopkWarps), dim3(kTopkWarps * 32),
+                       0, s, logits, nsplit, split_stride, bias, T, E, k, ids, w, st);
 }
 
 
@@ -287,7 +284,6 @@ __global__ void __launch_bounds__(kSmallThreads) router_small_kernel(
   __shared__ int32_t cnt[kMaxExperts];
   __shared__ int32_t warp_sums[kSmallThreads / 32];
   __shared__ int is_last;
-  pdl_enter();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cs = blockIdx.x, hy = blockIdx.y;
   const int h0 = hy * chunk, h1 = min(H, h0 + chunk);
@@ -438,9 +434,9 @@ cudaError_t launch_router_small_t(const uint16_t* x, const float* w, const float
                                   int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
                                   DevStatus* st, cudaStream_t s) {
   const SmallGrid g = small_grid(H, E);
-  return launch_pdl(router_small_kernel<TT, EPL>, dim3(g.ncs, g.hs), dim3(kSmallThreads), 0, s,
-                    reinterpret_cast<const __nv_bfloat16*>(x), w, bias, T, H, E, k, g.chunk, g.hs, partial, arrivals,
-                    ids, wout, counts, offsets, sorted_ids, inv_perm, st);
+  return launch_kernel(router_small_kernel<TT, EPL>, dim3(g.ncs, g.hs), dim3(kSmallThreads), 0, s,
+                       reinterpret_cast<const __nv_bfloat16*>(x), w, bias, T, H, E, k, g.chunk, g.hs, partial,
+                       arrivals, ids, wout, counts, offsets, sorted_ids, inv_perm, st);
 }
 
 // accumulators for 1, 4 or 16 tokens
@@ -455,7 +451,7 @@ cudaError_t launch_router_small_e(int T, A... args) {
 
 cudaError_t launch_router_split(const float* w, int H, int E, uint16_t* planes, cudaStream_t s) {
   const int n = H * E;
-  return launch_pdl(router_split_kernel, dim3(min(4096, (n + 255) / 256)), dim3(256), 0, s, w, n, planes);
+  return launch_kernel(router_split_kernel, dim3(min(4096, (n + 255) / 256)), dim3(256), 0, s, w, n, planes);
 }
 
 int fma_router_splits(int T, int H) {
@@ -470,8 +466,8 @@ int fma_router_splits(int T, int H) {
 cudaError_t launch_router_logits_fma(const uint16_t* x, const float* w, int T, int H, int E, float* logits,
                                      cudaStream_t s) {
   const dim3 grid((T + kFmaTok - 1) / kFmaTok, fma_router_splits(T, H));
-  return launch_pdl(router_logits_fma_kernel, grid, dim3(kFmaThreads), 0, s, reinterpret_cast<const __nv_bfloat16*>(x),
-                    w, T, H, E, logits);
+  return launch_kernel(router_logits_fma_kernel, grid, dim3(kFmaThreads), 0, s,
+                       reinterpret_cast<const __nv_bfloat16*>(x), w, T, H, E, logits);
 }
 
 cudaError_t launch_topk(const float* logits, int nsplit, size_t split_stride, const float* bias, int T, int E, int k,
