@@ -283,31 +283,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                 out[(size_t)(un.row0 + c0 + j) * a.ld_out + col] = __float2bfloat16_rn(silu_f(g[j]) * v[j]);
             }
           }
-        } else if (EPI == EPI_STORE_F32) {
-          float* out = reinterpret_cast<float*>(a.out) + (size_t)un.ks * a.split_stride;
-#pragma unroll
-          for (int t = 0; t < MT; ++t) {
-            float v[32];
-            tmem_ld_2x16(tbase + t * NT + c0, tbase + t * NT + c0 + 16, v, v + 16);
-            const int ct = col + t * a.out_col1_off;
-            if (ct < a.n_valid) {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                if (j < nr) out[(size_t)(un.row0 + c0 + j) * a.ld_out + ct] = v[j];
-              }
-            }
-          }
         } else {
-          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+          // both tiles' 32 rows in one batch of TMEM loads (one wait), then the stores
+          float v[MT][32];
+          if constexpr (MT == 2) {
+            tmem_ld_4x16(tbase + c0, tbase + c0 + 16, tbase + NT + c0, tbase + NT + c0 + 16, v[0], v[0] + 16, v[1],
+                         v[1] + 16);
+          } else {
+            tmem_ld_2x16(tbase + c0, tbase + c0 + 16, v[0], v[0] + 16);
+          }
 #pragma unroll
           for (int t = 0; t < MT; ++t) {
-            float v[32];
-            tmem_ld_2x16(tbase + t * NT + c0, tbase + t * NT + c0 + 16, v, v + 16);
             const int ct = col + t * a.out_col1_off;
             if (ct < a.n_valid) {
+              if (EPI == EPI_STORE_F32) {
+                float* out = reinterpret_cast<float*>(a.out) + (size_t)un.ks * a.split_stride;
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                if (j < nr) out[(size_t)(un.row0 + c0 + j) * a.ld_out + ct] = __float2bfloat16_rn(v[j]);
+                for (int j = 0; j < 32; ++j)
+                  if (j < nr) out[(size_t)(un.row0 + c0 + j) * a.ld_out + ct] = v[t][j];
+              } else {
+                __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (j < nr) out[(size_t)(un.row0 + c0 + j) * a.ld_out + ct] = __float2bfloat16_rn(v[t][j]);
               }
             }
           }
