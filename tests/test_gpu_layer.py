@@ -30,6 +30,7 @@ CASES = {
         Config("decode_split", T=1, H=1024, E=64, I=512, k=8),      # gate/up 4 K slices, down 2
         Config("few_e20", T=12, H=512, E=20, I=256, k=5),           # E % 8 != 0: ragged column slice
         Config("three_shared", T=3, H=768, E=32, I=128, k=4, I_s=128),
+        Config("few_bias", T=7, H=1024, E=128, I=256, k=6, bias="zipf:1.2"),  # biased few-token routing
     ]
 }
 
@@ -194,7 +195,7 @@ def test_few_token_router_repeated_calls():
     launch: back-to-back calls (also through the whole layer) stay correct
     and leave the workspace's status block all zero."""
     import torch
-    for name in ("decode_split", "few_e20", "three_shared"):
+    for name in ("decode_split", "few_e20", "three_shared", "few_bias"):
         cfg, inp, ref = case(name)
         d = dev_inputs(inp)
         ws = workspace(cfg)
