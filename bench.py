@@ -450,13 +450,13 @@ def run_ours(args):
         pres_e = time_workload(pcfg, d2, ws2, args.steps, args.warmup, rank, world, flush, moe, gpu_index,
                                sample_clocks=False, tiles=tiles)
         pres = time_workload(pcfg, d2, ws2, args.steps, args.warmup, rank, world, flush, moe, gpu_index,
-                             sample_clocks=False, tiles=tiles, graph=True)
+                             tiles=tiles, graph=True)
         pcounts = moe.workspace_view(ws2, pcfg.T, pcfg.H, pcfg.E, pcfg.I, pcfg.k)["counts"].cpu().numpy()
         pacc = layer_accounting(pcfg, pcounts)
         pe2e = time_e2e(pcfg, d2, ws2, max(3, args.steps // 2), args.warmup, rank, world, moe, tiles=tiles)
         prefill = {"workload": pcfg.name, "value": round(pres["value"], 1), "unit": "tokens/s",
                    "ms_per_step": round(pres["ms_per_step"], 4), "gpu_launches": pres["launches"],
-                   "eager": eager_of(pres_e),
+                   "eager": eager_of(pres_e), "clocks": pres["clocks"],
                    "e2e": {k: (round(v, 1) if isinstance(v, float) else v) for k, v in pe2e.items()},
                    **roof(pcfg, pres_e, pacc, pres["ms_per_step"])}
         del ws2
