@@ -102,7 +102,7 @@ int moe_abi_version(void);
  * after moe_forward; all 256-byte aligned).  Regions:
  *   topk_ids [T,k] i32, topk_w [T,k] f32, counts [E] i32, offsets [E+1] i32,
  *   sorted_token_ids [T*k] i32, inv_perm [T,k] i32, h [T*k, I] bf16,
- *   o [T*k, H] bf16 (expert outputs, permuted order), h_shared [T, I_s] bf16,
+ *   o [T*k, H] f32 (expert outputs, permuted order), h_shared [T, I_s] bf16,
  *   o_shared [T, H] f32,
  *   logits [S, T, E] f32 (S router partial slabs), router_split [3, H, E]
  *   bf16, block_hist (permute), split: K-split partial slabs of the expert
@@ -195,9 +195,8 @@ moe_status_t moe_grouped_down(const uint16_t *h, const uint16_t *w_down, const i
 /* Down GEMM + weighted combine: y [T,H] bf16 from h [T*k, I] bf16 (permuted
  * order), W_down [E, I, H] bf16, topk_w [T,k] f32, inv_perm [T,k] i32,
  * offsets [E+1] i32 and an optional shared-expert output shared_out [T,H]
- * f32 (NULL for none), added after the k routed terms.  Each expert output
- * row is accumulated in fp32 and stored as bf16 (the layer's activation
- * type); the k terms of a token are summed in slot order j = 0..k-1 in
+ * f32 (NULL for none), added after the k routed terms.  Expert output rows
+ * stay fp32; the k terms of a token are summed in slot order j = 0..k-1 in
  * fp32, so y is bitwise reproducible. */
 moe_status_t moe_down_combine(const uint16_t *h, const uint16_t *w_down,
                               const float *topk_w, const int32_t *inv_perm,

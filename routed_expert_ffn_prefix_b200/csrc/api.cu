@@ -93,7 +93,7 @@ moe_workspace_layout_t make_layout(int T, int H, int E, int I, int k, int I_s) {
   L.logits = take((size_t)(H > 0 ? router_slabs(T, H, E) : 1) * T * E * 4);
   L.router_split = take((size_t)3 * H * E * 2);
   L.h = take(tk * I * 2);
-  L.o = take(tk * H * 2);
+  L.o = take(tk * H * 4);
   L.h_shared = take((size_t)T * I_s * 2);
   L.o_shared = take(I_s > 0 ? (size_t)T * H * 4 : 0);
   // Sized for SMALL tiles, the only policy that splits K.
@@ -344,10 +344,9 @@ moe_status_t run_swiglu(const uint16_t* x, int src_rows, const uint16_t* w_gate_
   return cuda_status(launch_grouped_gemm(map, a, EPI_SWIGLU, tiles, dev.num_sms, s));
 }
 
-// o: fp32 rows (epilogue EPI_STORE_F32; nsplit > 1: K-split into partial
-// slabs [nsplit][rows][H]) or bf16 rows (EPI_STORE_BF16, nsplit == 1).
+// o: fp32 rows; nsplit > 1: K-split into partial slabs [nsplit][rows][H].
 moe_status_t run_down(const uint16_t* h, const uint16_t* w_down, const int32_t* offsets, int rows, int H, int E,
-                      int I, int tiles, void* o, int epilogue, DevStatus* st, const DeviceInfo& dev, cudaStream_t s,
+                      int I, int tiles, float* o, DevStatus* st, const DeviceInfo& dev, cudaStream_t s,
                       int nsplit = 1) {
   CUtensorMap map;
   if (!make_weight_map(&map, w_down, (uint64_t)H, (uint64_t)I, (uint64_t)E)) return MOE_ERR_CUDA;
@@ -381,9 +380,9 @@ moe_status_t run_down(const uint16_t* h, const uint16_t* w_down, const int32_t* 
     a.col1_off = 256;
     a.out_col_stride = 512;
     a.out_col1_off = 256;
-    return cuda_status(launch_grouped_gemm_pair(map, a, epilogue, dev.num_sms, s));
+    return cuda_status(launch_grouped_gemm_pair(map, a, EPI_STORE_F32, dev.num_sms, s));
   }
-  return cuda_status(launch_grouped_gemm(map, a, epilogue, tiles, dev.num_sms, s));
+  return cuda_status(launch_grouped_gemm(map, a, EPI_STORE_F32, tiles, dev.num_sms, s));
 }
 
 }  // namespace
@@ -503,8 +502,8 @@ moe_status_t moe_grouped_down(const uint16_t* h, const uint16_t* w_down, const i
   MOE_TRY(check_ws(workspace, workspace_bytes, sizeof(DevStatus)));
   DeviceInfo dev;
   MOE_TRY(check_device(&dev));
-  return run_down(h, w_down, offsets, rows, H, E, I, choose_tiles(tile_policy, rows, E), o, EPI_STORE_F32,
-                  status_of(workspace), dev, static_cast<cudaStream_t>(stream));
+  return run_down(h, w_down, offsets, rows, H, E, I, choose_tiles(tile_policy, rows, E), o, status_of(workspace),
+                  dev, static_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_down_combine(const uint16_t* h, const uint16_t* w_down, const float* topk_w,
@@ -522,11 +521,10 @@ moe_status_t moe_down_combine(const uint16_t* h, const uint16_t* w_down, const f
   MOE_TRY(check_device(&dev));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int rows = T * k;
-  uint16_t* o = at<uint16_t>(workspace, L.o);
+  float* o = at<float>(workspace, L.o);
   DevStatus* st = status_of(workspace);
-  MOE_TRY(run_down(h, w_down, offsets, rows, H, E, I, choose_tiles(tile_policy, rows, E), o, EPI_STORE_BF16, st, dev,
-                   s));
-  return cuda_status(launch_combine_bf16(o, topk_w, inv_perm, shared_out, T, H, k, rows, y, st, s));
+  MOE_TRY(run_down(h, w_down, offsets, rows, H, E, I, choose_tiles(tile_policy, rows, E), o, st, dev, s));
+  return cuda_status(launch_combine(o, topk_w, inv_perm, shared_out, T, H, k, rows, 1, 0, y, st, s));
 }
 
 moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const float* bias, const uint16_t* w_gate_up,
@@ -560,7 +558,7 @@ moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const floa
   int32_t* sids = at<int32_t>(ws, L.sorted_token_ids);
   int32_t* inv = at<int32_t>(ws, L.inv_perm);
   uint16_t* h = at<uint16_t>(ws, L.h);
-  uint16_t* o = at<uint16_t>(ws, L.o);
+  float* o = at<float>(ws, L.o);
   const int rows = T * k;
 
   void* const* ev = options ? options->stage_events : nullptr;
@@ -594,22 +592,17 @@ moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const floa
     o_sh = at<float>(ws, L.o_shared);
     const int sh_tiles = choose_tiles(tile_policy, T, 1);
     MOE_TRY(run_swiglu(x, T, w_sh_gate_up, nullptr, nullptr, T, H, 1, I_s, sh_tiles, h_sh, st, dev, s));
-    MOE_TRY(run_down(h_sh, w_sh_down, nullptr, T, H, 1, I_s, sh_tiles, o_sh, EPI_STORE_F32, st, dev, s));
+    MOE_TRY(run_down(h_sh, w_sh_down, nullptr, T, H, 1, I_s, sh_tiles, o_sh, st, dev, s));
     launches += 2;
   }
   MOE_TRY(mark(3));
   MOE_TRY(run_swiglu(x, T, w_gate_up, offs, sids, rows, H, E, I, tiles, h, st, dev, s, sp.gate_up, split));
   launches += sp.gate_up > 1 ? 2 : 1;
   MOE_TRY(mark(4));
-  if (sp.down > 1) {
-    MOE_TRY(run_down(h, w_down, offs, rows, H, E, I, tiles, split, EPI_STORE_F32, st, dev, s, sp.down));
-    MOE_TRY(mark(5));
-    MOE_TRY(cuda_status(launch_combine(split, tw, inv, o_sh, T, H, k, rows, sp.down, (size_t)rows * H, y, st, s)));
-  } else {
-    MOE_TRY(run_down(h, w_down, offs, rows, H, E, I, tiles, o, EPI_STORE_BF16, st, dev, s));
-    MOE_TRY(mark(5));
-    MOE_TRY(cuda_status(launch_combine_bf16(o, tw, inv, o_sh, T, H, k, rows, y, st, s)));
-  }
+  float* od = sp.down > 1 ? split : o;
+  MOE_TRY(run_down(h, w_down, offs, rows, H, E, I, tiles, od, st, dev, s, sp.down));
+  MOE_TRY(mark(5));
+  MOE_TRY(cuda_status(launch_combine(od, tw, inv, o_sh, T, H, k, rows, sp.down, (size_t)rows * H, y, st, s)));
   launches += 2;  // down GEMM, combine
   MOE_TRY(mark(6));
   if (options) options->launches = launches;

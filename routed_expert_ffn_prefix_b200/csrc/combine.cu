@@ -3,16 +3,16 @@
 // The Qwen 3.5-397B-on-Ironwood page (sec. 7.2) un-permutes the [T*k, H]
 // expert outputs and gather-reduces them per token; the Ling-2.6-1T /
 // SGLang-JAX page fuses scatter, expert FFN and gather ("Fused MoE V2").
-// Here each token's k expert rows (bf16, or fp32 K-split partial slabs that
-// are first summed in slab order) are read through inv_perm and summed in
+// Here each token's k expert rows (fp32; K-split partial slabs are first
+// summed in slab order) are read through inv_perm and summed in
 // slot order j = 0..k-1 in fp32 (w_j * o_j, one fused multiply-add per
 // term), the shared-expert row (weight 1) is added last, and y is rounded
 // to bf16 once.  A fixed summation order makes y bitwise reproducible
 // run to run, whatever order the expert GEMM tiles finished in.
 //
 // Memory-bound: a block per (token, column slice), one 16-byte vector of a
-// row per thread and slot (8 bf16 or 4 fp32 columns), the k slot loads of a
-// thread issued together.
+// row (4 columns) per thread and slot, the k slot loads of a thread issued
+// together.
 #include "gemm_units.cuh"
 
 namespace moe {
@@ -21,8 +21,7 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// V consecutive columns of an expert output row in one 16-byte load, widened
-// to fp32: 4 fp32 columns or 8 bf16 columns.
+// V consecutive columns of an expert output row in one 16-byte load.
 template <typename OT>
 struct Vec;
 template <>
@@ -33,21 +32,6 @@ struct Vec<float> {
     v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
   }
 };
-template <>
-struct Vec<__nv_bfloat16> {
-  static constexpr int V = 8;
-  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[8]) {
-    const uint4 q = __ldcs(reinterpret_cast<const uint4*>(p));
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
-      v[2 * i] = f.x;
-      v[2 * i + 1] = f.y;
-    }
-  }
-};
-
 template <typename OT>
 __global__ void __launch_bounds__(kThreads) combine_kernel(const OT* __restrict__ o, const float* __restrict__ w,
                                                          const int32_t* __restrict__ inv_perm,
@@ -199,12 +183,6 @@ cudaError_t launch_combine(const float* o, const float* topk_w, const int32_t* i
                            int H, int k, int rows, int nsplit, size_t split_stride, uint16_t* y, DevStatus* st,
                            cudaStream_t s) {
   return launch_combine_t(o, topk_w, inv_perm, shared, T, H, k, rows, nsplit, split_stride, y, st, s);
-}
-
-cudaError_t launch_combine_bf16(const uint16_t* o, const float* topk_w, const int32_t* inv_perm, const float* shared,
-                                int T, int H, int k, int rows, uint16_t* y, DevStatus* st, cudaStream_t s) {
-  return launch_combine_t(reinterpret_cast<const __nv_bfloat16*>(o), topk_w, inv_perm, shared, T, H, k, rows, 1, 0, y,
-                          st, s);
 }
 
 }  // namespace moe

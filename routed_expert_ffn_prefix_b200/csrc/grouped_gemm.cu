@@ -296,17 +296,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int t = 0; t < MT; ++t) {
             const int ct = col + t * a.out_col1_off;
             if (ct < a.n_valid) {
-              if (EPI == EPI_STORE_F32) {
-                float* out = reinterpret_cast<float*>(a.out) + (size_t)un.ks * a.split_stride;
+              float* out = reinterpret_cast<float*>(a.out) + (size_t)un.ks * a.split_stride;
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                  if (j < nr) out[(size_t)(un.row0 + c0 + j) * a.ld_out + ct] = v[t][j];
-              } else {
-                __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                  if (j < nr) out[(size_t)(un.row0 + c0 + j) * a.ld_out + ct] = __float2bfloat16_rn(v[t][j]);
-              }
+              for (int j = 0; j < 32; ++j)
+                if (j < nr) out[(size_t)(un.row0 + c0 + j) * a.ld_out + ct] = v[t][j];
             }
           }
         }
@@ -348,19 +341,13 @@ int gemm_tiles_per_unit(int tiles, int epilogue) {
 cudaError_t launch_grouped_gemm(const CUtensorMap& wmap, const GemmArgs& a, int epilogue, int tiles, int num_sms,
                                 cudaStream_t stream) {
   if (tiles == MOE_TILES_LARGE) {
-    switch (epilogue) {
-      case EPI_SWIGLU: return launch_cfg<256, 3, 2, EPI_SWIGLU>(wmap, a, num_sms, stream);
-      case EPI_STORE_F32: return launch_cfg<256, 3, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
-      default: return launch_cfg<256, 3, 2, EPI_STORE_BF16>(wmap, a, num_sms, stream);
-    }
+    return epilogue == EPI_SWIGLU ? launch_cfg<256, 3, 2, EPI_SWIGLU>(wmap, a, num_sms, stream)
+                                  : launch_cfg<256, 3, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
   }
   // Small groups (decode): 128-row passes, 4 stages -- measured ~5% faster
   // than 64-row passes with 5 stages at 1-30 rows per expert.
-  switch (epilogue) {
-    case EPI_SWIGLU: return launch_cfg<128, 4, 2, EPI_SWIGLU>(wmap, a, num_sms, stream);
-    case EPI_STORE_F32: return launch_cfg<128, 4, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
-    default: return launch_cfg<128, 4, 2, EPI_STORE_BF16>(wmap, a, num_sms, stream);
-  }
+  return epilogue == EPI_SWIGLU ? launch_cfg<128, 4, 2, EPI_SWIGLU>(wmap, a, num_sms, stream)
+                                : launch_cfg<128, 4, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
 }
 
 }  // namespace moe

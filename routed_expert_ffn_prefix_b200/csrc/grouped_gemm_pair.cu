@@ -384,17 +384,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
           for (int t = 0; t < MT; ++t) {
             const int ct = col + t * a.out_col1_off;
             if (ct < a.n_valid) {
-              if (EPI == EPI_STORE_F32) {
-                float* out = reinterpret_cast<float*>(a.out) + (size_t)un.ks * a.split_stride;
+              float* out = reinterpret_cast<float*>(a.out) + (size_t)un.ks * a.split_stride;
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                  if (j < nr) out[(size_t)(un.row0 + c0 + j) * a.ld_out + ct] = v[t][j];
-              } else {
-                __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                  if (j < nr) out[(size_t)(un.row0 + c0 + j) * a.ld_out + ct] = __float2bfloat16_rn(v[t][j]);
-              }
+              for (int j = 0; j < 32; ++j)
+                if (j < nr) out[(size_t)(un.row0 + c0 + j) * a.ld_out + ct] = v[t][j];
             }
           }
         }
@@ -469,8 +462,7 @@ cudaError_t launch_grouped_gemm_pair(const CUtensorMap& wmap, const GemmArgs& a,
     // One 256-column tile per unit with a double-buffered accumulator: down
     // 1.03 / 2.35 ms.
     case EPI_SWIGLU: return launch_pair<256, 4, 2, EPI_SWIGLU>(wmap, a, num_sms, stream);
-    case EPI_STORE_F32: return launch_pair<256, 4, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
-    default: return launch_pair<256, 4, 2, EPI_STORE_BF16>(wmap, a, num_sms, stream);
+    default: return launch_pair<256, 4, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
   }
 }
 

@@ -68,9 +68,8 @@ struct GemmArgs {
   uint64_t timeout_ns;
 };
 
-// SWIGLU: h = bf16(silu(gate) * up); STORE_F32: fp32 rows (K splits to their own slabs);
-// STORE_BF16: rows rounded to bf16 (expert outputs read once by the combine).
-enum Epilogue { EPI_SWIGLU = 0, EPI_STORE_F32 = 1, EPI_STORE_BF16 = 2 };
+// SWIGLU: h = bf16(silu(gate) * up); STORE_F32: fp32 rows (K splits to their own slabs).
+enum Epilogue { EPI_SWIGLU = 0, EPI_STORE_F32 = 1 };
 
 // MMA tiles (128 weight columns each) per work unit of the given tile
 // policy and epilogue; the caller sets n_blocks/col_stride/out_col_stride
@@ -109,10 +108,6 @@ cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* cou
 cudaError_t launch_combine(const float* o, const float* topk_w, const int32_t* inv_perm, const float* shared,
                            int T, int H, int k, int rows, int nsplit, size_t split_stride, uint16_t* y, DevStatus* st,
                            cudaStream_t s);
-
-// Same from bf16 expert outputs o [rows, H] (one slab).
-cudaError_t launch_combine_bf16(const uint16_t* o, const float* topk_w, const int32_t* inv_perm, const float* shared,
-                                int T, int H, int k, int rows, uint16_t* y, DevStatus* st, cudaStream_t s);
 
 // h = bf16(silu(sum_s gate_s) * sum_s up_s) from K-split partial slabs [rows, 2I].
 cudaError_t launch_swiglu_reduce(const float* partials, int nsplit, size_t split_stride, int rows, int I, uint16_t* h,
