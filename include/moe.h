@@ -76,8 +76,13 @@ enum {
   MOE_TILES_AUTO = 0,   /* chosen from the mean rows per expert, T*k/E: SMALL up to 64, else PAIR */
   MOE_TILES_SMALL = 1,  /* <= 128 token rows per tile pass, 4-stage ring: decode */
   MOE_TILES_LARGE = 2,  /* <= 256 token rows per tile pass, 3-stage ring: prefill */
-  MOE_TILES_PAIR = 3    /* SM pairs (2-SM tcgen05 MMA): 256 weight columns per MMA, 128 per SM; <= 256
+  MOE_TILES_PAIR = 3,   /* SM pairs (2-SM tcgen05 MMA): 256 weight columns per MMA, 128 per SM; <= 256
                            token rows per pass, half gathered by each SM; 4-stage ring: prefill */
+  MOE_TILES_FUSED = 4   /* moe_forward_ex only, T <= 4: the whole layer (routing, permutation, both
+                           expert matrix-vector products, combine) in one cooperative launch with
+                           grid barriers; CUDA-core weight streams.  Needs k <= 16, E % 4 == 0,
+                           H, I, I_s multiples of 256, H <= 8192, I, I_s <= 4096.  Never chosen
+                           by AUTO (measured slower than SMALL with its K split). */
 };
 
 /* Router logits implementation. */
@@ -106,10 +111,11 @@ int moe_abi_version(void);
  *   o_shared [T, H] f32,
  *   logits [S, T, E] f32 (S router partial slabs), router_split [3, H, E]
  *   bf16, block_hist (permute), split: K-split partial slabs of the expert
- *   GEMMs when few tokens leave SMs idle (f32; 0 bytes when unused). */
+ *   GEMMs when few tokens leave SMs idle (f32; 0 bytes when unused), fused:
+ *   partial slabs of the one-launch layer for T <= 4 (f32; 0 bytes above). */
 typedef struct moe_workspace_layout {
   size_t status, topk_ids, topk_w, counts, offsets, sorted_token_ids, inv_perm;
-  size_t h, o, h_shared, o_shared, logits, router_split, block_hist, split;
+  size_t h, o, h_shared, o_shared, logits, router_split, block_hist, split, fused;
   size_t total;
 } moe_workspace_layout_t;
 
@@ -124,7 +130,9 @@ moe_status_t moe_workspace_size(int T, int H, int E, int I, int k, int I_s, size
 moe_status_t moe_get_device_status(const void *workspace, void *stream, int32_t *out);
 
 /* Resets the workspace status block (stream-ordered): the status word to
- * MOE_OK and the block counter the few-token router keeps beside it. */
+ * MOE_OK and the counters the few-token router and the one-launch layer keep
+ * beside it (each returns its counter to zero when it finishes; after a
+ * device timeout, clear the block before the next call). */
 moe_status_t moe_clear_device_status(void *workspace, void *stream);
 
 /* Route: topk_ids [T,k] i32 and topk_w [T,k] f32 from x [T,H] bf16,

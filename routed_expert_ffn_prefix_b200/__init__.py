@@ -17,14 +17,14 @@ from dataclasses import dataclass
 from . import build as _build
 
 __all__ = [
-    "MoEError", "lib", "TILES_AUTO", "TILES_SMALL", "TILES_LARGE", "TILES_PAIR",
+    "MoEError", "lib", "TILES_AUTO", "TILES_SMALL", "TILES_LARGE", "TILES_PAIR", "TILES_FUSED",
     "ROUTER_AUTO", "ROUTER_FMA", "ROUTER_TC", "ROUTER_SMALL",
     "workspace_size", "workspace_layout", "alloc_workspace", "route", "permute", "grouped_swiglu",
     "grouped_down", "down_combine", "forward", "device_status", "clear_device_status", "selftest_timeout",
     "STATUS",
 ]
 
-TILES_AUTO, TILES_SMALL, TILES_LARGE, TILES_PAIR = 0, 1, 2, 3
+TILES_AUTO, TILES_SMALL, TILES_LARGE, TILES_PAIR, TILES_FUSED = 0, 1, 2, 3, 4
 ROUTER_AUTO, ROUTER_FMA, ROUTER_TC, ROUTER_SMALL = 0, 1, 2, 3
 
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_ALIGNMENT", 3: "MOE_ERR_WORKSPACE",
@@ -41,7 +41,7 @@ class MoEError(RuntimeError):
 class _Layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "status", "topk_ids", "topk_w", "counts", "offsets", "sorted_token_ids", "inv_perm",
-        "h", "o", "h_shared", "o_shared", "logits", "router_split", "block_hist", "split", "total")]
+        "h", "o", "h_shared", "o_shared", "logits", "router_split", "block_hist", "split", "fused", "total")]
 
 
 class _Options(ctypes.Structure):

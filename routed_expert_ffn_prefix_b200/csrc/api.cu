@@ -101,6 +101,14 @@ moe_workspace_layout_t make_layout(int T, int H, int E, int I, int k, int I_s) {
   const size_t gu = sp.gate_up > 1 ? (size_t)sp.gate_up * tk * 2 * I : 0;
   const size_t dn = sp.down > 1 ? (size_t)sp.down * tk * H : 0;
   L.split = take((gu > dn ? gu : dn) * 4);
+  // slabs of the one-launch few-token layer
+  size_t fused = 0;
+  if (T <= kFusedMaxT && H > 0 && I > 0) {
+    const size_t frows = tk + (I_s > 0 ? (size_t)T : 0);
+    const size_t imax = (size_t)(I > I_s ? I : I_s);
+    fused = (size_t)kFusedMaxSplit * frows * (2 * imax + H) * 4;
+  }
+  L.fused = take(fused);
   L.total = off;
   return L;
 }
@@ -541,7 +549,7 @@ moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const floa
   }
   const int tile_policy = options ? options->tile_policy : MOE_TILES_AUTO;
   const int router_impl = options ? options->router_impl : MOE_ROUTER_AUTO;
-  if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_PAIR) return MOE_ERR_INVALID_ARG;
+  if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_FUSED) return MOE_ERR_INVALID_ARG;
   if (router_impl < MOE_ROUTER_AUTO || router_impl > MOE_ROUTER_SMALL) return MOE_ERR_INVALID_ARG;
   if (!all_aligned(x, w_router, w_gate_up, w_down, y) || (bias && !aligned16(bias))) return MOE_ERR_ALIGNMENT;
   const moe_workspace_layout_t L = make_layout(T, H, E, I, k, shared ? I_s : 0);
@@ -567,6 +575,25 @@ moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const floa
     return MOE_OK;
   };
   int launches = 0;
+
+  // A few tokens, on request: the whole layer in one cooperative launch.
+  if (tile_policy == MOE_TILES_FUSED) {
+    if (!fused_decode_supported(T, H, E, I, k, shared ? I_s : 0)) return MOE_ERR_INVALID_ARG;
+    float* slabs = at<float>(ws, L.fused);
+    const size_t frows = (size_t)rows + (shared ? (size_t)T : 0);
+    const int imax = I > I_s ? I : I_s;
+    float* gslabs = slabs;
+    float* dslabs = slabs + (size_t)kFusedMaxSplit * frows * 2 * imax;
+    MOE_TRY(mark(0));
+    MOE_TRY(cuda_status(launch_fused_decode(x, w_router, bias, w_gate_up, w_down, shared ? w_sh_gate_up : nullptr,
+                                            shared ? w_sh_down : nullptr, shared ? I_s : 0, T, H, E, I, k,
+                                            at<float>(ws, L.logits), gslabs, dslabs, ids, tw, counts, offs, sids, inv,
+                                            y, st, kDefaultTimeoutNs, dev.num_sms, s)));
+    for (int i = 1; i < 7; ++i) MOE_TRY(mark(i));
+    if (options) options->launches = 1;
+    return MOE_OK;
+  }
+
   const int ri = resolve_router(router_impl, T, E);
   MOE_TRY(mark(0));
   if (ri == MOE_ROUTER_SMALL) {

@@ -20,6 +20,8 @@ struct DevStatus {
   int32_t site;
   int32_t aux;
   uint32_t arrivals;  // block counter of the few-token router: zero between its launches
+  uint32_t grid_bar;  // grid-barrier counter of the one-launch few-token layer: zero between launches
+  uint32_t reserved[3];
 };
 
 // Where an error was raised (DevStatus::site).
@@ -34,6 +36,7 @@ enum Site : int32_t {
   SITE_COMBINE = 7,
   SITE_SELFTEST = 8,
   SITE_TOPK = 9,
+  SITE_FUSED = 10,
 };
 
 __device__ __forceinline__ void raise_error(DevStatus* st, int code, int site, int aux) {

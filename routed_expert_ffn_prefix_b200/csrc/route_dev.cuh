@@ -1,0 +1,214 @@
+// route_dev.cuh -- device pieces of the router shared by the router kernels
+// (route.cu) and the one-launch few-token layer (fused_decode.cu): the warp
+// top-k and the split-H partial logits of a few tokens.
+#pragma once
+
+#include "kernels.h"
+
+namespace moe {
+
+// Top-k of one token by one warp: lane L holds the logits of experts
+// L + 32 i in v (entries >= E ignored).  k rounds of a warp arg-max (larger
+// logit first, ties to the lower expert id; NaN logits are never chosen),
+// then w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0) over the k selected
+// logits.  Each round takes the lane's best by a pairwise tree over its EPL
+// entries (log2 EPL dependent steps) and the warp's best by 5 shuffles.
+// sel, if given, receives the k ids too (shared memory of the caller).
+constexpr int kNoExpert = 0x7fffffff;
+
+__device__ __forceinline__ bool topk_better(float av, int ai, float bv, int bi) {
+  return av > bv || (av == bv && ai < bi);
+}
+
+// Expert held in entry i of a lane's EPL logits: scalar layout e = lane + 32 i;
+// quad layout (16-byte loads, E % 4 == 0) e = 128 (i / 4) + 4 lane + i % 4.
+template <bool QUAD>
+__device__ __forceinline__ int entry_expert(int lane, int i) {
+  return QUAD ? 128 * (i >> 2) + 4 * lane + (i & 3) : lane + 32 * i;
+}
+
+template <int EPL, bool QUAD = false>
+__device__ __forceinline__ void warp_topk(const float (&vin)[EPL], int E, int k, int t, int32_t* idrow, float* wrow,
+                                          int32_t* sel, DevStatus* st) {
+  const int lane = threadIdx.x & 31;
+  float v[EPL];
+  int id[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = entry_expert<QUAD>(lane, i);
+    const bool ok = e < E && !isnan(vin[i]);
+    v[i] = ok ? vin[i] : -INFINITY;
+    id[i] = ok ? e : kNoExpert;
+  }
+  float lead = 0.f, sum = 0.f;
+  for (int j = 0; j < k; ++j) {
+    float tv[EPL];
+    int ti[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) { tv[i] = v[i]; ti[i] = id[i]; }
+#pragma unroll
+    for (int w = 1; w < EPL; w <<= 1)
+#pragma unroll
+      for (int i = 0; i + w < EPL; i += 2 * w)
+        if (topk_better(tv[i + w], ti[i + w], tv[i], ti[i])) { tv[i] = tv[i + w]; ti[i] = ti[i + w]; }
+    float bv = tv[0];
+    int bi = ti[0];
+#pragma unroll
+    for (int d = 16; d >= 1; d >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, d);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, d);
+      if (topk_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+    }
+    if (bi == kNoExpert) {  // no candidate left: the logits were NaN
+      if (lane == 0) raise_error(st, MOE_ERR_DEVICE_BOUNDS, SITE_TOPK, t);
+      bi = 0;
+      bv = lead;
+    }
+#pragma unroll
+    for (int i = 0; i < EPL; ++i)
+      if (id[i] == bi) { v[i] = -INFINITY; id[i] = kNoExpert; }
+    if (j == 0) lead = bv;
+    const float z = expf(bv - lead);
+    sum += z;
+    if (lane == 0) {
+      idrow[j] = bi;
+      wrow[j] = z;
+      if (sel) sel[j] = bi;
+    }
+  }
+  __syncwarp();
+  const float inv = 1.0f / sum;
+  for (int j = lane; j < k; j += 32) wrow[j] = wrow[j] * inv;
+}
+
+// ---------------------------------------------------------------- few tokens
+// For T <= kSmallRouterT the logits are a matrix-vector product whose cost is
+// reading W_router (H x E fp32) once, so the work is spread over ~148 blocks:
+// block item (cs, hy) owns W columns [8 cs, 8 cs + 8) (one 32-byte sector per
+// row) and rows [hy * chunk, (hy + 1) * chunk).  Each thread streams its rows
+// as float4s (all issued before any is used), multiplies them by the bf16 x
+// staged in shared memory and the block reduces over its rows in a fixed
+// order into partial slab hy.
+constexpr int kSmallThreads = 256;
+constexpr int kSmallCols = 8;
+constexpr int kSmallPass = 128;  // rows per block pass: 8 warps x 16
+constexpr int kSmallIters = 8;   // passes per block: chunk <= 1024 rows
+constexpr int kSmallMaxSlots = kSmallRouterT * 64;
+
+struct SmallGrid {
+  int ncs, hs, chunk;
+};
+
+inline SmallGrid small_grid(int H, int E) {
+  SmallGrid g;
+  g.ncs = (E + kSmallCols - 1) / kSmallCols;
+  int hs = 148 / g.ncs;
+  const int hs_min = (H + kSmallPass * kSmallIters - 1) / (kSmallPass * kSmallIters);
+  if (hs < hs_min) hs = hs_min;
+  if (hs < 1) hs = 1;
+  g.chunk = (((H + hs - 1) / hs) + 15) & ~15;
+  g.hs = (H + g.chunk - 1) / g.chunk;
+  return g;
+}
+
+// Shared memory of one partial-logits item (TT tokens).
+template <int TT>
+struct RouterSmem {
+  __nv_bfloat16 xs[TT][kSmallPass * kSmallIters];
+  float red[kSmallThreads / 32][TT][kSmallCols];
+};
+
+// Partial logits of item (cs, hy) for T <= TT tokens into slab hy of
+// partial [hs][T][E].  Called by all kSmallThreads threads of a block;
+// ends with the partial written (no fence).
+template <int TT>
+__device__ __forceinline__ void router_partial(const __nv_bfloat16* __restrict__ x, const float* __restrict__ w,
+                                               int T, int H, int E, int chunk, int cs, int hy,
+                                               float* __restrict__ partial, RouterSmem<TT>& sm) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h0 = hy * chunk, h1 = min(H, h0 + chunk);
+  const int q = lane & 1, r = lane >> 1;
+  const int c0 = cs * kSmallCols + q * 4;
+  const bool cval = c0 < E;  // E % 4 == 0: a quad is all in or all out
+
+  float4 wr[kSmallIters];
+#pragma unroll
+  for (int i = 0; i < kSmallIters; ++i) {
+    const int h = h0 + warp * 16 + r + kSmallPass * i;
+    wr[i] = (cval && h < h1) ? __ldcs(reinterpret_cast<const float4*>(w + (size_t)h * E + c0))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  // x rows [h0, h1) of every token, zero beyond T and h1
+  constexpr int kVec = kSmallPass * kSmallIters / 8;  // 16-byte vectors per staged row
+  for (int i = tid; i < TT * kVec; i += kSmallThreads) {
+    const int t = i / kVec, v = i - t * kVec, h = h0 + v * 8;
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (t < T && h < h1) val = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H + h));
+    reinterpret_cast<uint4*>(&sm.xs[t][0])[v] = val;
+  }
+  __syncthreads();
+  float acc[TT][4];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+#pragma unroll
+  for (int i = 0; i < kSmallIters; ++i) {
+    const int hl = warp * 16 + r + kSmallPass * i;
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+      const float xv = __bfloat162float(sm.xs[t][hl]);
+      acc[t][0] = fmaf(xv, wr[i].x, acc[t][0]);
+      acc[t][1] = fmaf(xv, wr[i].y, acc[t][1]);
+      acc[t][2] = fmaf(xv, wr[i].z, acc[t][2]);
+      acc[t][3] = fmaf(xv, wr[i].w, acc[t][3]);
+    }
+  }
+  // rows of a warp (lane bits 1..4), then the 8 warps in order
+#pragma unroll
+  for (int d = 2; d < 32; d <<= 1)
+#pragma unroll
+    for (int t = 0; t < TT; ++t)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[t][j] += __shfl_xor_sync(0xffffffffu, acc[t][j], d);
+  if (r == 0) {
+#pragma unroll
+    for (int t = 0; t < TT; ++t)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sm.red[warp][t][q * 4 + j] = acc[t][j];
+  }
+  __syncthreads();
+  if (tid < TT * kSmallCols) {
+    const int t = tid / kSmallCols, c = tid - t * kSmallCols;
+    float sum = 0.f;
+#pragma unroll
+    for (int v = 0; v < kSmallThreads / 32; ++v) sum += sm.red[v][t][c];
+    const int e = cs * kSmallCols + c;
+    if (t < T && e < E) partial[((size_t)hy * T + t) * E + e] = sum;
+  }
+}
+
+// Slab sum (slab order), bias, top-k of token t by the calling warp.
+template <int EPL>
+__device__ __forceinline__ void router_select(const float* partial, int hs, const float* __restrict__ bias, int T,
+                                              int E, int k, int t, int32_t* idrow, float* wrow, int32_t* sel,
+                                              DevStatus* st) {
+  const int lane = threadIdx.x & 31;
+  float v[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) v[i] = 0.f;
+  for (int sp = 0; sp < hs; ++sp) {
+    const float* slab = partial + ((size_t)sp * T + t) * E;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E) v[i] += __ldcg(slab + e);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = e < E ? v[i] + (bias ? bias[e] : 0.f) : -INFINITY;
+  }
+  warp_topk<EPL>(v, E, k, t, idrow, wrow, sel, st);
+}
+
+}  // namespace moe

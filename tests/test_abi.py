@@ -48,15 +48,15 @@ def test_workspace_layout_is_ordered_and_aligned(lib):
     L = moe.workspace_layout(8192, 4096, 512, 1024, 10)
     offs = [L[n] for n in ("status", "topk_ids", "topk_w", "counts", "offsets", "sorted_token_ids",
                            "inv_perm", "block_hist", "logits", "router_split", "h", "o", "h_shared",
-                           "o_shared", "split", "total")]
+                           "o_shared", "split", "fused", "total")]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
     assert L["o"] - L["h"] >= 81920 * 1024 * 2          # h: [T*k, I] bf16
     assert L["h_shared"] - L["o"] >= 81920 * 4096 * 4   # o: [T*k, H] f32
     assert moe.workspace_size(8192, 4096, 512, 1024, 10) == L["total"]
     Ls = moe.workspace_layout(4096, 8192, 256, 2048, 8, 2048)
     assert Ls["split"] - Ls["o_shared"] >= 4096 * 8192 * 4
-    # many tokens: no K split, so no partial slabs
-    assert L["total"] == L["split"] and Ls["total"] == Ls["split"]
+    # many tokens: no K split and no one-launch layer, so no partial slabs
+    assert L["total"] == L["fused"] == L["split"] and Ls["total"] == Ls["fused"] == Ls["split"]
 
 
 def test_workspace_layout_reserves_k_split_slabs_for_one_token(lib):
@@ -64,7 +64,9 @@ def test_workspace_layout_reserves_k_split_slabs_for_one_token(lib):
     96 gate/up units (-> 3 K slices) and 128 down units (-> 2 slices) for
     148 SMs.  The split region holds the larger: 3 x 8 rows x 3072 f32."""
     L = moe.workspace_layout(1, 4096, 256, 1536, 8)
-    assert L["total"] - L["split"] == max(3 * 8 * 3072, 2 * 8 * 4096) * 4
+    assert L["fused"] - L["split"] == max(3 * 8 * 3072, 2 * 8 * 4096) * 4
+    # the one-launch layer (T <= 4): 8 K slices of gate/up (2 x I) and down (H) rows, f32
+    assert L["total"] - L["fused"] == 8 * 8 * (2 * 1536 + 4096) * 4
     # the router's partial slabs: one per H slice of the few-token router
     assert L["router_split"] - L["logits"] >= 4 * 1 * 256 * 4
 
