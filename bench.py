@@ -229,7 +229,7 @@ def recorded_traffic(workload):
 
 
 # ---------------------------------------------------------------- timed runs
-TILES = {"auto": 0, "small": 1, "large": 2, "pair": 3}
+TILES = {"auto": 0, "small": 1, "large": 2, "pair": 3, "fused": 4}
 
 
 def time_workload(cfg, d, ws, steps, warmup, rank, world, flush, moe, gpu_index, sample_clocks=True, tiles=0,
