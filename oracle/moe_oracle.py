@@ -32,6 +32,23 @@ What it computes (plain definitions, in the order the layer applies them):
    weight 1 when the layer has one -- "top-8 routing plus a shared expert",
    Ling page, introduction).
 
+Router scoring variants (steps 1-3 replaced; everything after is unchanged).
+The Qwen-3.5-397B-on-Ironwood page ("key optimisations", step 1, expert load
+balancing) names hot experts and a balancing term in the router but gives no
+formula, and the Ling page says only that router logits get a per-expert
+bias.  Besides the rule above (bias added to the logits, so it moves both
+selection and weights: scoring "softmax"), two plain forms in which a
+per-expert bias b steers only which experts are picked are supported:
+
+- "softmax_select_bias": the k experts with the largest l + b (descending,
+  ties to the lower id) are selected; their weights are the softmax of the
+  unbiased logits over the selected set, w_j = exp(l_j) / sum_i exp(l_i).
+- "sigmoid": s = sigmoid(l) per expert; the k experts with the largest
+  s + b are selected (same order rule); w_j = s_j / sum_i s_i over them.
+
+Without a bias both select exactly what "softmax" selects (sigmoid and
+exp are monotone); the weights differ for "sigmoid".
+
 Nothing is rounded to bf16 inside the oracle; y stays float64.
 """
 from __future__ import annotations
@@ -41,8 +58,11 @@ import numpy as np
 __all__ = [
     "bf16_to_f64", "router_logits", "topk_route", "permute", "silu", "swiglu_ffn_rows",
     "expert_down_rows", "dense_swiglu_ffn", "layer_forward", "layer_forward_tokens",
-    "h_rows", "down_combine", "TEST_INFRASTRUCTURE_ONLY",
+    "h_rows", "down_combine", "SCORINGS", "selection_keys", "route_scored",
+    "TEST_INFRASTRUCTURE_ONLY",
 ]
+
+SCORINGS = ("softmax", "softmax_select_bias", "sigmoid")
 
 TEST_INFRASTRUCTURE_ONLY = True
 
@@ -82,6 +102,52 @@ def topk_route(logits: np.ndarray, k: int) -> tuple[np.ndarray, np.ndarray]:
         sel = order[:k]
         ids[t] = sel
         z = np.exp(logits[t, sel] - logits[t, sel[0]])
+        w[t] = z / z.sum()
+    return ids, w
+
+
+def _sigmoid(z: np.ndarray) -> np.ndarray:
+    """1 / (1 + exp(-z)), evaluated without overflow for either sign."""
+    z = np.asarray(z, np.float64)
+    e = np.exp(-np.abs(z))
+    return np.where(z >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+def selection_keys(l_raw: np.ndarray, bias, scoring: str) -> np.ndarray:
+    """The per-expert value whose k largest decide the selection, from the
+    unbiased logits l_raw [T,E]: l + b ("softmax", "softmax_select_bias") or
+    sigmoid(l) + b ("sigmoid")."""
+    if scoring not in SCORINGS:
+        raise ValueError(f"unknown scoring {scoring!r}")
+    l = np.asarray(l_raw, np.float64)
+    base = _sigmoid(l) if scoring == "sigmoid" else l
+    if bias is None:
+        return base
+    return base + np.asarray(bias, np.float64)[None, :]
+
+
+def route_scored(l_raw: np.ndarray, bias, k: int, scoring: str = "softmax"
+                 ) -> tuple[np.ndarray, np.ndarray]:
+    """Steps 2-3 under a scoring rule (module docstring): ids [T,k] int32 in
+    descending key order (ties to the lower id) and weights [T,k] float64 in
+    the same slot order."""
+    keys = selection_keys(l_raw, bias, scoring)
+    if scoring == "softmax":
+        return topk_route(keys, k)
+    T, E = keys.shape
+    if not 1 <= k <= E:
+        raise ValueError("need 1 <= k <= E")
+    l = np.asarray(l_raw, np.float64)
+    ids = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    expert = np.arange(E)
+    for t in range(T):
+        sel = np.lexsort((expert, -keys[t]))[:k]
+        ids[t] = sel
+        if scoring == "softmax_select_bias":
+            z = np.exp(l[t, sel] - l[t, sel].max())
+        else:
+            z = _sigmoid(l[t, sel])
         w[t] = z / z.sum()
     return ids, w
 
@@ -174,13 +240,14 @@ def down_combine(h, offsets, inv_perm, topk_w, expert_down, shared=None) -> np.n
 
 
 def layer_forward(x_bits, w_router, bias, w_gate_up, w_down, k,
-                  w_sh_gate_up=None, w_sh_down=None) -> dict:
+                  w_sh_gate_up=None, w_sh_down=None, scoring: str = "softmax") -> dict:
     """The whole layer for all tokens.  Returns y (float64 [T,H]) and every
-    intermediate: logits, ids, w, counts, offsets, sorted_token_ids, inv_perm,
-    h (float64, permuted order)."""
+    intermediate: logits (the selection keys), ids, w, counts, offsets,
+    sorted_token_ids, inv_perm, h (float64, permuted order)."""
     E = w_router.shape[1]
-    logits = router_logits(x_bits, w_router, bias)
-    ids, w = topk_route(logits, k)
+    l_raw = router_logits(x_bits, w_router, None)
+    logits = selection_keys(l_raw, bias, scoring)
+    ids, w = route_scored(l_raw, bias, k, scoring)
     counts, offsets, sorted_ids, inv_perm = permute(ids, E)
     h = h_rows(x_bits, sorted_ids, offsets, lambda e: w_gate_up[e])
     shared = None

@@ -111,6 +111,133 @@ def test_router_logits_bias_and_orientation():
     np.testing.assert_array_equal(l, W.astype(np.float64) + b)
 
 
+# ---------------------------------------------------------------- scoring variants
+
+def test_scored_routing_without_bias_selects_like_softmax():
+    """exp and sigmoid are monotone: with no bias every scoring picks the
+    same experts in the same order, and select-only-bias weights are the
+    plain softmax ones."""
+    rng = np.random.default_rng(21)
+    l = rng.standard_normal((40, 12)) * 2
+    ids0, w0 = om.topk_route(l, 4)
+    for scoring in om.SCORINGS:
+        ids, w = om.route_scored(l, None, 4, scoring)
+        np.testing.assert_array_equal(ids, ids0)
+        np.testing.assert_allclose(w.sum(1), 1.0, rtol=0, atol=1e-15)
+    _, w1 = om.route_scored(l, None, 4, "softmax_select_bias")
+    np.testing.assert_allclose(w1, w0, rtol=1e-14)
+
+
+def test_select_bias_picks_best_biased_subset_and_weights_ignore_bias():
+    """Selection: the k-subset with the largest sum of l + b, by descending
+    l + b.  Weights: scipy's softmax over the selected unbiased logits."""
+    rng = np.random.default_rng(22)
+    for E, k in [(6, 2), (7, 3), (5, 5)]:
+        l = rng.standard_normal((25, E))
+        b = rng.standard_normal(E) * 1.5
+        ids, w = om.route_scored(l, b, k, "softmax_select_bias")
+        for t in range(25):
+            key = [l[t, i] + b[i] for i in range(E)]
+            best = max(itertools.combinations(range(E), k), key=lambda s: sum(key[i] for i in s))
+            assert ids[t].tolist() == sorted(best, key=lambda i: -key[i])
+            np.testing.assert_allclose(w[t], scipy.special.softmax(l[t, ids[t]]), rtol=1e-13)
+
+
+def test_select_bias_forces_expert_without_changing_its_share():
+    """A large bias on expert 3 makes it slot 0 of every token; the weights
+    are those of softmax over the same experts with no bias."""
+    rng = np.random.default_rng(23)
+    l = rng.standard_normal((30, 8))
+    b = np.zeros(8)
+    b[3] = 50.0
+    ids, w = om.route_scored(l, b, 3, "softmax_select_bias")
+    assert np.all(ids[:, 0] == 3)
+    ids_sm, w_sm = om.route_scored(l, b, 3, "softmax")
+    np.testing.assert_array_equal(ids, ids_sm)
+    assert np.all(w_sm[:, 0] > 1 - 1e-15)         # bias inside the softmax swamps the rest
+    assert np.all(w[:, 0] < 0.999)                # ... but not under select-only bias
+    # shifting every bias by a constant changes nothing
+    ids2, w2 = om.route_scored(l, b - 7.25, 3, "softmax_select_bias")
+    np.testing.assert_array_equal(ids2, ids)
+    np.testing.assert_allclose(w2, w, rtol=1e-15)
+
+
+def test_sigmoid_weights_worked_by_hand():
+    """l = [ln 3, 0, -ln 3] has sigmoids [3/4, 1/2, 1/4]: top-2 weights
+    (3/5, 2/5), all three (1/2, 1/3, 1/6), top-1 exactly 1."""
+    l = np.array([[math.log(3.0), 0.0, -math.log(3.0)]])
+    ids, w = om.route_scored(l, None, 2, "sigmoid")
+    assert ids[0].tolist() == [0, 1]
+    np.testing.assert_allclose(w[0], [3 / 5, 2 / 5], rtol=1e-15)
+    ids, w = om.route_scored(l, None, 3, "sigmoid")
+    np.testing.assert_allclose(w[0], [1 / 2, 1 / 3, 1 / 6], rtol=1e-15)
+    _, w = om.route_scored(l[:, ::-1].copy(), None, 1, "sigmoid")
+    assert w[0, 0] == 1.0
+
+
+def test_sigmoid_bias_is_added_after_the_sigmoid():
+    """l = [2, 0], b = [0, 0.5]: sigmoid keys 0.881 < 1.0 pick expert 1,
+    while l + b = [2, 0.5] picks expert 0.  Weights never see the bias."""
+    l = np.array([[2.0, 0.0]])
+    b = np.array([0.0, 0.5])
+    ids, w = om.route_scored(l, b, 1, "sigmoid")
+    assert ids[0].tolist() == [1] and w[0, 0] == 1.0
+    ids, _ = om.route_scored(l, b, 1, "softmax_select_bias")
+    assert ids[0].tolist() == [0]
+    ids, w = om.route_scored(l, b, 2, "sigmoid")
+    assert ids[0].tolist() == [1, 0]
+    np.testing.assert_allclose(w[0], [0.5 / (0.5 + sig(2)), sig(2) / (0.5 + sig(2))], rtol=1e-14)
+
+
+def test_sigmoid_picks_best_subset_and_matches_expit():
+    rng = np.random.default_rng(24)
+    for E, k in [(6, 2), (7, 4), (4, 4)]:
+        l = rng.standard_normal((25, E)) * 2
+        b = rng.standard_normal(E) * 0.2
+        ids, w = om.route_scored(l, b, k, "sigmoid")
+        for t in range(25):
+            key = [sig(l[t, i]) + b[i] for i in range(E)]
+            best = max(itertools.combinations(range(E), k), key=lambda s: sum(key[i] for i in s))
+            assert ids[t].tolist() == sorted(best, key=lambda i: -key[i])
+            s = scipy.special.expit(l[t, ids[t]])
+            np.testing.assert_allclose(w[t], s / s.sum(), rtol=1e-14)
+
+
+def test_sigmoid_extreme_logits_stay_finite():
+    l = np.array([[800.0, -800.0, 0.0, -30.0]])
+    ids, w = om.route_scored(l, None, 4, "sigmoid")
+    assert ids[0].tolist() == [0, 2, 3, 1]
+    assert np.all(np.isfinite(w)) and w[0, 3] == 0.0
+    np.testing.assert_allclose(w[0, :2], [2 / 3, 1 / 3], rtol=1e-12)
+    with pytest.raises(ValueError):
+        om.route_scored(l, None, 2, "tanh")
+
+
+def test_identical_experts_give_dense_ffn_under_every_scoring():
+    rng = np.random.default_rng(25)
+    T, H, E, I, k = 10, 16, 6, 8, 3
+    x = _bf(rng, (T, H), 1)
+    gu1, d1 = _bf(rng, (H, 2 * I), 0.3), _bf(rng, (I, H), 0.3)
+    Wgu, Wd = np.stack([gu1] * E), np.stack([d1] * E)
+    Wr = rng.standard_normal((H, E)).astype(np.float32)
+    b = rng.standard_normal(E).astype(np.float32)
+    dense = om.dense_swiglu_ffn(x, gu1, d1)
+    for scoring in om.SCORINGS:
+        out = om.layer_forward(x, Wr, b, Wgu, Wd, k, scoring=scoring)
+        np.testing.assert_allclose(out["y"], dense, rtol=1e-12, atol=1e-14)
+        ids, _ = om.route_scored(om.router_logits(x, Wr, None), b, k, scoring)
+        np.testing.assert_array_equal(out["ids"], ids)
+
+
+def test_gap_guarantee_holds_on_sigmoid_keys():
+    cfg = synth.Config("gap_sig", T=64, H=256, E=16, I=128, k=4, bias="zipf:0.05")
+    inp = synth.make_inputs(cfg)
+    oracle.enforce_logit_gap(inp, scoring="sigmoid")
+    keys = om.selection_keys(om.router_logits(inp.x, inp.w_router, None), inp.bias, "sigmoid")
+    top = -np.sort(-keys, axis=1)[:, :cfg.k + 1]
+    assert np.all(top[:, :-1] - top[:, 1:] >= synth.gap_target())
+
+
 # ---------------------------------------------------------------- permutation
 
 def _random_ids(rng, T, E, k):
