@@ -230,10 +230,12 @@ def recorded_traffic(workload):
 
 # ---------------------------------------------------------------- timed runs
 TILES = {"auto": 0, "small": 1, "large": 2, "pair": 3, "fused": 4}
+# router scoring rules (an extra workload "name:rule" is timed under that rule)
+SCORING = {"softmax": 0, "softmax_select_bias": 1, "sigmoid": 2}
 
 
 def time_workload(cfg, d, ws, steps, warmup, rank, world, flush, moe, gpu_index, sample_clocks=True, tiles=0,
-                  graph=False):
+                  graph=False, scoring=0):
     """K timed steps (L2 flushed before each).  graph=True captures one layer
     call in a CUDA graph and replays it per step (no host launch overhead);
     otherwise every step is an eager library call."""
@@ -244,7 +246,8 @@ def time_workload(cfg, d, ws, steps, warmup, rank, world, flush, moe, gpu_index,
 
     def step(evs=None, info=None):
         return moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws,
-                           d["w_sh_gate_up"], d["w_sh_down"], stage_events=evs, info=info, tiles=tiles, out=out)
+                           d["w_sh_gate_up"], d["w_sh_down"], stage_events=evs, info=info, tiles=tiles, out=out,
+                           scoring=scoring)
 
     def events(n):
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
@@ -466,7 +469,9 @@ def run_ours(args):
         del d
         torch.cuda.empty_cache()
         loaded = None
-        for name in args.extra.split(","):
+        for spec in args.extra.split(","):
+            name, _, sc_name = spec.partition(":")
+            scoring = SCORING[sc_name or "softmax"]
             ecfg = synth.CONFIGS[name]
             key = (ecfg.H, ecfg.E, ecfg.I, ecfg.I_s, ecfg.bias)
             if loaded is None or loaded[0] != key:
@@ -478,12 +483,12 @@ def run_ours(args):
                 torch.bfloat16).cuda()
             wse = moe.alloc_workspace(ecfg.T, ecfg.H, ecfg.E, ecfg.I, ecfg.k, ecfg.I_s)
             eres = time_workload(ecfg, de, wse, args.steps, args.warmup, rank, world, flush, moe, gpu_index,
-                                 sample_clocks=False, tiles=tiles)
+                                 sample_clocks=False, tiles=tiles, scoring=scoring)
             gres = time_workload(ecfg, de, wse, args.steps, args.warmup, rank, world, flush, moe, gpu_index,
-                                 sample_clocks=False, tiles=tiles, graph=True)
+                                 sample_clocks=False, tiles=tiles, graph=True, scoring=scoring)
             ecounts = moe.workspace_view(wse, ecfg.T, ecfg.H, ecfg.E, ecfg.I, ecfg.k, ecfg.I_s)["counts"]
             eacc = layer_accounting(ecfg, ecounts.cpu().numpy())
-            extra[name] = {"value": round(gres["value"], 1), "unit": "tokens/s",
+            extra[spec] = {"value": round(gres["value"], 1), "unit": "tokens/s",
                            "ms_per_step": round(gres["ms_per_step"], 4), "eager": eager_of(eres),
                            **roof(ecfg, eres, eacc, gres["ms_per_step"])}
             del wse
@@ -568,7 +573,9 @@ def main():
     ap.add_argument("--ref-sample-tokens", type=int, default=2)
     ap.add_argument("--tiles", choices=sorted(TILES), default="auto", help="grouped GEMM tile policy (tuning)")
     ap.add_argument("--extra", default="", help="comma-separated further workloads to time, e.g. "
-                                                 "ling_skewed_t4096,sweep_decode_t1")
+                                                 "ling_skewed_t4096,sweep_decode_t1; name:sigmoid or "
+                                                 "name:softmax_select_bias times it under that router "
+                                                 "scoring rule")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

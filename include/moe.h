@@ -5,7 +5,9 @@
  *
  *   route    l = x . W_router (+ bias), fp32; p = softmax(l) over E experts;
  *            the k largest p per token (descending, ties to the lower id);
- *            w_j = p_j / sum of the k selected p.
+ *            w_j = p_j / sum of the k selected p.  (Two further scoring
+ *            rules, in which the bias steers only the selection:
+ *            MOE_SCORE_* below.)
  *   permute  slots (t, j) sorted into expert-contiguous order, experts
  *            ascending, tokens ascending within an expert.
  *   gate/up  per permuted row r (token t, expert e):
@@ -97,6 +99,20 @@ enum {
 /* MOE_ROUTER_AUTO picks SMALL when T <= 16 and E % 4 == 0, else TC when
  * E % 8 == 0, else FMA. */
 
+/* Router scoring: how the k experts of a token are selected and weighted
+ * from its fp32 logits l[e] and the optional per-expert bias b[e].  The
+ * Qwen 3.5-397B-on-Ironwood page ("key optimisations", expert load
+ * balancing) names hot experts and a router balancing term, and the Ling
+ * page a per-expert router bias, without a formula; SOFTMAX is the rule of
+ * the layer's workloads, the other two are the common forms in which the
+ * bias steers only the selection.  In every form the k selected are listed
+ * by descending key, ties to the lower expert id. */
+enum {
+  MOE_SCORE_SOFTMAX = 0,             /* key = l + b; w_j = softmax over the selected keys */
+  MOE_SCORE_SOFTMAX_SELECT_BIAS = 1, /* key = l + b; w_j = softmax over the selected unbiased l */
+  MOE_SCORE_SIGMOID = 2              /* s = sigmoid(l); key = s + b; w_j = s_j / sum of the selected s */
+};
+
 /* Human-readable name of a status code (static storage). */
 const char *moe_status_string(int status);
 
@@ -149,6 +165,14 @@ moe_status_t moe_route_ex(const uint16_t *x, const float *w_router, const float 
                           int T, int H, int E, int k,
                           int32_t *topk_ids, float *topk_w, int router_impl,
                           void *workspace, size_t workspace_bytes, void *stream);
+
+/* Same, under a scoring rule (MOE_SCORE_*; moe_route_ex is MOE_SCORE_SOFTMAX).
+ * bias may be NULL under every rule.  An unknown rule returns
+ * MOE_ERR_INVALID_ARG. */
+moe_status_t moe_route_scored(const uint16_t *x, const float *w_router, const float *bias,
+                              int T, int H, int E, int k, int scoring,
+                              int32_t *topk_ids, float *topk_w, int router_impl,
+                              void *workspace, size_t workspace_bytes, void *stream);
 
 /* Permute: counts [E], offsets [E+1] (exclusive prefix sum, offsets[E] =
  * T*k), sorted_token_ids [T*k] (permuted row -> token) and inv_perm [T,k]
@@ -240,7 +264,10 @@ typedef struct moe_forward_options {
   void *stage_events[7];
   /* Output: the number of kernels this call enqueued. */
   int launches;
-  int reserved[5];
+  /* Router scoring rule (MOE_SCORE_*; 0, the zero-initialised default, is
+   * MOE_SCORE_SOFTMAX). */
+  int scoring;
+  int reserved[4];
 } moe_forward_options_t;
 
 moe_status_t moe_forward_ex(const uint16_t *x, const float *w_router, const float *bias,

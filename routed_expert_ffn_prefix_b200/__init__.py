@@ -19,6 +19,7 @@ from . import build as _build
 __all__ = [
     "MoEError", "lib", "TILES_AUTO", "TILES_SMALL", "TILES_LARGE", "TILES_PAIR", "TILES_FUSED",
     "ROUTER_AUTO", "ROUTER_FMA", "ROUTER_TC", "ROUTER_SMALL",
+    "SCORE_SOFTMAX", "SCORE_SOFTMAX_SELECT_BIAS", "SCORE_SIGMOID",
     "workspace_size", "workspace_layout", "alloc_workspace", "route", "permute", "grouped_swiglu",
     "grouped_down", "down_combine", "forward", "device_status", "clear_device_status", "selftest_timeout",
     "STATUS",
@@ -26,6 +27,7 @@ __all__ = [
 
 TILES_AUTO, TILES_SMALL, TILES_LARGE, TILES_PAIR, TILES_FUSED = 0, 1, 2, 3, 4
 ROUTER_AUTO, ROUTER_FMA, ROUTER_TC, ROUTER_SMALL = 0, 1, 2, 3
+SCORE_SOFTMAX, SCORE_SOFTMAX_SELECT_BIAS, SCORE_SIGMOID = 0, 1, 2
 
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_ALIGNMENT", 3: "MOE_ERR_WORKSPACE",
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT", 6: "MOE_ERR_UNSUPPORTED_ARCH",
@@ -46,7 +48,8 @@ class _Layout(ctypes.Structure):
 
 class _Options(ctypes.Structure):
     _fields_ = [("tile_policy", ctypes.c_int), ("router_impl", ctypes.c_int),
-                ("stage_events", ctypes.c_void_p * 7), ("launches", ctypes.c_int), ("reserved", ctypes.c_int * 5)]
+                ("stage_events", ctypes.c_void_p * 7), ("launches", ctypes.c_int), ("scoring", ctypes.c_int),
+                ("reserved", ctypes.c_int * 4)]
 
 
 _P, _I, _Z, _U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint64
@@ -59,6 +62,7 @@ _SIGS = {
     "moe_clear_device_status": ([_P, _P], _I),
     "moe_route": ([_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _Z, _P], _I),
     "moe_route_ex": ([_P, _P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _Z, _P], _I),
+    "moe_route_scored": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _Z, _P], _I),
     "moe_permute": ([_P, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P], _I),
     "moe_grouped_swiglu": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _Z, _P], _I),
     "moe_grouped_down": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _Z, _P], _I),
@@ -143,8 +147,8 @@ def clear_device_status(ws) -> None:
     _check(lib().moe_clear_device_status(_ptr(ws), _stream()), "moe_clear_device_status")
 
 
-def route(x, w_router, bias, k, ws, impl=ROUTER_AUTO, out=None):
-    """topk_ids [T,k] int32, topk_w [T,k] float32."""
+def route(x, w_router, bias, k, ws, impl=ROUTER_AUTO, out=None, scoring=SCORE_SOFTMAX):
+    """topk_ids [T,k] int32, topk_w [T,k] float32 (scoring: SCORE_*)."""
     import torch
     _need(x, torch.bfloat16, "x", 2)
     _need(w_router, torch.float32, "w_router", 2)
@@ -154,8 +158,8 @@ def route(x, w_router, bias, k, ws, impl=ROUTER_AUTO, out=None):
     E = w_router.shape[1]
     ids, w = out if out is not None else (
         torch.empty(T, k, dtype=torch.int32, device=x.device), torch.empty(T, k, dtype=torch.float32, device=x.device))
-    _check(lib().moe_route_ex(_ptr(x), _ptr(w_router), _ptr(bias), T, H, E, k, _ptr(ids), _ptr(w), impl,
-                              _ptr(ws), ws.numel(), _stream()), "moe_route")
+    _check(lib().moe_route_scored(_ptr(x), _ptr(w_router), _ptr(bias), T, H, E, k, scoring, _ptr(ids), _ptr(w),
+                                  impl, _ptr(ws), ws.numel(), _stream()), "moe_route")
     return ids, w
 
 
@@ -222,8 +226,9 @@ def down_combine(h, w_down, topk_w, inv_perm, offsets, shared_out, ws, tiles=TIL
 
 
 def forward(x, w_router, bias, w_gate_up, w_down, k, ws, w_sh_gate_up=None, w_sh_down=None,
-            tiles=TILES_AUTO, router=ROUTER_AUTO, out=None, stage_events=None, info=None):
-    """The whole layer: y [T,H] bf16.
+            tiles=TILES_AUTO, router=ROUTER_AUTO, out=None, stage_events=None, info=None,
+            scoring=SCORE_SOFTMAX):
+    """The whole layer: y [T,H] bf16 (scoring: the router's SCORE_* rule).
 
     stage_events: optional list of 7 torch.cuda.Event recorded at the stage
     boundaries (see include/moe.h); info: optional dict that receives the
@@ -243,6 +248,7 @@ def forward(x, w_router, bias, w_gate_up, w_down, k, ws, w_sh_gate_up=None, w_sh
         I_s = w_sh_gate_up.shape[1] // 2
     y = out if out is not None else torch.empty(T, H, dtype=torch.bfloat16, device=x.device)
     opt = _Options(tiles, router)
+    opt.scoring = scoring
     if stage_events is not None:
         for i, ev in enumerate(stage_events):
             if ev is not None:

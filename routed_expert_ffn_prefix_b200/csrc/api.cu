@@ -20,6 +20,10 @@ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 // MOE_ROUTER_AUTO: a few tokens -> the one-launch split-H router; else tensor
 // cores whenever the 16-byte row pitch of the split planes allows it
 // (E % 8 == 0), else fp32 CUDA cores.
+inline bool valid_scoring(int scoring) {
+  return scoring == MOE_SCORE_SOFTMAX || scoring == MOE_SCORE_SOFTMAX_SELECT_BIAS || scoring == MOE_SCORE_SIGMOID;
+}
+
 inline int resolve_router(int impl, int T, int E) {
   if (impl != MOE_ROUTER_AUTO) return impl;
   if (T <= kSmallRouterT && E % 4 == 0) return MOE_ROUTER_SMALL;
@@ -249,7 +253,7 @@ struct PermOut {
 };
 
 moe_status_t run_route(const uint16_t* x, const float* w_router, const float* bias, int T, int H, int E, int k,
-                       int32_t* ids, float* w, int impl, void* ws, const moe_workspace_layout_t& L,
+                       int scoring, int32_t* ids, float* w, int impl, void* ws, const moe_workspace_layout_t& L,
                        const DeviceInfo& dev, cudaStream_t s, const PermOut* perm = nullptr) {
   DevStatus* st = status_of(ws);
   float* logits = at<float>(ws, L.logits);
@@ -257,7 +261,7 @@ moe_status_t run_route(const uint16_t* x, const float* w_router, const float* bi
   if (impl == MOE_ROUTER_SMALL) {
     if (T > kSmallRouterT) return MOE_ERR_INVALID_ARG;
     if (E % 4 != 0) return MOE_ERR_ALIGNMENT;
-    return cuda_status(launch_router_small(x, w_router, bias, T, H, E, k, logits, &st->arrivals, ids, w,
+    return cuda_status(launch_router_small(x, w_router, bias, T, H, E, k, scoring, logits, &st->arrivals, ids, w,
                                            perm ? perm->counts : nullptr, perm ? perm->offsets : nullptr,
                                            perm ? perm->sorted_ids : nullptr, perm ? perm->inv_perm : nullptr, st,
                                            s));
@@ -299,7 +303,7 @@ moe_status_t run_route(const uint16_t* x, const float* w_router, const float* bi
     MOE_TRY(cuda_status(launch_router_logits_fma(x, w_router, T, H, E, logits, s)));
     nsplit = fma_router_splits(T, H);
   }
-  return cuda_status(launch_topk(logits, nsplit, (size_t)T * E, bias, T, E, k, ids, w, st, s));
+  return cuda_status(launch_topk(logits, nsplit, (size_t)T * E, bias, T, E, k, scoring, ids, w, st, s));
 }
 
 // nsplit > 1: K-split into partial slabs [nsplit][rows][2I] f32 at `partials`
@@ -445,19 +449,27 @@ moe_status_t moe_clear_device_status(void* workspace, void* stream) {
   return cuda_status(cudaMemsetAsync(workspace, 0, sizeof(DevStatus), static_cast<cudaStream_t>(stream)));
 }
 
-moe_status_t moe_route_ex(const uint16_t* x, const float* w_router, const float* bias, int T, int H, int E, int k,
-                          int32_t* topk_ids, float* topk_w, int router_impl, void* workspace,
-                          size_t workspace_bytes, void* stream) {
+moe_status_t moe_route_scored(const uint16_t* x, const float* w_router, const float* bias, int T, int H, int E,
+                              int k, int scoring, int32_t* topk_ids, float* topk_w, int router_impl, void* workspace,
+                              size_t workspace_bytes, void* stream) {
   if (!all_nonnull(x, w_router, topk_ids, topk_w)) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_shapes(T, H, E, 0, k, false));
   if (router_impl < MOE_ROUTER_AUTO || router_impl > MOE_ROUTER_SMALL) return MOE_ERR_INVALID_ARG;
+  if (!valid_scoring(scoring)) return MOE_ERR_INVALID_ARG;
   if (!all_aligned(x, w_router, topk_ids, topk_w) || (bias && !aligned16(bias))) return MOE_ERR_ALIGNMENT;
   const moe_workspace_layout_t L = make_layout(T, H, E, 0, k, 0);
   MOE_TRY(check_ws(workspace, workspace_bytes, L.h));
   DeviceInfo dev;
   MOE_TRY(check_device(&dev));
-  return run_route(x, w_router, bias, T, H, E, k, topk_ids, topk_w, router_impl, workspace, L, dev,
+  return run_route(x, w_router, bias, T, H, E, k, scoring, topk_ids, topk_w, router_impl, workspace, L, dev,
                    static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_route_ex(const uint16_t* x, const float* w_router, const float* bias, int T, int H, int E, int k,
+                          int32_t* topk_ids, float* topk_w, int router_impl, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  return moe_route_scored(x, w_router, bias, T, H, E, k, MOE_SCORE_SOFTMAX, topk_ids, topk_w, router_impl, workspace,
+                          workspace_bytes, stream);
 }
 
 moe_status_t moe_route(const uint16_t* x, const float* w_router, const float* bias, int T, int H, int E, int k,
@@ -549,8 +561,10 @@ moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const floa
   }
   const int tile_policy = options ? options->tile_policy : MOE_TILES_AUTO;
   const int router_impl = options ? options->router_impl : MOE_ROUTER_AUTO;
+  const int scoring = options ? options->scoring : MOE_SCORE_SOFTMAX;
   if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_FUSED) return MOE_ERR_INVALID_ARG;
   if (router_impl < MOE_ROUTER_AUTO || router_impl > MOE_ROUTER_SMALL) return MOE_ERR_INVALID_ARG;
+  if (!valid_scoring(scoring)) return MOE_ERR_INVALID_ARG;
   if (!all_aligned(x, w_router, w_gate_up, w_down, y) || (bias && !aligned16(bias))) return MOE_ERR_ALIGNMENT;
   const moe_workspace_layout_t L = make_layout(T, H, E, I, k, shared ? I_s : 0);
   MOE_TRY(check_ws(workspace, workspace_bytes, L.total));
@@ -585,8 +599,9 @@ moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const floa
     float* gslabs = slabs;
     float* dslabs = slabs + (size_t)kFusedMaxSplit * frows * 2 * imax;
     MOE_TRY(mark(0));
-    MOE_TRY(cuda_status(launch_fused_decode(x, w_router, bias, w_gate_up, w_down, shared ? w_sh_gate_up : nullptr,
-                                            shared ? w_sh_down : nullptr, shared ? I_s : 0, T, H, E, I, k,
+    MOE_TRY(cuda_status(launch_fused_decode(x, w_router, bias, scoring, w_gate_up, w_down,
+                                            shared ? w_sh_gate_up : nullptr, shared ? w_sh_down : nullptr,
+                                            shared ? I_s : 0, T, H, E, I, k,
                                             at<float>(ws, L.logits), gslabs, dslabs, ids, tw, counts, offs, sids, inv,
                                             y, st, kDefaultTimeoutNs, dev.num_sms, s)));
     for (int i = 1; i < 7; ++i) MOE_TRY(mark(i));
@@ -598,11 +613,11 @@ moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const floa
   MOE_TRY(mark(0));
   if (ri == MOE_ROUTER_SMALL) {
     const PermOut perm{counts, offs, sids, inv};
-    MOE_TRY(run_route(x, w_router, bias, T, H, E, k, ids, tw, ri, ws, L, dev, s, &perm));
+    MOE_TRY(run_route(x, w_router, bias, T, H, E, k, scoring, ids, tw, ri, ws, L, dev, s, &perm));
     launches += 1;
     MOE_TRY(mark(1));
   } else {
-    MOE_TRY(run_route(x, w_router, bias, T, H, E, k, ids, tw, ri, ws, L, dev, s));
+    MOE_TRY(run_route(x, w_router, bias, T, H, E, k, scoring, ids, tw, ri, ws, L, dev, s));
     launches += ri == MOE_ROUTER_TC ? 3 : 2;
     MOE_TRY(mark(1));
     MOE_TRY(cuda_status(

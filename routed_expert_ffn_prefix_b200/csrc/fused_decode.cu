@@ -56,6 +56,7 @@ struct FusedArgs {
   const __nv_bfloat16* x;
   const float* w_router;
   const float* bias;
+  int scoring;  // MOE_SCORE_*
   const __nv_bfloat16* w_gate_up;
   const __nv_bfloat16* w_down;
   const __nv_bfloat16* w_sh_gate_up;
@@ -223,7 +224,8 @@ __global__ void __launch_bounds__(kFThreads) fused_decode_kernel(const FusedArgs
 
   // ---------------------------------------------------------------- P: top-k, permutation, plan
   for (int t = warp; t < T; t += kFWarps)
-    router_select<EPL>(a.rslabs, a.rhs, a.bias, T, a.E, k, t, P.sel + t * k, P.w + t * k, nullptr, a.st);
+    router_select<EPL>(a.rslabs, a.rhs, a.bias, T, a.E, k, a.scoring, t, P.sel + t * k, P.w + t * k, nullptr,
+                       a.st);
   for (int e = tid; e < a.E; e += kFThreads) P.cnt[e] = 0;
   __syncthreads();
   for (int s = tid; s < n; s += kFThreads) atomicAdd(&P.cnt[P.sel[s]], 1);
@@ -470,7 +472,7 @@ size_t fused_decode_smem(int H, int I, int I_s) {
          (size_t)kFT * Imax * 2;
 }
 
-cudaError_t launch_fused_decode(const uint16_t* x, const float* w_router, const float* bias,
+cudaError_t launch_fused_decode(const uint16_t* x, const float* w_router, const float* bias, int scoring,
                                 const uint16_t* w_gate_up, const uint16_t* w_down, const uint16_t* w_sh_gate_up,
                                 const uint16_t* w_sh_down, int I_s, int T, int H, int E, int I, int k,
                                 float* rslabs, float* gslabs, float* dslabs, int32_t* ids, float* tw,
@@ -480,6 +482,7 @@ cudaError_t launch_fused_decode(const uint16_t* x, const float* w_router, const 
   a.x = reinterpret_cast<const __nv_bfloat16*>(x);
   a.w_router = w_router;
   a.bias = bias;
+  a.scoring = scoring;
   a.w_gate_up = reinterpret_cast<const __nv_bfloat16*>(w_gate_up);
   a.w_down = reinterpret_cast<const __nv_bfloat16*>(w_down);
   a.w_sh_gate_up = reinterpret_cast<const __nv_bfloat16*>(w_sh_gate_up);

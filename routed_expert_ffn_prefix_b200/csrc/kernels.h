@@ -93,9 +93,10 @@ cudaError_t launch_router_split(const float* w, int H, int E, uint16_t* planes, 
 int fma_router_splits(int T, int H);
 cudaError_t launch_router_logits_fma(const uint16_t* x, const float* w, int T, int H, int E, float* logits,
                                      cudaStream_t s);
-// logits: nsplit partial slabs of [T, E], split_stride elements apart, summed in slab order.
+// logits: nsplit partial slabs of [T, E], split_stride elements apart, summed in slab order;
+// scoring: MOE_SCORE_*.
 cudaError_t launch_topk(const float* logits, int nsplit, size_t split_stride, const float* bias, int T, int E, int k,
-                        int32_t* ids, float* w, DevStatus* st, cudaStream_t s);
+                        int scoring, int32_t* ids, float* w, DevStatus* st, cudaStream_t s);
 
 // Permutation.
 int permute_num_blocks(int T, int k);
@@ -116,7 +117,7 @@ cudaError_t launch_swiglu_reduce(const float* partials, int nsplit, size_t split
 // Router for a few tokens (T <= kSmallRouterT, E % 4 == 0): fp32 logits with
 // H split over blocks; the last block to finish sums the partial slabs
 // (small_router_slabs(H, E) of them, [slab][T][E] in `partial`) in slab
-// order, selects the top-k and, if counts != nullptr, writes the
+// order, selects the top-k under the scoring rule (MOE_SCORE_*) and, if counts != nullptr, writes the
 // permutation (counts, offsets, sorted_ids, inv_perm) as launch_permute
 // would.  *arrivals must be zero on entry and is zero again on exit.
 constexpr int kSmallRouterT = 16;
@@ -132,7 +133,7 @@ constexpr int kFusedMaxT = 4;
 constexpr int kFusedMaxK = 16;
 constexpr int kFusedMaxSplit = 8;
 bool fused_decode_supported(int T, int H, int E, int I, int k, int I_s);
-cudaError_t launch_fused_decode(const uint16_t* x, const float* w_router, const float* bias,
+cudaError_t launch_fused_decode(const uint16_t* x, const float* w_router, const float* bias, int scoring,
                                 const uint16_t* w_gate_up, const uint16_t* w_down, const uint16_t* w_sh_gate_up,
                                 const uint16_t* w_sh_down, int I_s, int T, int H, int E, int I, int k,
                                 float* rslabs, float* gslabs, float* dslabs, int32_t* ids, float* tw,
@@ -140,9 +141,9 @@ cudaError_t launch_fused_decode(const uint16_t* x, const float* w_router, const 
                                 uint16_t* y, DevStatus* st, uint64_t timeout_ns, int num_sms, cudaStream_t s);
 int small_router_slabs(int H, int E);
 cudaError_t launch_router_small(const uint16_t* x, const float* w, const float* bias, int T, int H, int E, int k,
-                                float* partial, unsigned int* arrivals, int32_t* ids, float* wout, int32_t* counts,
-                                int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm, DevStatus* st,
-                                cudaStream_t s);
+                                int scoring, float* partial, unsigned int* arrivals, int32_t* ids, float* wout,
+                                int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
+                                DevStatus* st, cudaStream_t s);
 
 cudaError_t launch_selftest_timeout(DevStatus* st, uint64_t timeout_ns, cudaStream_t s);
 

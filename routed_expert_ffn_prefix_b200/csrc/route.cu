@@ -120,12 +120,15 @@ __device__ __forceinline__ void load_logits(const float* __restrict__ row, int E
 
 // One warp per token; EPL = experts per lane (E <= 32 * EPL).  The K-split
 // partial slabs are summed in slab order; UNR slabs are loaded before any is
-// added so that UNR * EPL values per lane are in flight at once.
-template <int EPL, int UNR, bool QUAD>
+// added so that UNR * EPL values per lane are in flight at once.  SEL: a
+// scoring rule in which the bias steers only the selection (scoring is
+// MOE_SCORE_SOFTMAX_SELECT_BIAS or MOE_SCORE_SIGMOID); otherwise softmax.
+template <int EPL, int UNR, bool QUAD, bool SEL>
 __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __restrict__ logits, int nsplit,
                                                              size_t split_stride, const float* __restrict__ bias,
-                                                             int T, int E, int k, int32_t* __restrict__ ids,
-                                                             float* __restrict__ wout, DevStatus* st) {
+                                                             int T, int E, int k, int scoring,
+                                                             int32_t* __restrict__ ids, float* __restrict__ wout,
+                                                             DevStatus* st) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kTopkWarps + warp;
   if (t >= T) return;
@@ -148,19 +151,18 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
 #pragma unroll
     for (int i = 0; i < EPL; ++i) v[i] += p[i];
   }
-#pragma unroll
-  for (int i = 0; i < EPL; ++i) {
-    const int e = entry_expert<QUAD>(lane, i);
-    v[i] = e < E ? v[i] + (bias ? bias[e] : 0.f) : -INFINITY;
-  }
-  warp_topk<EPL, QUAD>(v, E, k, t, ids + (size_t)t * k, wout + (size_t)t * k, nullptr, st);
+  float src[EPL];
+  score_entries<EPL, QUAD>(v, src, bias, E, lane, SEL ? scoring : MOE_SCORE_SOFTMAX);
+  warp_topk<EPL, QUAD, SEL>(v, src, scoring == MOE_SCORE_SOFTMAX_SELECT_BIAS, E, k, t, ids + (size_t)t * k,
+                            wout + (size_t)t * k, nullptr, st);
 }
 
 template <int EPL, int UNR, bool QUAD = false>
 cudaError_t launch_topk_t(const float* logits, int nsplit, size_t split_stride, const float* bias, int T, int E,
-                          int k, int32_t* ids, float* w, DevStatus* st, cudaStream_t s) {
-  return launch_kernel(topk_kernel<EPL, UNR, QUAD>, dim3((T + kTopkWarps - 1) / kTopkWarps), dim3(kTopkWarps * 32),
-                       0, s, logits, nsplit, split_stride, bias, T, E, k, ids, w, st);
+                          int k, int scoring, int32_t* ids, float* w, DevStatus* st, cudaStream_t s) {
+  auto kern = scoring == MOE_SCORE_SOFTMAX ? topk_kernel<EPL, UNR, QUAD, false> : topk_kernel<EPL, UNR, QUAD, true>;
+  return launch_kernel(kern, dim3((T + kTopkWarps - 1) / kTopkWarps), dim3(kTopkWarps * 32), 0, s, logits, nsplit,
+                       split_stride, bias, T, E, k, scoring, ids, w, st);
 }
 
 
@@ -173,7 +175,8 @@ cudaError_t launch_topk_t(const float* logits, int nsplit, size_t split_stride, 
 template <int TT, int EPL>
 __global__ void __launch_bounds__(kSmallThreads) router_small_kernel(
     const __nv_bfloat16* __restrict__ x, const float* __restrict__ w, const float* __restrict__ bias, int T, int H,
-    int E, int k, int chunk, int hs, float* __restrict__ partial, unsigned int* arrivals, int32_t* __restrict__ ids,
+    int E, int k, int scoring, int chunk, int hs, float* __restrict__ partial, unsigned int* arrivals,
+    int32_t* __restrict__ ids,
     float* __restrict__ wout, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
     int32_t* __restrict__ sorted_ids, int32_t* __restrict__ inv_perm, DevStatus* st) {
   __shared__ RouterSmem<TT> rsm;
@@ -190,9 +193,10 @@ __global__ void __launch_bounds__(kSmallThreads) router_small_kernel(
   if (!is_last) return;
   __threadfence();
 
-  // ---- last block: slab sum in slab order, bias, top-k (one warp per token)
+  // ---- last block: slab sum in slab order, scoring, top-k (one warp per token)
   for (int t = warp; t < T; t += kSmallThreads / 32)
-    router_select<EPL>(partial, hs, bias, T, E, k, t, ids + (size_t)t * k, wout + (size_t)t * k, sel + t * k, st);
+    router_select<EPL>(partial, hs, bias, T, E, k, scoring, t, ids + (size_t)t * k, wout + (size_t)t * k,
+                       sel + t * k, st);
   if (counts != nullptr) {
     // ---- permutation of the n = T*k slots, stable counting sort by expert
     const int n = T * k;
@@ -252,13 +256,13 @@ __global__ void __launch_bounds__(kSmallThreads) router_small_kernel(
 
 template <int TT, int EPL>
 cudaError_t launch_router_small_t(const uint16_t* x, const float* w, const float* bias, int T, int H, int E, int k,
-                                  float* partial, unsigned int* arrivals, int32_t* ids, float* wout,
+                                  int scoring, float* partial, unsigned int* arrivals, int32_t* ids, float* wout,
                                   int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
                                   DevStatus* st, cudaStream_t s) {
   const SmallGrid g = small_grid(H, E);
   return launch_kernel(router_small_kernel<TT, EPL>, dim3(g.ncs, g.hs), dim3(kSmallThreads), 0, s,
-                       reinterpret_cast<const __nv_bfloat16*>(x), w, bias, T, H, E, k, g.chunk, g.hs, partial,
-                       arrivals, ids, wout, counts, offsets, sorted_ids, inv_perm, st);
+                       reinterpret_cast<const __nv_bfloat16*>(x), w, bias, T, H, E, k, scoring, g.chunk, g.hs,
+                       partial, arrivals, ids, wout, counts, offsets, sorted_ids, inv_perm, st);
 }
 
 // accumulators for 1, 4 or 16 tokens
@@ -293,39 +297,40 @@ cudaError_t launch_router_logits_fma(const uint16_t* x, const float* w, int T, i
 }
 
 cudaError_t launch_topk(const float* logits, int nsplit, size_t split_stride, const float* bias, int T, int E, int k,
-                        int32_t* ids, float* w, DevStatus* st, cudaStream_t s) {
-  if (E <= 32) return launch_topk_t<1, 8>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
-  if (E <= 64) return launch_topk_t<2, 8>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
+                        int scoring, int32_t* ids, float* w, DevStatus* st, cudaStream_t s) {
+  if (E <= 32) return launch_topk_t<1, 8>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
+  if (E <= 64) return launch_topk_t<2, 8>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
   // E % 4 == 0 (and 16-byte aligned rows): each lane loads 4 experts per 16-byte load
   if (E % 4 == 0) {
-    if (E <= 128) return launch_topk_t<4, 8, true>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
-    if (E <= 256) return launch_topk_t<8, 4, true>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
-    if (E <= 512) return launch_topk_t<16, 4, true>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
-    return launch_topk_t<32, 2, true>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
+    if (E <= 128)
+      return launch_topk_t<4, 8, true>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
+    if (E <= 256)
+      return launch_topk_t<8, 4, true>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
+    if (E <= 512)
+      return launch_topk_t<16, 4, true>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
+    return launch_topk_t<32, 2, true>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
   }
-  if (E <= 128) return launch_topk_t<4, 8>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
-  if (E <= 256) return launch_topk_t<8, 4>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
-  if (E <= 512) return launch_topk_t<16, 4>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
-  return launch_topk_t<32, 2>(logits, nsplit, split_stride, bias, T, E, k, ids, w, st, s);
+  if (E <= 128) return launch_topk_t<4, 8>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
+  if (E <= 256) return launch_topk_t<8, 4>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
+  if (E <= 512) return launch_topk_t<16, 4>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
+  return launch_topk_t<32, 2>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
 }
 
 int small_router_slabs(int H, int E) { return small_grid(H, E).hs; }
 
 cudaError_t launch_router_small(const uint16_t* x, const float* w, const float* bias, int T, int H, int E, int k,
-                                float* partial, unsigned int* arrivals, int32_t* ids, float* wout, int32_t* counts,
-                                int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm, DevStatus* st,
-                                cudaStream_t s) {
+                                int scoring, float* partial, unsigned int* arrivals, int32_t* ids, float* wout,
+                                int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
+                                DevStatus* st, cudaStream_t s) {
   if (T < 1 || T > kSmallRouterT || E % 4 != 0 || k > 64) return cudaErrorInvalidValue;
-  if (E <= 64) return launch_router_small_e<2>(T, x, w, bias, T, H, E, k, partial, arrivals, ids, wout, counts,
-                                                offsets, sorted_ids, inv_perm, st, s);
-  if (E <= 128) return launch_router_small_e<4>(T, x, w, bias, T, H, E, k, partial, arrivals, ids, wout, counts,
-                                                 offsets, sorted_ids, inv_perm, st, s);
-  if (E <= 256) return launch_router_small_e<8>(T, x, w, bias, T, H, E, k, partial, arrivals, ids, wout, counts,
-                                                 offsets, sorted_ids, inv_perm, st, s);
-  if (E <= 512) return launch_router_small_e<16>(T, x, w, bias, T, H, E, k, partial, arrivals, ids, wout, counts,
-                                                  offsets, sorted_ids, inv_perm, st, s);
-  return launch_router_small_e<32>(T, x, w, bias, T, H, E, k, partial, arrivals, ids, wout, counts, offsets,
-                                   sorted_ids, inv_perm, st, s);
+#define MOE_SMALL_ARGS T, x, w, bias, T, H, E, k, scoring, partial, arrivals, ids, wout, counts, offsets, sorted_ids, \
+                       inv_perm, st, s
+  if (E <= 64) return launch_router_small_e<2>(MOE_SMALL_ARGS);
+  if (E <= 128) return launch_router_small_e<4>(MOE_SMALL_ARGS);
+  if (E <= 256) return launch_router_small_e<8>(MOE_SMALL_ARGS);
+  if (E <= 512) return launch_router_small_e<16>(MOE_SMALL_ARGS);
+  return launch_router_small_e<32>(MOE_SMALL_ARGS);
+#undef MOE_SMALL_ARGS
 }
 
 }  // namespace moe

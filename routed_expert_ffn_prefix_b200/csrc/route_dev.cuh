@@ -7,13 +7,21 @@
 
 namespace moe {
 
-// Top-k of one token by one warp: lane L holds the logits of experts
-// L + 32 i in v (entries >= E ignored).  k rounds of a warp arg-max (larger
-// logit first, ties to the lower expert id; NaN logits are never chosen),
-// then w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0) over the k selected
-// logits.  Each round takes the lane's best by a pairwise tree over its EPL
-// entries (log2 EPL dependent steps) and the warp's best by 5 shuffles.
-// sel, if given, receives the k ids too (shared memory of the caller).
+// Top-k of one token by one warp: lane L holds the selection keys of
+// experts L + 32 i in v (entries >= E ignored).  k rounds of a warp arg-max
+// (larger key first, ties to the lower expert id; NaN keys are never
+// chosen), then the weights.  Each round takes the lane's best by a pairwise
+// tree over its EPL entries (log2 EPL dependent steps) and the warp's best by
+// 5 shuffles.  sel, if given, receives the k ids too (shared memory of the
+// caller).
+//
+// Weights.  SEL = false (softmax scoring, bias inside the logits): the keys
+// are the logits and w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0) over the k
+// selected.  SEL = true (the bias steers only the selection): the weights
+// come from the unbiased per-expert values in `src` -- logits, normalised as
+// a softmax over the selected (exp_w), or sigmoid scores normalised by
+// their sum (!exp_w).  Lane j % 32 keeps the source value of slot j; the
+// max and the sum run over fixed shuffle trees.
 constexpr int kNoExpert = 0x7fffffff;
 
 __device__ __forceinline__ bool topk_better(float av, int ai, float bv, int bi) {
@@ -27,9 +35,17 @@ __device__ __forceinline__ int entry_expert(int lane, int i) {
   return QUAD ? 128 * (i >> 2) + 4 * lane + (i & 3) : lane + 32 * i;
 }
 
-template <int EPL, bool QUAD = false>
-__device__ __forceinline__ void warp_topk(const float (&vin)[EPL], int E, int k, int t, int32_t* idrow, float* wrow,
-                                          int32_t* sel, DevStatus* st) {
+// Lane holding expert e (inverse of entry_expert).
+template <bool QUAD>
+__device__ __forceinline__ int entry_lane(int e) {
+  return QUAD ? (e >> 2) & 31 : e & 31;
+}
+
+__device__ __forceinline__ float sigmoid_score(float z) { return 1.0f / (1.0f + expf(-z)); }
+
+template <int EPL, bool QUAD = false, bool SEL = false>
+__device__ __forceinline__ void warp_topk(const float (&vin)[EPL], const float (&src)[EPL], bool exp_w, int E, int k,
+                                          int t, int32_t* idrow, float* wrow, int32_t* sel, DevStatus* st) {
   const int lane = threadIdx.x & 31;
   float v[EPL];
   int id[EPL];
@@ -41,6 +57,7 @@ __device__ __forceinline__ void warp_topk(const float (&vin)[EPL], int E, int k,
     id[i] = ok ? e : kNoExpert;
   }
   float lead = 0.f, sum = 0.f;
+  float held0 = 0.f, held1 = 0.f;  // SEL: source values of slots lane and lane + 32
   for (int j = 0; j < k; ++j) {
     float tv[EPL];
     int ti[EPL];
@@ -59,26 +76,78 @@ __device__ __forceinline__ void warp_topk(const float (&vin)[EPL], int E, int k,
       const int oi = __shfl_xor_sync(0xffffffffu, bi, d);
       if (topk_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
     }
-    if (bi == kNoExpert) {  // no candidate left: the logits were NaN
+    if (bi == kNoExpert) {  // no candidate left: the keys were NaN
       if (lane == 0) raise_error(st, MOE_ERR_DEVICE_BOUNDS, SITE_TOPK, t);
       bi = 0;
       bv = lead;
     }
+    float mine = 0.f;
 #pragma unroll
     for (int i = 0; i < EPL; ++i)
-      if (id[i] == bi) { v[i] = -INFINITY; id[i] = kNoExpert; }
-    if (j == 0) lead = bv;
-    const float z = expf(bv - lead);
-    sum += z;
-    if (lane == 0) {
-      idrow[j] = bi;
-      wrow[j] = z;
-      if (sel) sel[j] = bi;
+      if (id[i] == bi) {
+        v[i] = -INFINITY;
+        id[i] = kNoExpert;
+        if constexpr (SEL) mine = src[i];
+      }
+    if constexpr (SEL) {
+      const float ws = __shfl_sync(0xffffffffu, mine, entry_lane<QUAD>(bi));
+      if (lane == (j & 31)) {
+        if (j < 32) held0 = ws;
+        else held1 = ws;
+      }
+      if (lane == 0) {
+        idrow[j] = bi;
+        if (sel) sel[j] = bi;
+      }
+    } else {
+      if (j == 0) lead = bv;
+      const float z = expf(bv - lead);
+      sum += z;
+      if (lane == 0) {
+        idrow[j] = bi;
+        wrow[j] = z;
+        if (sel) sel[j] = bi;
+      }
     }
   }
-  __syncwarp();
-  const float inv = 1.0f / sum;
-  for (int j = lane; j < k; j += 32) wrow[j] = wrow[j] * inv;
+  if constexpr (SEL) {
+    const bool h0 = lane < k, h1 = lane + 32 < k;
+    float z0 = h0 ? held0 : 0.f, z1 = h1 ? held1 : 0.f;
+    if (exp_w) {
+      float m = h0 ? held0 : -INFINITY;
+      if (h1) m = fmaxf(m, held1);
+#pragma unroll
+      for (int d = 16; d >= 1; d >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, d));
+      z0 = h0 ? expf(held0 - m) : 0.f;
+      z1 = h1 ? expf(held1 - m) : 0.f;
+    }
+    float tot = z0 + z1;
+#pragma unroll
+    for (int d = 16; d >= 1; d >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, d);
+    if (h0) wrow[lane] = z0 / tot;  // a division: one selected expert gets exactly 1
+    if (h1) wrow[lane + 32] = z1 / tot;
+  } else {
+    __syncwarp();
+    const float inv = 1.0f / sum;
+    for (int j = lane; j < k; j += 32) wrow[j] = wrow[j] * inv;
+  }
+}
+
+// Selection keys and weight sources of one lane's entries from its unbiased
+// logits v (in place: v becomes the keys), per scoring rule (MOE_SCORE_*):
+// softmax: key = l + b; select-only bias: key = l + b, src = l; sigmoid:
+// src = sigmoid(l), key = src + b.  Entries >= E get key -inf.
+template <int EPL, bool QUAD>
+__device__ __forceinline__ void score_entries(float (&v)[EPL], float (&src)[EPL], const float* __restrict__ bias,
+                                              int E, int lane, int scoring) {
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = entry_expert<QUAD>(lane, i);
+    const float l = v[i];
+    const float sv = scoring == MOE_SCORE_SIGMOID ? sigmoid_score(l) : l;
+    src[i] = e < E ? sv : 0.f;
+    v[i] = e < E ? sv + (bias ? bias[e] : 0.f) : -INFINITY;
+  }
 }
 
 // ---------------------------------------------------------------- few tokens
@@ -186,11 +255,12 @@ __device__ __forceinline__ void router_partial(const __nv_bfloat16* __restrict__
   }
 }
 
-// Slab sum (slab order), bias, top-k of token t by the calling warp.
+// Slab sum (slab order), scoring (MOE_SCORE_*), top-k of token t by the
+// calling warp.
 template <int EPL>
 __device__ __forceinline__ void router_select(const float* partial, int hs, const float* __restrict__ bias, int T,
-                                              int E, int k, int t, int32_t* idrow, float* wrow, int32_t* sel,
-                                              DevStatus* st) {
+                                              int E, int k, int scoring, int t, int32_t* idrow, float* wrow,
+                                              int32_t* sel, DevStatus* st) {
   const int lane = threadIdx.x & 31;
   float v[EPL];
 #pragma unroll
@@ -203,12 +273,12 @@ __device__ __forceinline__ void router_select(const float* partial, int hs, cons
       if (e < E) v[i] += __ldcg(slab + e);
     }
   }
-#pragma unroll
-  for (int i = 0; i < EPL; ++i) {
-    const int e = lane + 32 * i;
-    v[i] = e < E ? v[i] + (bias ? bias[e] : 0.f) : -INFINITY;
-  }
-  warp_topk<EPL>(v, E, k, t, idrow, wrow, sel, st);
+  float src[EPL];
+  score_entries<EPL, false>(v, src, bias, E, lane, scoring);
+  if (scoring == MOE_SCORE_SOFTMAX)
+    warp_topk<EPL, false, false>(v, v, true, E, k, t, idrow, wrow, sel, st);
+  else
+    warp_topk<EPL, false, true>(v, src, scoring == MOE_SCORE_SOFTMAX_SELECT_BIAS, E, k, t, idrow, wrow, sel, st);
 }
 
 }  // namespace moe

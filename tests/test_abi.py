@@ -93,6 +93,18 @@ def test_layout_rejects_bad_shapes(lib, T, H, E, I, k, Is, code):
     assert lib.moe_workspace_size(T, H, E, I, k, Is, ctypes.byref(n)) == code
 
 
+def test_forward_options_scoring_is_checked(lib):
+    """An unknown scoring rule in the options is refused on the host; the
+    options struct keeps its size (the field took a reserved slot)."""
+    ws = moe.workspace_size(64, 256, 8, 128, 2)
+    assert ctypes.sizeof(moe._Options) == 4 * 2 + 8 * 7 + 4 * 6
+    for bad_scoring in (-1, 3):
+        opt = moe._Options(0, 0)
+        opt.scoring = bad_scoring
+        assert lib.moe_forward_ex(p(), p(), None, p(), p(), None, None, 0, 64, 256, 8, 128, 2, p(), p(), ws,
+                                  ctypes.byref(opt), None) == 1
+
+
 def test_forward_argument_errors_before_any_launch(lib):
     f = lib.moe_forward
     ws = moe.workspace_size(64, 256, 8, 128, 2)
@@ -115,6 +127,9 @@ def test_stage_argument_errors(lib):
     ws = moe.workspace_size(64, 256, 8, 128, 2)
     assert lib.moe_route(None, p(), None, 64, 256, 8, 2, p(), p(), p(), ws, None) == 1
     assert lib.moe_route_ex(p(), p(), None, 64, 256, 8, 2, p(), p(), 7, p(), ws, None) == 1
+    for bad_scoring in (-1, 3):
+        assert lib.moe_route_scored(p(), p(), None, 64, 256, 8, 2, bad_scoring, p(), p(), 0, p(), ws, None) == 1
+    assert lib.moe_route_scored(p(), p(), p(FAKE + 4), 64, 256, 8, 2, 2, p(), p(), 0, p(), ws, None) == 2
     assert lib.moe_permute(p(), 64, 8, 2, p(), p(), p(), None, p(), ws, None) == 1
     assert lib.moe_permute(p(), 64, 8, 2, p(), p(), p(), p(), p(), 16, None) == 3
     assert lib.moe_grouped_swiglu(p(), p(), p(), p(), 64, 256, 8, 100, 2, 0, p(), p(), ws, None) == 2
