@@ -11,8 +11,8 @@
 // run to run, whatever order the expert GEMM tiles finished in.
 //
 // Memory-bound: a block per (token, column slice), one 16-byte vector of a
-// row (4 columns) per thread and slot, the k slot loads of a thread issued
-// together.
+// row (4 columns) per thread and slot, the slot loads of a thread issued
+// eight rows (and, for K-split slabs, up to two slabs) at a time.
 #include "gemm_units.cuh"
 
 namespace moe {
@@ -30,6 +30,14 @@ struct Vec<float> {
   static __device__ __forceinline__ void load(const float* p, float (&v)[4]) {
     const float4 q = __ldcs(reinterpret_cast<const float4*>(p));
     v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+  }
+  // load when `live`, zeros otherwise (rows past the token's k slots)
+  static __device__ __forceinline__ void load_if(bool live, const float* p, float (&v)[4]) {
+    if (live) {
+      load(p, v);
+    } else {
+      v[0] = v[1] = v[2] = v[3] = 0.f;
+    }
   }
 };
 template <typename OT>
@@ -80,17 +88,45 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const OT* __restrict_
         for (int i = 0; i < V; ++i) acc[i] = fmaf(sw[j], v[i], acc[i]);
       }
     } else {
-      for (int j = 0; j < k; ++j) {
-        float v[V];
-        Vec<OT>::load(o + (size_t)srow[j] * H + V * c, v);
-        for (int sp = 1; sp < nsplit; ++sp) {  // K-split partial slabs of the down GEMM, in slab order
-          float p[V];
-          Vec<OT>::load(o + sp * split_stride + (size_t)srow[j] * H + V * c, p);
+      // K-split partial slabs of the down GEMM: for 8 rows at a time, slab 0
+      // and then the other slabs two at a time are loaded together; each
+      // row's slabs are summed in slab order, then the slot-order sum
+      int j = 0;
+      for (; j < k; j += 8) {
+        const int nq = k - j < 8 ? k - j : 8;
+        float v[8][V];
 #pragma unroll
-          for (int i = 0; i < V; ++i) v[i] += p[i];
+        for (int q = 0; q < 8; ++q) Vec<OT>::load_if(q < nq, o + (size_t)srow[j + q % nq] * H + V * c, v[q]);
+        int sp = 1;
+        for (; sp + 2 <= nsplit; sp += 2) {
+          float p[2][8][V];
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              Vec<OT>::load_if(q < nq, o + (sp + u) * split_stride + (size_t)srow[j + q % nq] * H + V * c, p[u][q]);
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+#pragma unroll
+              for (int i = 0; i < V; ++i) v[q][i] += p[u][q][i];
+        }
+        if (sp < nsplit) {
+          float p[8][V];
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            Vec<OT>::load_if(q < nq, o + sp * split_stride + (size_t)srow[j + q % nq] * H + V * c, p[q]);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+#pragma unroll
+            for (int i = 0; i < V; ++i) v[q][i] += p[q][i];
         }
 #pragma unroll
-        for (int i = 0; i < V; ++i) acc[i] = fmaf(sw[j], v[i], acc[i]);
+        for (int q = 0; q < 8; ++q)
+          if (q < nq)
+#pragma unroll
+            for (int i = 0; i < V; ++i) acc[i] = fmaf(sw[j + q], v[q][i], acc[i]);
       }
     }
     if (shared) {
@@ -130,7 +166,18 @@ __global__ void __launch_bounds__(kThreads) swiglu_reduce_kernel(const float* __
     const float* row = p + (size_t)r * 2 * I;
     float4 g = reinterpret_cast<const float4*>(row)[c];
     float4 u = reinterpret_cast<const float4*>(row + I)[c];
-    for (int sp = 1; sp < nsplit; ++sp) {
+    int sp = 1;
+    for (; sp + 2 <= nsplit; sp += 2) {  // two slabs' loads in flight together, added in slab order
+      const float4 g2 = reinterpret_cast<const float4*>(row + sp * split_stride)[c];
+      const float4 u2 = reinterpret_cast<const float4*>(row + sp * split_stride + I)[c];
+      const float4 g3 = reinterpret_cast<const float4*>(row + (sp + 1) * split_stride)[c];
+      const float4 u3 = reinterpret_cast<const float4*>(row + (sp + 1) * split_stride + I)[c];
+      g.x += g2.x; g.y += g2.y; g.z += g2.z; g.w += g2.w;
+      u.x += u2.x; u.y += u2.y; u.z += u2.z; u.w += u2.w;
+      g.x += g3.x; g.y += g3.y; g.z += g3.z; g.w += g3.w;
+      u.x += u3.x; u.y += u3.y; u.z += u3.z; u.w += u3.w;
+    }
+    if (sp < nsplit) {
       const float4 g2 = reinterpret_cast<const float4*>(row + sp * split_stride)[c];
       const float4 u2 = reinterpret_cast<const float4*>(row + sp * split_stride + I)[c];
       g.x += g2.x; g.y += g2.y; g.z += g2.z; g.w += g2.w;
@@ -150,8 +197,10 @@ __global__ void __launch_bounds__(kThreads) swiglu_reduce_kernel(const float* __
 cudaError_t launch_swiglu_reduce(const float* partials, int nsplit, size_t split_stride, int rows, int I, uint16_t* h,
                                  cudaStream_t s) {
   const long long n = (long long)rows * (I / 4);
-  const int blocks = (int)((n + kThreads - 1) / kThreads < 4096 ? (n + kThreads - 1) / kThreads : 4096);
-  return launch_kernel(swiglu_reduce_kernel, dim3(blocks), dim3(kThreads), 0, s, partials, nsplit, split_stride,
+  int threads = kThreads;  // few rows: smaller blocks so more SMs share the loads
+  while (threads > 64 && (n + threads - 1) / threads < 148) threads >>= 1;
+  const int blocks = (int)((n + threads - 1) / threads < 4096 ? (n + threads - 1) / threads : 4096);
+  return launch_kernel(swiglu_reduce_kernel, dim3(blocks), dim3(threads), 0, s, partials, nsplit, split_stride,
                        rows, I, reinterpret_cast<__nv_bfloat16*>(h));
 }
 
@@ -162,15 +211,19 @@ cudaError_t launch_combine_t(const OT* o, const float* topk_w, const int32_t* in
                              int H, int k, int rows, int nsplit, size_t split_stride, uint16_t* y, DevStatus* st,
                              cudaStream_t s) {
   if (k > 64) return cudaErrorInvalidValue;
-  // Few tokens: split each row over several blocks so every SM has work;
-  // many tokens: one block per token, each thread looping over its vectors.
-  const int slices_max = (H / Vec<OT>::V + kThreads - 1) / kThreads;
+  // Few tokens: split each row over several blocks so every SM has work
+  // (down to 64 threads per block); many tokens: one block per token, each
+  // thread looping over its vectors.
+  const int HV = H / Vec<OT>::V;
+  int threads = kThreads;
+  while (threads > 64 && (long long)T * ((HV + threads - 1) / threads) < 148) threads >>= 1;
+  const int slices_max = (HV + threads - 1) / threads;
   int slices = (2 * 148 + T - 1) / T;
   slices = slices < 1 ? 1 : (slices > slices_max ? slices_max : slices);
   for (int t0 = 0; t0 < T; t0 += 65535) {  // grid.y limit
     const dim3 grid(slices, T - t0 < 65535 ? T - t0 : 65535);
     const cudaError_t err =
-        launch_kernel(combine_kernel<OT>, grid, dim3(kThreads), 0, s, o, topk_w, inv_perm, shared, H, k, rows, nsplit,
+        launch_kernel(combine_kernel<OT>, grid, dim3(threads), 0, s, o, topk_w, inv_perm, shared, H, k, rows, nsplit,
                       split_stride, reinterpret_cast<__nv_bfloat16*>(y), st, t0);
     if (err != cudaSuccess) return err;
   }

@@ -265,7 +265,26 @@ __device__ __forceinline__ void router_select(const float* partial, int hs, cons
   float v[EPL];
 #pragma unroll
   for (int i = 0; i < EPL; ++i) v[i] = 0.f;
-  for (int sp = 0; sp < hs; ++sp) {
+  // G slabs loaded together, then added in slab order
+  constexpr int G = EPL <= 8 ? 4 : (EPL <= 16 ? 2 : 1);
+  int sp = 0;
+  for (; sp + G <= hs; sp += G) {
+    float p[G][EPL];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float* slab = partial + ((size_t)(sp + g) * T + t) * E;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        p[g][i] = e < E ? __ldcg(slab + e) : 0.f;
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) v[i] += p[g][i];
+  }
+  for (; sp < hs; ++sp) {
     const float* slab = partial + ((size_t)sp * T + t) * E;
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
