@@ -101,9 +101,10 @@ enum {
 
 /* Router scoring: how the k experts of a token are selected and weighted
  * from its fp32 logits l[e] and the optional per-expert bias b[e].  The
- * Qwen 3.5-397B-on-Ironwood page ("key optimisations", expert load
- * balancing) names hot experts and a router balancing term, and the Ling
- * page a per-expert router bias, without a formula; SOFTMAX is the rule of
+ * systems-engineering handbook page on Qwen 3.5-397B MoE on Ironwood
+ * ("key optimisations", step 1 "expert load balancing") names hot experts
+ * and a balancing term in the router, and the Ling page a per-expert
+ * router bias, neither with a formula; SOFTMAX is the rule of
  * the layer's workloads, the other two are the common forms in which the
  * bias steers only the selection.  In every form the k selected are listed
  * by descending key, ties to the lower expert id. */

@@ -33,10 +33,10 @@ What it computes (plain definitions, in the order the layer applies them):
    Ling page, introduction).
 
 Router scoring variants (steps 1-3 replaced; everything after is unchanged).
-The Qwen-3.5-397B-on-Ironwood page ("key optimisations", step 1, expert load
-balancing) names hot experts and a balancing term in the router but gives no
-formula, and the Ling page says only that router logits get a per-expert
-bias.  Besides the rule above (bias added to the logits, so it moves both
+The systems-engineering handbook page on Qwen 3.5-397B MoE on Ironwood
+("key optimisations", step 1 "expert load balancing") names hot experts and
+a balancing term in the router but gives no formula, and the Ling page says
+only that router logits get a per-expert bias.  Besides the rule above (bias added to the logits, so it moves both
 selection and weights: scoring "softmax"), two plain forms in which a
 per-expert bias b steers only which experts are picked are supported:
 
