@@ -34,12 +34,13 @@ import numpy as np
 __all__ = [
     "Config", "CONFIGS", "TID", "bf16_from_f32", "normal_bf16", "normal_f32",
     "uniform_bf16", "Inputs", "make_inputs", "zipf_bias", "redraw_x_rows",
-    "fill_expert_weights",
+    "fill_expert_weights", "fp8_e4m3_codes", "e8m0_scale_codes", "mx_expert_weights", "MX_BLOCK",
 ]
 
 # Tensor ids: the second word of every counter key.
 TID = dict(x=1, w_router=2, w_gate_up=3, w_down=4, w_sh_gate_up=5, w_sh_down=6,
-           x_redraw=7, h_stage=8, topk_w_stage=9, misc=10)
+           x_redraw=7, h_stage=8, topk_w_stage=9, misc=10,
+           mx_gate_up=11, mx_down=12, mx_gate_up_scale=13, mx_down_scale=14)
 
 
 @dataclass(frozen=True)
@@ -193,6 +194,45 @@ def fill_expert_weights(cfg: Config, which: str, out: np.ndarray, experts=None,
 
     with ThreadPoolExecutor(threads) as ex:
         list(ex.map(one, experts))
+
+
+# ---------------------------------------------------------------- block-scaled fp8 weights
+# Codes only: random bit fields, no quantisation of any real-valued tensor.
+MX_BLOCK = 32  # weights along the reduction dimension that share one scale
+
+
+def fp8_e4m3_codes(seed: int, tid: int, idx: int, shape, exp_lo: int = 3, exp_hi: int = 9) -> np.ndarray:
+    """Random FP8 E4M3 bytes: sign bit uniform, exponent field uniform in
+    [exp_lo, exp_hi], mantissa field uniform in [0, 7]; exp_hi <= 14 keeps
+    every code finite."""
+    if not 0 <= exp_lo <= exp_hi <= 14:
+        raise ValueError("exponent field range must lie in [0, 14]")
+    g = _gen(seed, tid, idx)
+    n = int(np.prod(shape))
+    sign = g.integers(0, 2, n, dtype=np.uint8)
+    expo = g.integers(exp_lo, exp_hi + 1, n, dtype=np.uint8)
+    mant = g.integers(0, 8, n, dtype=np.uint8)
+    return ((sign << 7) | (expo << 3) | mant).astype(np.uint8).reshape(shape)
+
+
+def e8m0_scale_codes(seed: int, tid: int, idx: int, shape, lo: int = 118, hi: int = 122) -> np.ndarray:
+    """Random E8M0 scale bytes (power-of-two exponents, bias 127), uniform in [lo, hi]."""
+    if not 0 <= lo <= hi <= 254:
+        raise ValueError("scale codes must lie in [0, 254]")
+    return _gen(seed, tid, idx).integers(lo, hi + 1, int(np.prod(shape)), dtype=np.uint8).reshape(shape)
+
+
+def mx_expert_weights(cfg: Config, e: int, which: str) -> tuple[np.ndarray, np.ndarray]:
+    """One expert's block-scaled fp8 weights: codes [K, N] uint8 and scale codes
+    [K / MX_BLOCK, N] uint8, K the reduction dimension (gate_up: K = H,
+    N = 2I; down: K = I, N = H).  Magnitudes come out near the bf16 weights'
+    (exponent fields 3..9 times scales 2^-9..2^-5)."""
+    K, N = {"gate_up": (cfg.H, 2 * cfg.I), "down": (cfg.I, cfg.H)}[which]
+    if K % MX_BLOCK:
+        raise ValueError("reduction dimension must be a multiple of the scale block")
+    codes = fp8_e4m3_codes(cfg.seed, TID["mx_" + which], e, (K, N))
+    scales = e8m0_scale_codes(cfg.seed, TID["mx_" + which + "_scale"], e, (K // MX_BLOCK, N))
+    return codes, scales
 
 
 @dataclass
