@@ -128,3 +128,72 @@ def test_fp8_code_generator_is_finite_keyed_and_in_range():
         synth.fp8_e4m3_codes(0, 11, 5, (4,), exp_hi=15)
     s = synth.e8m0_scale_codes(0, 13, 0, (8, 8))
     assert s.min() >= 118 and s.max() <= 122
+
+
+# ---------------------------------------------------------------- quantisation (E4M3 encode, MX blocks)
+
+def test_e4m3_encode_round_trips_every_finite_code():
+    codes = np.arange(256, dtype=np.uint8)
+    vals = mx.e4m3_to_f64(codes)
+    ok = ~np.isnan(vals)
+    np.testing.assert_array_equal(mx.e4m3_encode(vals[ok]), codes[ok])   # -0 keeps its sign bit
+    with pytest.raises(ValueError):
+        mx.e4m3_encode(np.array([np.nan]))
+
+
+def test_e4m3_encode_ties_and_saturation_worked_by_hand():
+    cases = {
+        1.0625: 0x38,           # halfway 1.0 | 1.125 -> even mantissa 000
+        1.1875: 0x3A,           # halfway 1.125 | 1.25 -> even mantissa 010
+        2.0 ** -10: 0x00,       # halfway 0 | 2^-9 -> 0
+        3 * 2.0 ** -11: 0x01,   # 0.75 * 2^-9 -> 2^-9
+        15 * 2.0 ** -10: 0x08,  # halfway 7*2^-9 | 2^-6 -> the smallest normal (even)
+        440.0: 0x7E,            # nearest is 448
+        470.0: 0x7E,            # above 448: clamped
+        1e6: 0x7E,
+        -500.0: 0xFE,
+        -3.3: 0xC5,             # 1 1000 101 = -3.25
+    }
+    got = mx.e4m3_encode(np.array(list(cases)))
+    assert [hex(c) for c in got] == [hex(c) for c in cases.values()]
+
+
+def test_e4m3_encode_matches_torch_below_its_overflow():
+    """PyTorch's float8_e4m3fn cast rounds to nearest-even too; it turns
+    magnitudes from 464 up into NaN, where the MX rule clamps, so the
+    comparison stays below 464."""
+    rng = np.random.default_rng(41)
+    v = rng.uniform(-463.9, 463.9, 200_000) * np.exp2(rng.integers(-16, 1, 200_000))
+    v = v.astype(np.float32)
+    want = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(mx.e4m3_encode(v.astype(np.float64)), want)
+
+
+def test_mx_quantize_scale_rule():
+    v = np.zeros((96, 4))
+    v[:32, 0] = np.linspace(-1.0, 1.0, 32)           # amax 1: floor(log2 1) - 8 = -8
+    v[32:64, 1] = 448.0 * 4 * np.sign(np.arange(32) - 15.5)   # amax 448 * 2^2: exact
+    v[64:, 2] = 500.0                                # amax 500: shared exponent 0, 500 clamps to 448
+    codes, scales = mx.mx_quantize(v)
+    assert scales[0, 0] == 127 - 8 and scales[1, 1] == 127 + 2 and scales[2, 2] == 127
+    assert scales[1, 0] == 0 and scales[0, 3] == 0     # all-zero blocks take the smallest scale
+    deq = mx.mx_dequant(codes, scales)
+    np.testing.assert_array_equal(deq[32:64, 1], v[32:64, 1])
+    assert np.all(deq[64:, 2] == 448.0)
+    assert np.all(deq[:, 3] == 0.0) and np.all(codes[:, 3] == 0)
+
+
+def test_mx_quantize_error_bound():
+    """Three mantissa bits: relative error <= 2^-4 in the normal range, and
+    absolute error <= half a subnormal step (2^-10 of the scale) below it."""
+    rng = np.random.default_rng(42)
+    v = rng.standard_normal((256, 16)) * np.exp2(rng.integers(-20, 20, (8, 1, 16))).repeat(32, axis=0).reshape(256, 16)
+    codes, scales = mx.mx_quantize(v)
+    deq = mx.mx_dequant(codes, scales)
+    X = np.repeat(mx.e8m0_to_f64(scales), 32, axis=0)
+    p = np.abs(v) / X
+    normal = (p >= 2.0 ** -6) & (p <= 448.0)
+    assert np.all(np.abs(deq - v)[normal] <= 2.0 ** -4 * np.abs(v)[normal])
+    sub = p < 2.0 ** -6
+    assert np.all(np.abs(deq - v)[sub] <= 2.0 ** -10 * X[sub])
+    assert np.all(p <= 512.0)                          # the largest element of a block scales into [256, 512)
