@@ -105,16 +105,51 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _need(t, dtype, name, ndim=None):
+def _dims(t, ndim, name):
+    """The shape of a tensor argument after checking its rank."""
     import torch
-    if not isinstance(t, torch.Tensor) or not t.is_cuda:
-        raise TypeError(f"{name} must be a CUDA tensor")
-    if t.dtype != dtype:
-        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
-    if not t.is_contiguous():
-        raise ValueError(f"{name} must be contiguous")
-    if ndim is not None and t.dim() != ndim:
-        raise ValueError(f"{name} must have {ndim} dims")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+    return tuple(t.shape)
+
+
+def _check_args(specs, ws=None):
+    """Checks every tensor argument before anything reaches the library: the
+    library sees raw pointers and sizes only, so a tensor of the wrong shape,
+    dtype or device would be read or written out of bounds.  specs: (tensor
+    or None, dtype, name, shape with None for any size).  All shapes and
+    dtypes are checked first, then that every tensor (and the workspace ws)
+    is a CUDA tensor on one device."""
+    import torch
+    live = []
+    for t, dtype, name, shape in specs:
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor")
+        if t.dtype != dtype:
+            raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+        if shape is not None:
+            if t.dim() != len(shape) or any(w is not None and w != g for w, g in zip(shape, t.shape)):
+                want = "[" + ", ".join("*" if w is None else str(w) for w in shape) + "]"
+                raise ValueError(f"{name} must have shape {want}, got {list(t.shape)}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        live.append((t, name))
+    if ws is not None:
+        if not isinstance(ws, torch.Tensor) or ws.dtype != torch.uint8 or ws.dim() != 1 or not ws.is_contiguous():
+            raise TypeError("the workspace must be a contiguous 1-D uint8 tensor (alloc_workspace)")
+        live.append((ws, "workspace"))
+    device = None
+    for t, name in live:
+        if not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA tensor")
+        if device is None:
+            device = t.device
+        elif t.device != device:
+            raise ValueError(f"{name} is on {t.device}, the other arguments on {device}")
 
 
 def workspace_layout(T, H, E, I, k, I_s=0) -> dict:
@@ -138,26 +173,29 @@ def alloc_workspace(T, H, E, I, k, I_s=0, device="cuda"):
 
 
 def device_status(ws) -> int:
+    _check_args([], ws)
     out = ctypes.c_int32()
     _check(lib().moe_get_device_status(_ptr(ws), _stream(), ctypes.byref(out)), "moe_get_device_status")
     return out.value
 
 
 def clear_device_status(ws) -> None:
+    _check_args([], ws)
     _check(lib().moe_clear_device_status(_ptr(ws), _stream()), "moe_clear_device_status")
 
 
 def route(x, w_router, bias, k, ws, impl=ROUTER_AUTO, out=None, scoring=SCORE_SOFTMAX):
     """topk_ids [T,k] int32, topk_w [T,k] float32 (scoring: SCORE_*)."""
     import torch
-    _need(x, torch.bfloat16, "x", 2)
-    _need(w_router, torch.float32, "w_router", 2)
-    if bias is not None:
-        _need(bias, torch.float32, "bias", 1)
-    T, H = x.shape
-    E = w_router.shape[1]
-    ids, w = out if out is not None else (
-        torch.empty(T, k, dtype=torch.int32, device=x.device), torch.empty(T, k, dtype=torch.float32, device=x.device))
+    T, H = _dims(x, 2, "x")
+    E = _dims(w_router, 2, "w_router")[1]
+    ids, w = out if out is not None else (None, None)
+    _check_args([(x, torch.bfloat16, "x", (T, H)), (w_router, torch.float32, "w_router", (H, E)),
+                 (bias, torch.float32, "bias", (E,)), (ids, torch.int32, "topk_ids", (T, k)),
+                 (w, torch.float32, "topk_w", (T, k))], ws)
+    if out is None:
+        ids = torch.empty(T, k, dtype=torch.int32, device=x.device)
+        w = torch.empty(T, k, dtype=torch.float32, device=x.device)
     _check(lib().moe_route_scored(_ptr(x), _ptr(w_router), _ptr(bias), T, H, E, k, scoring, _ptr(ids), _ptr(w),
                                   impl, _ptr(ws), ws.numel(), _stream()), "moe_route")
     return ids, w
@@ -166,8 +204,8 @@ def route(x, w_router, bias, k, ws, impl=ROUTER_AUTO, out=None, scoring=SCORE_SO
 def permute(topk_ids, E, ws):
     """counts [E], offsets [E+1], sorted_token_ids [T*k], inv_perm [T,k] (int32)."""
     import torch
-    _need(topk_ids, torch.int32, "topk_ids", 2)
-    T, k = topk_ids.shape
+    T, k = _dims(topk_ids, 2, "topk_ids")
+    _check_args([(topk_ids, torch.int32, "topk_ids", (T, k))], ws)
     dev = topk_ids.device
     counts = torch.empty(E, dtype=torch.int32, device=dev)
     offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
@@ -181,13 +219,15 @@ def permute(topk_ids, E, ws):
 def grouped_swiglu(x, w_gate_up, offsets, sorted_token_ids, k, ws, tiles=TILES_AUTO, out=None):
     """h [T*k, I] bf16 in permuted order."""
     import torch
-    _need(x, torch.bfloat16, "x", 2)
-    _need(w_gate_up, torch.bfloat16, "w_gate_up", 3)
-    _need(offsets, torch.int32, "offsets", 1)
-    _need(sorted_token_ids, torch.int32, "sorted_token_ids", 1)
-    T, H = x.shape
-    E, _, I2 = w_gate_up.shape
+    T, H = _dims(x, 2, "x")
+    E, _, I2 = _dims(w_gate_up, 3, "w_gate_up")
     I = I2 // 2
+    _check_args([(x, torch.bfloat16, "x", (T, H)), (w_gate_up, torch.bfloat16, "w_gate_up", (E, H, 2 * I)),
+                 (offsets, torch.int32, "offsets", (E + 1,)),
+                 (sorted_token_ids, torch.int32, "sorted_token_ids", (T * k,)),
+                 (out, torch.bfloat16, "out", (T * k, I))], ws)
+    if offsets is None or sorted_token_ids is None:
+        raise TypeError("offsets and sorted_token_ids are required")
     h = out if out is not None else torch.empty(T * k, I, dtype=torch.bfloat16, device=x.device)
     _check(lib().moe_grouped_swiglu(_ptr(x), _ptr(w_gate_up), _ptr(offsets), _ptr(sorted_token_ids), T, H, E, I, k,
                                     tiles, _ptr(h), _ptr(ws), ws.numel(), _stream()), "moe_grouped_swiglu")
@@ -197,10 +237,10 @@ def grouped_swiglu(x, w_gate_up, offsets, sorted_token_ids, k, ws, tiles=TILES_A
 def grouped_down(h, w_down, offsets, ws, tiles=TILES_AUTO, out=None):
     """o [rows, H] float32 = h . W_down[e] per group (offsets None: one group)."""
     import torch
-    _need(h, torch.bfloat16, "h", 2)
-    _need(w_down, torch.bfloat16, "w_down", 3)
-    rows, I = h.shape
-    E, _, H = w_down.shape
+    rows, I = _dims(h, 2, "h")
+    E, _, H = _dims(w_down, 3, "w_down")
+    _check_args([(h, torch.bfloat16, "h", (rows, I)), (w_down, torch.bfloat16, "w_down", (E, I, H)),
+                 (offsets, torch.int32, "offsets", (E + 1,)), (out, torch.float32, "out", (rows, H))], ws)
     o = out if out is not None else torch.empty(rows, H, dtype=torch.float32, device=h.device)
     _check(lib().moe_grouped_down(_ptr(h), _ptr(w_down), _ptr(offsets), rows, H, E, I, tiles, _ptr(o),
                                   _ptr(ws), ws.numel(), _stream()), "moe_grouped_down")
@@ -210,14 +250,14 @@ def grouped_down(h, w_down, offsets, ws, tiles=TILES_AUTO, out=None):
 def down_combine(h, w_down, topk_w, inv_perm, offsets, shared_out, ws, tiles=TILES_AUTO, out=None):
     """y [T,H] bf16."""
     import torch
-    _need(h, torch.bfloat16, "h", 2)
-    _need(w_down, torch.bfloat16, "w_down", 3)
-    _need(topk_w, torch.float32, "topk_w", 2)
-    _need(inv_perm, torch.int32, "inv_perm", 2)
-    if shared_out is not None:
-        _need(shared_out, torch.float32, "shared_out", 2)
-    T, k = topk_w.shape
-    E, I, H = w_down.shape
+    T, k = _dims(topk_w, 2, "topk_w")
+    E, I, H = _dims(w_down, 3, "w_down")
+    _check_args([(h, torch.bfloat16, "h", (T * k, I)), (w_down, torch.bfloat16, "w_down", (E, I, H)),
+                 (topk_w, torch.float32, "topk_w", (T, k)), (inv_perm, torch.int32, "inv_perm", (T, k)),
+                 (offsets, torch.int32, "offsets", (E + 1,)), (shared_out, torch.float32, "shared_out", (T, H)),
+                 (out, torch.bfloat16, "out", (T, H))], ws)
+    if h is None or inv_perm is None or offsets is None:
+        raise TypeError("h, inv_perm and offsets are required")
     y = out if out is not None else torch.empty(T, H, dtype=torch.bfloat16, device=h.device)
     _check(lib().moe_down_combine(_ptr(h), _ptr(w_down), _ptr(topk_w), _ptr(inv_perm), _ptr(offsets),
                                   _ptr(shared_out), T, H, E, I, k, tiles, _ptr(y), _ptr(ws), ws.numel(),
@@ -234,18 +274,22 @@ def forward(x, w_router, bias, w_gate_up, w_down, k, ws, w_sh_gate_up=None, w_sh
     boundaries (see include/moe.h); info: optional dict that receives the
     number of kernels enqueued under "launches"."""
     import torch
-    _need(x, torch.bfloat16, "x", 2)
-    _need(w_router, torch.float32, "w_router", 2)
-    _need(w_gate_up, torch.bfloat16, "w_gate_up", 3)
-    _need(w_down, torch.bfloat16, "w_down", 3)
-    T, H = x.shape
-    E, _, I2 = w_gate_up.shape
+    T, H = _dims(x, 2, "x")
+    E, _, I2 = _dims(w_gate_up, 3, "w_gate_up")
     I = I2 // 2
     I_s = 0
+    if (w_sh_gate_up is None) != (w_sh_down is None):
+        raise TypeError("the shared expert needs both w_sh_gate_up and w_sh_down")
     if w_sh_gate_up is not None:
-        _need(w_sh_gate_up, torch.bfloat16, "w_sh_gate_up", 2)
-        _need(w_sh_down, torch.bfloat16, "w_sh_down", 2)
-        I_s = w_sh_gate_up.shape[1] // 2
+        I_s = _dims(w_sh_gate_up, 2, "w_sh_gate_up")[1] // 2
+    E_r = _dims(w_router, 2, "w_router")[1]
+    if E_r != E:
+        raise ValueError(f"w_router has {E_r} experts, w_gate_up {E}")
+    _check_args([(x, torch.bfloat16, "x", (T, H)), (w_router, torch.float32, "w_router", (H, E)),
+                 (bias, torch.float32, "bias", (E,)), (w_gate_up, torch.bfloat16, "w_gate_up", (E, H, 2 * I)),
+                 (w_down, torch.bfloat16, "w_down", (E, I, H)),
+                 (w_sh_gate_up, torch.bfloat16, "w_sh_gate_up", (H, 2 * I_s)),
+                 (w_sh_down, torch.bfloat16, "w_sh_down", (I_s, H)), (out, torch.bfloat16, "out", (T, H))], ws)
     y = out if out is not None else torch.empty(T, H, dtype=torch.bfloat16, device=x.device)
     opt = _Options(tiles, router)
     opt.scoring = scoring
@@ -262,6 +306,7 @@ def forward(x, w_router, bias, w_gate_up, w_down, k, ws, w_sh_gate_up=None, w_sh
 
 
 def selftest_timeout(ws, timeout_ns: int) -> None:
+    _check_args([], ws)
     _check(lib().moe_selftest_timeout(_ptr(ws), ws.numel(), timeout_ns, _stream()), "moe_selftest_timeout")
 
 
