@@ -1,4 +1,4 @@
-// route.cu -- router of the MoE layer: fp32 logits, softmax, top-k, renormalise.
+// route.cu -- router of the MoE layer: fp32 logits, scoring, top-k, weights.
 //
 // The pages put routing first on the MoE path and plan to fuse the gating
 // projection with the top-k selection (Qwen 3.5-397B-on-Ironwood page,
@@ -18,7 +18,10 @@
 // k rounds of a warp arg-max by shuffles (larger logit first, ties to the
 // lower expert id); then w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0) over the
 // k selected logits, which equals softmax-then-renormalise because the full
-// softmax denominator cancels.
+// softmax denominator cancels.  Two further scoring rules (MOE_SCORE_*)
+// select on l + b or sigmoid(l) + b and weight by the unbiased logits or
+// sigmoid scores of the selected experts (route_dev.cuh); the softmax rule
+// keeps its own kernel instantiation.
 #include "route_dev.cuh"
 
 namespace moe {
