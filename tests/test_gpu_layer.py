@@ -2,8 +2,10 @@
 at sizes the oracle finishes in seconds: several tiles per expert, ragged
 per-expert row counts, empty experts, one token, k = E, a shared expert,
 experts with more rows than one tile pass, every tile policy, every router
-implementation and the K-split of the expert GEMMs for a few tokens.  Routing (ids, counts, offsets, permutation) must
-match bit for bit; floating-point outputs within the layer's tolerance."""
+implementation, the K-split of the expert GEMMs for a few tokens, E not a
+multiple of 4, the largest k (64) and k = 1.  Routing (ids, counts, offsets,
+permutation) must match bit for bit; floating-point outputs within the
+layer's tolerance."""
 import numpy as np
 import pytest
 
@@ -33,6 +35,11 @@ CASES = {
         Config("few_bias", T=7, H=1024, E=128, I=256, k=6, bias="zipf:1.2"),  # biased few-token routing
         # the one-launch layer: shared expert, biased routing, experts chosen by several tokens
         Config("fused_shared", T=4, H=512, E=16, I=256, k=4, I_s=256, bias="zipf:1.2"),
+        # edge cases: E % 4 != 0 above 128 experts (scalar 8-per-lane top-k), the largest k
+        # (k = E = 64: every token takes every expert), and k = 1 (every weight exactly 1)
+        Config("odd_e130", T=40, H=256, E=130, I=128, k=5),
+        Config("k64", T=8, H=2048, E=64, I=128, k=64),
+        Config("top1", T=50, H=256, E=8, I=128, k=1),
     ]
 }
 
