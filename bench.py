@@ -230,6 +230,9 @@ def recorded_traffic(workload):
 
 # ---------------------------------------------------------------- timed runs
 TILES = {"auto": 0, "small": 1, "large": 2, "pair": 3, "fused": 4}
+# further workloads timed with the default workload, reported under "extra" (their weights
+# replace the decode ones after the decode and prefill measurements)
+DEFAULT_EXTRA = "ling_skewed_t4096,sweep_decode_t1,sweep_decode_t4,sweep_decode_t16,sweep_decode_t64"
 # router scoring rules (an extra workload "name:rule" is timed under that rule)
 SCORING = {"softmax": 0, "softmax_select_bias": 1, "sigmoid": 2}
 
@@ -572,11 +575,14 @@ def main():
     ap.add_argument("--cpu-sample-tokens", type=int, default=16)
     ap.add_argument("--ref-sample-tokens", type=int, default=2)
     ap.add_argument("--tiles", choices=sorted(TILES), default="auto", help="grouped GEMM tile policy (tuning)")
-    ap.add_argument("--extra", default="", help="comma-separated further workloads to time, e.g. "
-                                                 "ling_skewed_t4096,sweep_decode_t1; name:sigmoid or "
-                                                 "name:softmax_select_bias times it under that router "
-                                                 "scoring rule")
+    ap.add_argument("--extra", default=None,
+                    help="comma-separated further workloads to time (default with the default workload: the "
+                         "Ling-like skewed prefill and the small-batch decode sweep; otherwise none); "
+                         "name:sigmoid or name:softmax_select_bias times it under that router scoring rule; "
+                         "'' for none")
     args = ap.parse_args()
+    if args.extra is None:
+        args.extra = DEFAULT_EXTRA if args.workload == ap.get_default("workload") else ""
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
