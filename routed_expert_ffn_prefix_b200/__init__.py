@@ -12,7 +12,6 @@ from __future__ import annotations
 
 import ctypes
 import os
-from dataclasses import dataclass
 
 from . import build as _build
 
