@@ -36,6 +36,13 @@
  *     patterns.  The library never allocates, frees or keeps a pointer
  *     past the call; work is enqueued on `stream` (a cudaStream_t; NULL is
  *     the legacy default stream) and the call returns without waiting.
+ *   - Process-wide state: the library keeps two host-side caches, both pure
+ *     functions of their keys and guarded by a mutex, so every call stays
+ *     re-entrant: kernel attributes and cluster occupancy per device, and
+ *     the last 16 TMA tensor descriptors keyed by (weight address,
+ *     extents).  A cached descriptor is rebuilt whenever the key differs;
+ *     it holds an address value but the library never dereferences it
+ *     outside a call that passes the same pointer again.
  *   - Shapes: T >= 1 tokens, H % 256 == 0, I % 128 == 0 (I_s likewise),
  *     1 <= k <= min(E, 64), E <= 1024, T*k < 2^31.
  *   - Alignment: every pointer 16-byte aligned (workspace 256-byte).
@@ -191,17 +198,23 @@ moe_status_t moe_permute(const int32_t *topk_ids, int T, int E, int k,
  * forbids allocation afterwards, a plugin inside a framework that owns every
  * device allocation, or code that must avoid the device-wide
  * synchronisation cudaMalloc/cudaFree can cause.  The outputs are identical
- * to moe_permute's.  The kernels' scratch lives in a 2 MiB array built into
- * the library, which every GPU that loads the library holds until the
+ * to moe_permute's.  The kernels' scratch lives in a 512 KiB array built
+ * into the library, which every GPU that loads the library holds until the
  * process exits; the call itself allocates and frees nothing.
- * Limits: T*k <= 131072 and E <= 1024 (larger sizes return
- * MOE_ERR_WORKSPACE and enqueue nothing).
- * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Limits: T*k <= 131072 (larger batches return MOE_ERR_WORKSPACE and enqueue
+ * nothing); E <= 1024 and k <= min(E, 64) as for every call (else
+ * MOE_ERR_INVALID_ARG).
+ * The first call from each device's context looks up the array's device
+ * address (cudaGetSymbolAddress); make that first call before any stream
+ * capture.  A device reset gives the device a new context, and the next
+ * call looks the address up again.
  * All calls share the one array: calls that overlap on the GPU (other
  * streams, other host threads) race and must be serialised by the caller.
- * No device status word is kept: an id outside [0,E) is skipped, so
- * offsets[E] then falls short of T*k. */
+ * No device status word is kept: a slot whose id lies outside [0,E) is
+ * skipped -- it is counted nowhere, no row is assigned to it and its
+ * inv_perm entry is left unwritten (it keeps whatever the caller's buffer
+ * held) -- so offsets[E] then falls short of T*k.  Check offsets[E] == T*k
+ * before passing the outputs to the expert GEMMs or the combine. */
 moe_status_t moe_permute_noalloc(const int32_t *topk_ids, int T, int E, int k,
                                  int32_t *counts, int32_t *offsets,
                                  int32_t *sorted_token_ids, int32_t *inv_perm, void *stream);

@@ -8,6 +8,7 @@ from __future__ import annotations
 
 import concurrent.futures
 import glob
+import hashlib
 import os
 import shutil
 import subprocess
@@ -20,6 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_NAME = "libmoe_b200.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
+HASH_PATH = LIB_PATH + ".srchash"  # source hash the library was built from
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE]
@@ -41,17 +43,33 @@ def _deps() -> list[str]:
         glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
+def source_hash() -> str:
+    """SHA-256 over the compiler flags and the name and bytes of every source
+    and header the library is built from."""
+    h = hashlib.sha256()
+    h.update(" ".join(ARCH_FLAGS + COMMON_FLAGS[:-1]).encode())
+    for d in sorted(_deps()):
+        h.update(os.path.relpath(d, ROOT).encode() + b"\0")
+        with open(d, "rb") as f:
+            h.update(f.read())
+        h.update(b"\0")
+    return h.hexdigest()
+
+
 def up_to_date() -> bool:
-    if not os.path.exists(LIB_PATH):
+    """True when the library exists and was built from exactly the current
+    sources (the hash recorded beside it matches); file times are not used."""
+    if not os.path.exists(LIB_PATH) or not os.path.exists(HASH_PATH):
         return False
-    t = os.path.getmtime(LIB_PATH)
-    return all(os.path.getmtime(d) <= t for d in _deps())
+    with open(HASH_PATH) as f:
+        return f.read().strip() == source_hash()
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
     """Compile (if needed) and return the library path."""
     if not force and up_to_date():
         return LIB_PATH
+    digest = source_hash()
     os.makedirs(BUILD_DIR, exist_ok=True)
     cc = nvcc()
 
@@ -73,6 +91,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     os.replace(tmp, LIB_PATH)
+    with open(HASH_PATH, "w") as f:
+        f.write(digest + "\n")
     return LIB_PATH
 
 

@@ -9,7 +9,6 @@ using namespace moe;
 namespace {
 
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded device wait
-constexpr int kMaxK = 64;
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 

@@ -12,6 +12,8 @@
 namespace moe {
 
 constexpr int kMaxExperts = 1024;
+constexpr int kMaxK = 64;          // largest top-k any entry point accepts
+constexpr int kPermuteChunk = 1024; // slots per block of the multi-block permutation (histogram rows)
 constexpr int kMaxDevices = 64;
 
 // Runs `setup` once per (call site, device): kernel attributes and occupancy

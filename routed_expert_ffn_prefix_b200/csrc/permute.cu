@@ -30,7 +30,7 @@ namespace moe {
 
 namespace {
 
-constexpr int kChunk = 1024;  // slots per block (hist/scatter)
+constexpr int kChunk = kPermuteChunk;  // slots per block (hist/scatter)
 constexpr int kScatterWarps = 4;
 constexpr int kRun = kChunk / kScatterWarps;  // slots walked in order by one warp
 

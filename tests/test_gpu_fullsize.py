@@ -3,7 +3,8 @@ configuration bench.py times (automatic tile and router choice).
 
 Routing is checked on every token (ids, weights, counts, offsets, the
 permutation and its inverse, bit for bit against the float64 oracle); the
-layer output on a sample of tokens the oracle computes one by one: the
+SwiGLU rows h of every slot of a sample of tokens, and the layer output on
+those tokens, which the oracle computes one by one: the
 first and last token, tokens that use the most and the least loaded
 expert, and a seeded random draw.  Expert weights for the oracle are drawn
 again on the host from the same counter keys, one expert at a time."""
@@ -80,6 +81,14 @@ def test_full_size_workload(name):
     np.testing.assert_array_equal(v["inv_perm"].cpu().numpy(), inv)
 
     toks = sample_tokens(cfg, counts, ids)
+    # h on every permuted row of the sampled tokens (one expert's rows at a time)
+    h_dev = v["h"]
+    for e in np.unique(ids[toks]):
+        tt, jj = np.nonzero(ids[toks] == e)
+        rows = inv[toks[tt], jj]
+        want_h = oracle.swiglu_ffn_rows(oracle.bf16_to_f64(inp.x[toks[tt]]), synth.expert_gate_up(cfg, int(e)))
+        got_h = host_f64(h_dev[torch_index(rows.astype(np.int64))])
+        assert_close_output(got_h, want_h, what=f"h of expert {int(e)}")
     want = oracle.layer_forward_tokens(inp.x, toks, ids, w, lambda e: synth.expert_gate_up(cfg, e),
                                        lambda e: synth.expert_down(cfg, e), inp.w_sh_gate_up, inp.w_sh_down)
     got = host_f64(y[torch_index(toks)])

@@ -450,6 +450,41 @@ def test_token_subset_path_agrees_with_full_layer():
     np.testing.assert_allclose(y2, full["y"], rtol=1e-13, atol=1e-16)
 
 
+def test_token_subset_path_with_shared_expert_matches_bruteforce_loops():
+    """The per-token path's shared-expert branch (the checker of the full-size
+    Ling-like parity test) against the pure-Python loops: the shared FFN is
+    added once per token with weight 1, over its own I_s split of the
+    columns.  Dropping the branch, scaling it by a routing weight or
+    splitting [H, 2 I_s] at the routed I would each fail here."""
+    rng = np.random.default_rng(21)
+    T, H, E, I, k, Is = 6, 8, 5, 3, 2, 4
+    x = _bf(rng, (T, H), 1.0)
+    Wr = (rng.standard_normal((H, E)) * 0.5).astype(np.float32)
+    b = synth.zipf_bias(E, 1.2)
+    Wgu, Wd = _bf(rng, (E, H, 2 * I), 0.5), _bf(rng, (E, I, H), 0.5)
+    sgu, sd = _bf(rng, (H, 2 * Is), 0.5), _bf(rng, (Is, H), 0.5)
+    want = _bruteforce_layer(x, Wr, b, Wgu, Wd, k, sgu, sd)
+    ids, w = om.topk_route(om.router_logits(x, Wr, b), k)
+    toks = [0, 2, 5]
+    got = om.layer_forward_tokens(x, toks, ids, w, lambda e: Wgu[e], lambda e: Wd[e], sgu, sd)
+    np.testing.assert_allclose(got, want[toks], rtol=1e-11, atol=1e-12)
+    without = om.layer_forward_tokens(x, toks, ids, w, lambda e: Wgu[e], lambda e: Wd[e])
+    assert np.abs(got - without).max() > 1e-2 * np.abs(got).max()
+
+
+def test_token_subset_path_worked_example_with_shared_expert():
+    """The two-token worked example through the per-token path: the shared
+    term 2*silu(1), -4*silu(1) is added to each token's closed-form output."""
+    x, Wr, Wgu, Wd, y = _worked_example()
+    Wsgu = np.array([[1, 1], [1, 1]], np.float32)
+    Wsd = np.array([[2, -4]], np.float32)
+    s = sig(1)
+    ids, w = om.topk_route(om.router_logits(bits(x), Wr), 2)
+    got = om.layer_forward_tokens(bits(x), [1, 0], ids, w, lambda e: bits(Wgu)[e], lambda e: bits(Wd)[e],
+                                  bits(Wsgu), bits(Wsd))
+    np.testing.assert_allclose(got, (y + np.array([[2 * s, -4 * s]] * 2))[[1, 0]], rtol=1e-13)
+
+
 # ---------------------------------------------------------------- inputs
 
 def test_logit_gap_enforcement():
