@@ -230,6 +230,7 @@ def recorded_traffic(workload):
 
 # ---------------------------------------------------------------- timed runs
 TILES = {"auto": 0, "small": 1, "large": 2, "pair": 3, "fused": 4}
+COMBINE = {"auto": 0, "fused": 1, "separate": 2}
 # further workloads timed with the default workload, reported under "extra" (their weights
 # replace the decode ones after the decode and prefill measurements)
 DEFAULT_EXTRA = "ling_skewed_t4096,sweep_decode_t1,sweep_decode_t4,sweep_decode_t16,sweep_decode_t64"
@@ -238,7 +239,7 @@ SCORING = {"softmax": 0, "softmax_select_bias": 1, "sigmoid": 2}
 
 
 def time_workload(cfg, d, ws, steps, warmup, rank, world, flush, moe, gpu_index, sample_clocks=True, tiles=0,
-                  graph=False, scoring=0):
+                  graph=False, scoring=0, combine=0):
     """K timed steps (L2 flushed before each).  graph=True captures one layer
     call in a CUDA graph and replays it per step (no host launch overhead);
     otherwise every step is an eager library call."""
@@ -250,7 +251,7 @@ def time_workload(cfg, d, ws, steps, warmup, rank, world, flush, moe, gpu_index,
     def step(evs=None, info=None):
         return moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws,
                            d["w_sh_gate_up"], d["w_sh_down"], stage_events=evs, info=info, tiles=tiles, out=out,
-                           scoring=scoring)
+                           scoring=scoring, combine=combine)
 
     def events(n):
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
@@ -319,7 +320,7 @@ def time_workload(cfg, d, ws, steps, warmup, rank, world, flush, moe, gpu_index,
                 step_ms_median=statistics.median(step_ms), host_us_per_call=host_us)
 
 
-def time_e2e(cfg, d, ws, steps, warmup, rank, world, moe, tiles=0):
+def time_e2e(cfg, d, ws, steps, warmup, rank, world, moe, tiles=0, combine=0):
     """Same metric through the public call with host buffers: pinned x in,
     y out, both copies inside the timed region."""
     import torch
@@ -332,7 +333,7 @@ def time_e2e(cfg, d, ws, steps, warmup, rank, world, moe, tiles=0):
     def step():
         x_d.copy_(x_h, non_blocking=True)
         moe.forward(x_d, d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws, d["w_sh_gate_up"],
-                    d["w_sh_down"], out=y_d, tiles=tiles)
+                    d["w_sh_down"], out=y_d, tiles=tiles, combine=combine)
         y_h.copy_(y_d, non_blocking=True)
 
     for _ in range(warmup):
@@ -408,16 +409,17 @@ def run_ours(args):
     ws = moe.alloc_workspace(cfg.T, cfg.H, cfg.E, cfg.I, cfg.k, cfg.I_s)
     flush = L2Flush()
     tiles = TILES[args.tiles]
+    comb = COMBINE[args.combine]
     # Timed: CUDA-graph replay of one layer call per step (how a serving loop
     # runs it; the kernels' programmatic launches overlap there).  A separate
     # eager pass records per-stage CUDA events for the breakdown.
     main_e = time_workload(cfg, d, ws, args.steps, args.warmup, rank, world, flush, moe, gpu_index,
-                           sample_clocks=False, tiles=tiles)
+                           sample_clocks=False, tiles=tiles, combine=comb)
     main = time_workload(cfg, d, ws, args.steps, args.warmup, rank, world, flush, moe, gpu_index, tiles=tiles,
-                         graph=True)
+                         combine=comb, graph=True)
     counts = moe.workspace_view(ws, cfg.T, cfg.H, cfg.E, cfg.I, cfg.k, cfg.I_s)["counts"].cpu().numpy()
     acc = layer_accounting(cfg, counts)
-    e2e = time_e2e(cfg, d, ws, args.steps, args.warmup, rank, world, moe, tiles=tiles)
+    e2e = time_e2e(cfg, d, ws, args.steps, args.warmup, rank, world, moe, tiles=tiles, combine=comb)
 
     def roof(cfg_, res, acc_, step_ms):
         gate_up_ms = res["stage_ms"][3]
@@ -454,12 +456,13 @@ def run_ours(args):
         d2["x"] = torch.from_numpy(px.view(np.int16)).view(torch.bfloat16).cuda()
         ws2 = moe.alloc_workspace(pcfg.T, pcfg.H, pcfg.E, pcfg.I, pcfg.k, pcfg.I_s)
         pres_e = time_workload(pcfg, d2, ws2, args.steps, args.warmup, rank, world, flush, moe, gpu_index,
-                               sample_clocks=False, tiles=tiles)
+                               sample_clocks=False, tiles=tiles, combine=comb)
         pres = time_workload(pcfg, d2, ws2, args.steps, args.warmup, rank, world, flush, moe, gpu_index,
-                             tiles=tiles, graph=True)
+                             tiles=tiles, graph=True, combine=comb)
         pcounts = moe.workspace_view(ws2, pcfg.T, pcfg.H, pcfg.E, pcfg.I, pcfg.k)["counts"].cpu().numpy()
         pacc = layer_accounting(pcfg, pcounts)
-        pe2e = time_e2e(pcfg, d2, ws2, max(3, args.steps // 2), args.warmup, rank, world, moe, tiles=tiles)
+        pe2e = time_e2e(pcfg, d2, ws2, max(3, args.steps // 2), args.warmup, rank, world, moe, tiles=tiles,
+                        combine=comb)
         prefill = {"workload": pcfg.name, "value": round(pres["value"], 1), "unit": "tokens/s",
                    "ms_per_step": round(pres["ms_per_step"], 4), "gpu_launches": pres["launches"],
                    "eager": eager_of(pres_e), "clocks": pres["clocks"],
@@ -486,9 +489,9 @@ def run_ours(args):
                 torch.bfloat16).cuda()
             wse = moe.alloc_workspace(ecfg.T, ecfg.H, ecfg.E, ecfg.I, ecfg.k, ecfg.I_s)
             eres = time_workload(ecfg, de, wse, args.steps, args.warmup, rank, world, flush, moe, gpu_index,
-                                 sample_clocks=False, tiles=tiles, scoring=scoring)
+                                 sample_clocks=False, tiles=tiles, scoring=scoring, combine=comb)
             gres = time_workload(ecfg, de, wse, args.steps, args.warmup, rank, world, flush, moe, gpu_index,
-                                 sample_clocks=False, tiles=tiles, graph=True, scoring=scoring)
+                                 sample_clocks=False, tiles=tiles, graph=True, scoring=scoring, combine=comb)
             ecounts = moe.workspace_view(wse, ecfg.T, ecfg.H, ecfg.E, ecfg.I, ecfg.k, ecfg.I_s)["counts"]
             eacc = layer_accounting(ecfg, ecounts.cpu().numpy())
             extra[spec] = {"value": round(gres["value"], 1), "unit": "tokens/s",
@@ -532,6 +535,8 @@ def run_ours(args):
             line["extra"] = extra
         if args.tiles != "auto":
             line["config"]["tiles"] = args.tiles
+        if args.combine != "auto":
+            line["config"]["combine"] = args.combine
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -575,6 +580,8 @@ def main():
     ap.add_argument("--cpu-sample-tokens", type=int, default=16)
     ap.add_argument("--ref-sample-tokens", type=int, default=2)
     ap.add_argument("--tiles", choices=sorted(TILES), default="auto", help="grouped GEMM tile policy (tuning)")
+    ap.add_argument("--combine", choices=sorted(COMBINE), default="auto",
+                    help="weighted combine in the down GEMM's epilogue (fused) or its own kernel (separate)")
     ap.add_argument("--extra", default=None,
                     help="comma-separated further workloads to time (default with the default workload: the "
                          "Ling-like skewed prefill and the small-batch decode sweep; otherwise none); "

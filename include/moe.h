@@ -106,6 +106,28 @@ enum {
 /* MOE_ROUTER_AUTO picks SMALL when T <= 16 and E % 4 == 0, else TC when
  * E % 8 == 0, else FMA. */
 
+/* Where the weighted combine runs (moe_forward_ex options).  Both give
+ * bitwise the same y: the k expert rows of a token (each first summed over
+ * its K slabs, slab order) are summed in slot order j = 0..k-1 in fp32, the
+ * shared-expert row is added last, and y is rounded to bf16 once.
+ *   FUSED:    in the down GEMM's epilogue.  Each epilogue warp counts the
+ *             rows it stored on a per-(token, 64-column chunk) counter in
+ *             the workspace; the warp whose store completes a token's chunk
+ *             (the last of its k rows, times the K slabs) sums the chunk and
+ *             writes it to y.  No warp waits for another.  A K-split
+ *             gate/up GEMM likewise sums its slabs and applies SwiGLU in the
+ *             epilogue of the last slab to land.  No combine launch.
+ *   SEPARATE: the down GEMM writes fp32 rows; a combine kernel (and, for a
+ *             K-split gate/up GEMM, a slab-sum + SwiGLU kernel) follows. */
+enum {
+  MOE_COMBINE_AUTO = 0,  /* the K-split gate/up's slab sum + SwiGLU in its epilogue, the combine in its own
+                            kernel: the fused combine measured slower at every size (its finishing warps
+                            gather a token's k rows one token at a time, while a separate kernel has
+                            every SM's warps loading at once) */
+  MOE_COMBINE_FUSED = 1,
+  MOE_COMBINE_SEPARATE = 2
+};
+
 /* Router scoring: how the k experts of a token are selected and weighted
  * from its fp32 logits l[e] and the optional per-expert bias b[e].  The
  * systems-engineering handbook page on Qwen 3.5-397B MoE on Ironwood
@@ -136,10 +158,15 @@ int moe_abi_version(void);
  *   logits [S, T, E] f32 (S router partial slabs), router_split [3, H, E]
  *   bf16, block_hist (permute), split: K-split partial slabs of the expert
  *   GEMMs when few tokens leave SMs idle (f32; 0 bytes when unused), fused:
- *   partial slabs of the one-launch layer for T <= 4 (f32; 0 bytes above). */
+ *   partial slabs of the one-launch layer for T <= 4 (f32; 0 bytes above),
+ *   arrivals: u32 counters of the combine in the down GEMM's epilogue (one
+ *   per token and 64 output columns) and of a K-split gate/up GEMM's
+ *   SwiGLU (one per row and 32 intermediate columns).  Each layer call
+ *   zeroes them in its routing kernel and leaves them zero. */
 typedef struct moe_workspace_layout {
   size_t status, topk_ids, topk_w, counts, offsets, sorted_token_ids, inv_perm;
   size_t h, o, h_shared, o_shared, logits, router_split, block_hist, split, fused;
+  size_t arrivals;
   size_t total;
 } moe_workspace_layout_t;
 
@@ -281,7 +308,10 @@ typedef struct moe_forward_options {
   /* Router scoring rule (MOE_SCORE_*; 0, the zero-initialised default, is
    * MOE_SCORE_SOFTMAX). */
   int scoring;
-  int reserved[4];
+  /* Where the weighted combine (and, when K is split, the slab sum + SwiGLU
+   * of the gate/up GEMM) runs (MOE_COMBINE_*; 0 is MOE_COMBINE_AUTO). */
+  int combine;
+  int reserved[3];
 } moe_forward_options_t;
 
 moe_status_t moe_forward_ex(const uint16_t *x, const float *w_router, const float *bias,

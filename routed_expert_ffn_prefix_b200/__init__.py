@@ -19,6 +19,7 @@ __all__ = [
     "MoEError", "lib", "TILES_AUTO", "TILES_SMALL", "TILES_LARGE", "TILES_PAIR", "TILES_FUSED",
     "ROUTER_AUTO", "ROUTER_FMA", "ROUTER_TC", "ROUTER_SMALL",
     "SCORE_SOFTMAX", "SCORE_SOFTMAX_SELECT_BIAS", "SCORE_SIGMOID",
+    "COMBINE_AUTO", "COMBINE_FUSED", "COMBINE_SEPARATE",
     "workspace_size", "workspace_layout", "alloc_workspace", "route", "permute", "grouped_swiglu",
     "grouped_down", "down_combine", "forward", "device_status", "clear_device_status", "selftest_timeout",
     "STATUS",
@@ -27,6 +28,7 @@ __all__ = [
 TILES_AUTO, TILES_SMALL, TILES_LARGE, TILES_PAIR, TILES_FUSED = 0, 1, 2, 3, 4
 ROUTER_AUTO, ROUTER_FMA, ROUTER_TC, ROUTER_SMALL = 0, 1, 2, 3
 SCORE_SOFTMAX, SCORE_SOFTMAX_SELECT_BIAS, SCORE_SIGMOID = 0, 1, 2
+COMBINE_AUTO, COMBINE_FUSED, COMBINE_SEPARATE = 0, 1, 2
 
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_ALIGNMENT", 3: "MOE_ERR_WORKSPACE",
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT", 6: "MOE_ERR_UNSUPPORTED_ARCH",
@@ -42,13 +44,14 @@ class MoEError(RuntimeError):
 class _Layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "status", "topk_ids", "topk_w", "counts", "offsets", "sorted_token_ids", "inv_perm",
-        "h", "o", "h_shared", "o_shared", "logits", "router_split", "block_hist", "split", "fused", "total")]
+        "h", "o", "h_shared", "o_shared", "logits", "router_split", "block_hist", "split", "fused", "arrivals",
+        "total")]
 
 
 class _Options(ctypes.Structure):
     _fields_ = [("tile_policy", ctypes.c_int), ("router_impl", ctypes.c_int),
                 ("stage_events", ctypes.c_void_p * 7), ("launches", ctypes.c_int), ("scoring", ctypes.c_int),
-                ("reserved", ctypes.c_int * 4)]
+                ("combine", ctypes.c_int), ("reserved", ctypes.c_int * 3)]
 
 
 _P, _I, _Z, _U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint64
@@ -266,8 +269,9 @@ def down_combine(h, w_down, topk_w, inv_perm, offsets, shared_out, ws, tiles=TIL
 
 def forward(x, w_router, bias, w_gate_up, w_down, k, ws, w_sh_gate_up=None, w_sh_down=None,
             tiles=TILES_AUTO, router=ROUTER_AUTO, out=None, stage_events=None, info=None,
-            scoring=SCORE_SOFTMAX):
-    """The whole layer: y [T,H] bf16 (scoring: the router's SCORE_* rule).
+            scoring=SCORE_SOFTMAX, combine=COMBINE_AUTO):
+    """The whole layer: y [T,H] bf16 (scoring: the router's SCORE_* rule;
+    combine: COMBINE_* -- in the down GEMM's epilogue or in its own kernel).
 
     stage_events: optional list of 7 torch.cuda.Event recorded at the stage
     boundaries (see include/moe.h); info: optional dict that receives the
@@ -292,6 +296,7 @@ def forward(x, w_router, bias, w_gate_up, w_down, k, ws, w_sh_gate_up=None, w_sh
     y = out if out is not None else torch.empty(T, H, dtype=torch.bfloat16, device=x.device)
     opt = _Options(tiles, router)
     opt.scoring = scoring
+    opt.combine = combine
     if stage_events is not None:
         for i, ev in enumerate(stage_events):
             if ev is not None:

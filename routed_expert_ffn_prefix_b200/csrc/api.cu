@@ -75,6 +75,22 @@ inline SplitPlan split_plan(int T, int H, int E, int I, int k, int tiles) {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Arrival counters of the last-arriver epilogues: one per (row, 32-column
+// chunk of the gate or up tile) for a K-split gate/up GEMM, one per (token,
+// column chunk) for the down GEMM with the combine.  Chunks per down row:
+// 8 per 512 output columns (SM pairs), which also covers the single-SM
+// kernel's 4 per 256.  A multiple of 64 words, so the region has no
+// alignment padding and the routing kernels zero all of it with 16-byte
+// stores.
+inline int down_cnt_stride(int H) { return ((H + 511) / 512) * 8; }
+inline size_t arrival_words(int T, int H, int E, int I, int k) {
+  const SplitPlan sp = split_plan(T, H, E, I, k, MOE_TILES_SMALL);
+  const size_t gu = sp.gate_up > 1 ? (size_t)T * k * (I / 128) * 4 : 0;
+  const size_t dn = (size_t)T * down_cnt_stride(H);
+  const size_t w = gu > dn ? gu : dn;
+  return (w + 63) & ~size_t(63);
+}
+
 // ---------------------------------------------------------------- workspace
 moe_workspace_layout_t make_layout(int T, int H, int E, int I, int k, int I_s) {
   moe_workspace_layout_t L{};
@@ -112,6 +128,7 @@ moe_workspace_layout_t make_layout(int T, int H, int E, int I, int k, int I_s) {
     fused = (size_t)kFusedMaxSplit * frows * (2 * imax + H) * 4;
   }
   L.fused = take(fused);
+  L.arrivals = take(arrival_words(T, H, E, I, k) * 4);
   L.total = off;
   return L;
 }
@@ -253,7 +270,8 @@ struct PermOut {
 
 moe_status_t run_route(const uint16_t* x, const float* w_router, const float* bias, int T, int H, int E, int k,
                        int scoring, int32_t* ids, float* w, int impl, void* ws, const moe_workspace_layout_t& L,
-                       const DeviceInfo& dev, cudaStream_t s, const PermOut* perm = nullptr) {
+                       const DeviceInfo& dev, cudaStream_t s, const PermOut* perm = nullptr,
+                       ZeroSpan zero = ZeroSpan{nullptr, 0}) {
   DevStatus* st = status_of(ws);
   float* logits = at<float>(ws, L.logits);
   impl = resolve_router(impl, T, E);
@@ -263,7 +281,7 @@ moe_status_t run_route(const uint16_t* x, const float* w_router, const float* bi
     return cuda_status(launch_router_small(x, w_router, bias, T, H, E, k, scoring, logits, &st->arrivals, ids, w,
                                            perm ? perm->counts : nullptr, perm ? perm->offsets : nullptr,
                                            perm ? perm->sorted_ids : nullptr, perm ? perm->inv_perm : nullptr, st,
-                                           s));
+                                           zero, s));
   }
   int nsplit = 1;
   if (impl == MOE_ROUTER_TC) {
@@ -302,15 +320,17 @@ moe_status_t run_route(const uint16_t* x, const float* w_router, const float* bi
     MOE_TRY(cuda_status(launch_router_logits_fma(x, w_router, T, H, E, logits, s)));
     nsplit = fma_router_splits(T, H);
   }
-  return cuda_status(launch_topk(logits, nsplit, (size_t)T * E, bias, T, E, k, scoring, ids, w, st, s));
+  return cuda_status(launch_topk(logits, nsplit, (size_t)T * E, bias, T, E, k, scoring, ids, w, st, zero, s));
 }
 
 // nsplit > 1: K-split into partial slabs [nsplit][rows][2I] f32 at `partials`
-// (gate columns [0, I), up [I, 2I)), then one reduce + SwiGLU pass into h.
+// (gate columns [0, I), up [I, 2I)), reduced into h either by the last slab
+// of each row chunk to land (arrivals != nullptr: zeroed counters, one per
+// row and 32-column chunk) or by a separate reduce + SwiGLU pass.
 moe_status_t run_swiglu(const uint16_t* x, int src_rows, const uint16_t* w_gate_up, const int32_t* offsets,
                         const int32_t* row_index, int rows, int H, int E, int I, int tiles, uint16_t* h,
                         DevStatus* st, const DeviceInfo& dev, cudaStream_t s, int nsplit = 1,
-                        float* partials = nullptr) {
+                        float* partials = nullptr, uint32_t* arrivals = nullptr) {
   CUtensorMap map;
   if (!make_weight_map(&map, w_gate_up, 2ull * I, (uint64_t)H, (uint64_t)E)) return MOE_ERR_CUDA;
   GemmArgs a{};
@@ -349,16 +369,37 @@ moe_status_t run_swiglu(const uint16_t* x, int src_rows, const uint16_t* w_gate_
     a.n_valid = 2 * I;
     a.k_splits = nsplit;
     a.split_stride = (size_t)rows * 2 * I;
+    if (arrivals != nullptr) {
+      a.arrivals = arrivals;
+      a.cnt_stride = a.n_blocks * 4;
+      a.arrive_target = nsplit;
+      a.fin_out = h;
+      a.fin_ld = I;
+      return cuda_status(launch_grouped_gemm(map, a, EPI_SWIGLU_SPLIT, tiles, dev.num_sms, s));
+    }
     MOE_TRY(cuda_status(launch_grouped_gemm(map, a, EPI_STORE_F32, tiles, dev.num_sms, s)));
     return cuda_status(launch_swiglu_reduce(partials, nsplit, a.split_stride, rows, I, h, s));
   }
   return cuda_status(launch_grouped_gemm(map, a, EPI_SWIGLU, tiles, dev.num_sms, s));
 }
 
+// The weighted combine taken into the down GEMM's epilogue (see Epilogue).
+struct CombineArgs {
+  const int32_t* row_token;  // sorted_token_ids
+  const int32_t* inv_perm;
+  const float* topk_w;
+  const float* shared;  // [T, H] f32 or nullptr
+  uint16_t* y;
+  uint32_t* arrivals;  // zeroed, arrival_words() of them
+  int T, k;
+};
+
 // o: fp32 rows; nsplit > 1: K-split into partial slabs [nsplit][rows][H].
+// comb != nullptr: the last of each token's k * nsplit row chunks to land
+// also writes that chunk of y.
 moe_status_t run_down(const uint16_t* h, const uint16_t* w_down, const int32_t* offsets, int rows, int H, int E,
                       int I, int tiles, float* o, DevStatus* st, const DeviceInfo& dev, cudaStream_t s,
-                      int nsplit = 1) {
+                      int nsplit = 1, const CombineArgs* comb = nullptr) {
   CUtensorMap map;
   if (!make_weight_map(&map, w_down, (uint64_t)H, (uint64_t)I, (uint64_t)E)) return MOE_ERR_CUDA;
   const int cols = 128 * gemm_tiles_per_unit(tiles, EPI_STORE_F32);  // output columns per work unit
@@ -385,15 +426,31 @@ moe_status_t run_down(const uint16_t* h, const uint16_t* w_down, const int32_t* 
   a.split_stride = nsplit > 1 ? (size_t)rows * H : 0;
   a.status = st;
   a.timeout_ns = kDefaultTimeoutNs;
+  int epi = EPI_STORE_F32;
+  if (comb != nullptr) {
+    epi = EPI_DOWN_COMBINE;
+    a.arrivals = comb->arrivals;
+    a.cnt_stride = down_cnt_stride(H);
+    a.arrive_target = comb->k * nsplit;
+    a.fin_out = comb->y;
+    a.fin_ld = H;
+    a.row_token = comb->row_token;
+    a.inv_perm = comb->inv_perm;
+    a.topk_w = comb->topk_w;
+    a.shared = comb->shared;
+    a.topk = comb->k;
+    a.n_tokens = comb->T;
+  }
   if (tiles == MOE_TILES_PAIR) {  // 2 x 256 output columns per unit (128 of each per SM of the pair)
+    if (nsplit > 1) return MOE_ERR_INVALID_ARG;
     a.n_blocks = (H + 511) / 512;
     a.col_stride = 512;
     a.col1_off = 256;
     a.out_col_stride = 512;
     a.out_col1_off = 256;
-    return cuda_status(launch_grouped_gemm_pair(map, a, EPI_STORE_F32, dev.num_sms, s));
+    return cuda_status(launch_grouped_gemm_pair(map, a, epi, dev.num_sms, s));
   }
-  return cuda_status(launch_grouped_gemm(map, a, EPI_STORE_F32, tiles, dev.num_sms, s));
+  return cuda_status(launch_grouped_gemm(map, a, epi, tiles, dev.num_sms, s));
 }
 
 }  // namespace
@@ -415,7 +472,7 @@ const char* moe_status_string(int status) {
   }
 }
 
-int moe_abi_version(void) { return 1; }
+int moe_abi_version(void) { return 2; }
 
 moe_status_t moe_workspace_layout(int T, int H, int E, int I, int k, int I_s, moe_workspace_layout_t* out) {
   if (out == nullptr || I_s < 0) return MOE_ERR_INVALID_ARG;
@@ -535,15 +592,25 @@ moe_status_t moe_down_combine(const uint16_t* h, const uint16_t* w_down, const f
   if (!all_aligned(h, w_down, topk_w, inv_perm, offsets, y) || (shared_out && !aligned16(shared_out)))
     return MOE_ERR_ALIGNMENT;
   const moe_workspace_layout_t L = make_layout(T, H, E, I, k, 0);
-  MOE_TRY(check_ws(workspace, workspace_bytes, L.h_shared));
+  MOE_TRY(check_ws(workspace, workspace_bytes, L.total));
   DeviceInfo dev;
   MOE_TRY(check_device(&dev));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int rows = T * k;
   float* o = at<float>(workspace, L.o);
   DevStatus* st = status_of(workspace);
-  MOE_TRY(run_down(h, w_down, offsets, rows, H, E, I, choose_tiles(tile_policy, rows, E), o, st, dev, s));
-  return cuda_status(launch_combine(o, topk_w, inv_perm, shared_out, T, H, k, rows, 1, 0, y, st, s));
+  // The combine runs in the down GEMM's epilogue; its token row of each
+  // permuted row is not an argument here, so it is derived from inv_perm
+  // into the workspace's sorted_token_ids region, and the arrival counters
+  // are zeroed, in one small kernel.
+  int32_t* sids = at<int32_t>(workspace, L.sorted_token_ids);
+  uint32_t* arrivals = at<uint32_t>(workspace, L.arrivals);
+  MOE_TRY(cuda_status(launch_row_tokens(inv_perm, T, k, sids,
+                                        ZeroSpan{reinterpret_cast<uint4*>(arrivals),
+                                                 (int)(arrival_words(T, H, E, I, k) / 4)},
+                                        st, s)));
+  const CombineArgs comb{sids, inv_perm, topk_w, shared_out, y, arrivals, T, k};
+  return run_down(h, w_down, offsets, rows, H, E, I, choose_tiles(tile_policy, rows, E), o, st, dev, s, 1, &comb);
 }
 
 moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const float* bias, const uint16_t* w_gate_up,
@@ -561,6 +628,8 @@ moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const floa
   const int tile_policy = options ? options->tile_policy : MOE_TILES_AUTO;
   const int router_impl = options ? options->router_impl : MOE_ROUTER_AUTO;
   const int scoring = options ? options->scoring : MOE_SCORE_SOFTMAX;
+  const int combine = options ? options->combine : MOE_COMBINE_AUTO;
+  if (combine < MOE_COMBINE_AUTO || combine > MOE_COMBINE_SEPARATE) return MOE_ERR_INVALID_ARG;
   if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_FUSED) return MOE_ERR_INVALID_ARG;
   if (router_impl < MOE_ROUTER_AUTO || router_impl > MOE_ROUTER_SMALL) return MOE_ERR_INVALID_ARG;
   if (!valid_scoring(scoring)) return MOE_ERR_INVALID_ARG;
@@ -609,14 +678,27 @@ moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const floa
   }
 
   const int ri = resolve_router(router_impl, T, E);
+  const int tiles = choose_tiles(tile_policy, rows, E);
+  const SplitPlan sp = split_plan(T, H, E, I, k, tiles);
+  // Last-arriver epilogues: the K-split gate/up GEMM sums its slabs in its
+  // epilogue unless SEPARATE is asked for; the down GEMM combines in its
+  // epilogue only on request (FUSED), because a separate combine kernel
+  // measured faster at every size (see the combine options in moe.h).
+  const bool fuse_swiglu = combine != MOE_COMBINE_SEPARATE && sp.gate_up > 1;
+  const bool fuse_combine = combine == MOE_COMBINE_FUSED;
+  uint32_t* arrivals = at<uint32_t>(ws, L.arrivals);
+  // the routing kernel zeroes the arrival counters of the fused epilogues
+  const bool need_zero = fuse_swiglu || fuse_combine;
+  const ZeroSpan zero{need_zero ? reinterpret_cast<uint4*>(arrivals) : nullptr,
+                      need_zero ? (int)(arrival_words(T, H, E, I, k) / 4) : 0};
   MOE_TRY(mark(0));
   if (ri == MOE_ROUTER_SMALL) {
     const PermOut perm{counts, offs, sids, inv};
-    MOE_TRY(run_route(x, w_router, bias, T, H, E, k, scoring, ids, tw, ri, ws, L, dev, s, &perm));
+    MOE_TRY(run_route(x, w_router, bias, T, H, E, k, scoring, ids, tw, ri, ws, L, dev, s, &perm, zero));
     launches += 1;
     MOE_TRY(mark(1));
   } else {
-    MOE_TRY(run_route(x, w_router, bias, T, H, E, k, scoring, ids, tw, ri, ws, L, dev, s));
+    MOE_TRY(run_route(x, w_router, bias, T, H, E, k, scoring, ids, tw, ri, ws, L, dev, s, nullptr, zero));
     launches += ri == MOE_ROUTER_TC ? 3 : 2;
     MOE_TRY(mark(1));
     MOE_TRY(cuda_status(
@@ -624,8 +706,6 @@ moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const floa
     launches += rows <= 8192 ? 1 : 3;
   }
   MOE_TRY(mark(2));
-  const int tiles = choose_tiles(tile_policy, rows, E);
-  const SplitPlan sp = split_plan(T, H, E, I, k, tiles);
   float* split = at<float>(ws, L.split);
   float* o_sh = nullptr;
   if (shared) {
@@ -637,14 +717,22 @@ moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const floa
     launches += 2;
   }
   MOE_TRY(mark(3));
-  MOE_TRY(run_swiglu(x, T, w_gate_up, offs, sids, rows, H, E, I, tiles, h, st, dev, s, sp.gate_up, split));
-  launches += sp.gate_up > 1 ? 2 : 1;
+  MOE_TRY(run_swiglu(x, T, w_gate_up, offs, sids, rows, H, E, I, tiles, h, st, dev, s, sp.gate_up, split,
+                     fuse_swiglu ? arrivals : nullptr));
+  launches += (sp.gate_up > 1 && !fuse_swiglu) ? 2 : 1;
   MOE_TRY(mark(4));
   float* od = sp.down > 1 ? split : o;
-  MOE_TRY(run_down(h, w_down, offs, rows, H, E, I, tiles, od, st, dev, s, sp.down));
-  MOE_TRY(mark(5));
-  MOE_TRY(cuda_status(launch_combine(od, tw, inv, o_sh, T, H, k, rows, sp.down, (size_t)rows * H, y, st, s)));
-  launches += 2;  // down GEMM, combine
+  if (fuse_combine) {
+    const CombineArgs comb{sids, inv, tw, o_sh, y, arrivals, T, k};
+    MOE_TRY(run_down(h, w_down, offs, rows, H, E, I, tiles, od, st, dev, s, sp.down, &comb));
+    launches += 1;
+    MOE_TRY(mark(5));
+  } else {
+    MOE_TRY(run_down(h, w_down, offs, rows, H, E, I, tiles, od, st, dev, s, sp.down));
+    MOE_TRY(mark(5));
+    MOE_TRY(cuda_status(launch_combine(od, tw, inv, o_sh, T, H, k, rows, sp.down, (size_t)rows * H, y, st, s)));
+    launches += 2;  // down GEMM, combine
+  }
   MOE_TRY(mark(6));
   if (options) options->launches = launches;
   return MOE_OK;

@@ -192,7 +192,31 @@ __global__ void __launch_bounds__(kThreads) swiglu_reduce_kernel(const float* __
   }
 }
 
+// row_token[inv_perm[s]] = s / k for every slot s (the token of each permuted
+// row, for a down GEMM that combines in its epilogue), and the zeroing of the
+// arrival counters that epilogue uses.
+__global__ void row_tokens_kernel(const int32_t* __restrict__ inv_perm, int n, int k, int32_t* __restrict__ row_token,
+                                  ZeroSpan zero, DevStatus* st) {
+  zero_span(zero);
+  for (int s = blockIdx.x * blockDim.x + threadIdx.x; s < n; s += gridDim.x * blockDim.x) {
+    const int r = inv_perm[s];
+    if (r < 0 || r >= n) {
+      raise_error(st, MOE_ERR_DEVICE_BOUNDS, SITE_COMBINE, s);
+    } else {
+      row_token[r] = s / k;
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_row_tokens(const int32_t* inv_perm, int T, int k, int32_t* row_token, ZeroSpan zero, DevStatus* st,
+                              cudaStream_t s) {
+  const long long n = (long long)T * k;
+  const long long work = n > zero.n16 ? n : zero.n16;
+  const int blocks = (int)((work + kThreads - 1) / kThreads < 1184 ? (work + kThreads - 1) / kThreads : 1184);
+  return launch_kernel(row_tokens_kernel, dim3(blocks), dim3(kThreads), 0, s, inv_perm, (int)n, k, row_token, zero, st);
+}
 
 cudaError_t launch_swiglu_reduce(const float* partials, int nsplit, size_t split_stride, int rows, int I, uint16_t* h,
                                  cudaStream_t s) {

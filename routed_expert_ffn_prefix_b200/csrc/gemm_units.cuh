@@ -90,4 +90,176 @@ __device__ void build_unit_prefix(const GemmArgs& a, int ngroups, int* ustart, i
 // exponential and division are accurate enough.
 __device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
+// ---------------------------------------------------------------- last-arriver reduction
+// The K-split gate/up slabs of a row, or the k expert-output rows of a token,
+// are produced by different work units on different SMs, in no fixed order.
+// Instead of a separate pass over them, every epilogue warp counts its
+// stores on a per-(key, column chunk) counter; the warp whose arrival
+// completes a counter reduces that chunk.  The reduction itself always runs
+// in the same order (K slabs ascending, then slots j = 0..k-1), so the
+// result does not depend on which warp finishes: it is bitwise the same as
+// a separate pass in that order.  No warp ever waits for another.
+constexpr int kMaxKSplit = 8;
+
+__device__ __forceinline__ uint32_t atom_add_relaxed_gpu(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.relaxed.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// h[r, c] = bf16(silu(sum_s gate_s) * sum_s up_s) for this lane's column:
+// cols[0] = gate column, cols[1] = up column of the fp32 slab rows (lane = column).
+__device__ __forceinline__ void finish_swiglu_row(const GemmArgs& a, int r, const int (&cols)[2]) {
+  if (cols[1] >= a.n_valid) return;  // never taken: the K-split gate/up units cover exactly 2I columns
+  const float* p = reinterpret_cast<const float*>(a.out) + (size_t)r * a.ld_out;
+  const int S = a.k_splits;
+  float g[kMaxKSplit], u[kMaxKSplit];
+#pragma unroll
+  for (int s = 0; s < kMaxKSplit; ++s) {
+    if (s < S) {
+      g[s] = __ldcg(p + (size_t)s * a.split_stride + cols[0]);
+      u[s] = __ldcg(p + (size_t)s * a.split_stride + cols[1]);
+    }
+  }
+  float gs = g[0], us = u[0];
+#pragma unroll
+  for (int s = 1; s < kMaxKSplit; ++s) {
+    if (s < S) {
+      gs += g[s];
+      us += u[s];
+    }
+  }
+  if (cols[0] < a.fin_ld)
+    reinterpret_cast<__nv_bfloat16*>(a.fin_out)[(size_t)r * a.fin_ld + cols[0]] = __float2bfloat16_rn(silu_f(gs) * us);
+}
+
+// y[t, c] = bf16(sum_{j<k} w[t,j] * (sum_s o_s[inv_perm[t,j], c]) + shared[t, c]) for this
+// lane's columns (one per MMA tile of the unit), slots in order, fp32.
+template <int MT>
+__device__ __forceinline__ void finish_combine_row(const GemmArgs& a, int t, const int (&cols)[MT]) {
+  const int lane = lane_id(), k = a.topk, S = a.k_splits;
+  const float* o = reinterpret_cast<const float*>(a.out);
+  int ra = 0, rb = 0;
+  float wa = 0.f, wb = 0.f;
+  if (lane < k) {
+    ra = __ldg(a.inv_perm + (size_t)t * k + lane);
+    wa = __ldg(a.topk_w + (size_t)t * k + lane);
+  }
+  if (lane + 32 < k) {
+    rb = __ldg(a.inv_perm + (size_t)t * k + lane + 32);
+    wb = __ldg(a.topk_w + (size_t)t * k + lane + 32);
+  }
+  const bool bad = (lane < k && (ra < 0 || ra >= a.rows_cap)) || (lane + 32 < k && (rb < 0 || rb >= a.rows_cap));
+  if (__any_sync(0xffffffffu, bad)) {
+    if (lane == 0) raise_error(a.status, MOE_ERR_DEVICE_BOUNDS, SITE_COMBINE, t);
+    return;
+  }
+  // output columns past n_valid (the pair kernel's last block when H % 512 != 0) are never read
+  bool live[MT];
+#pragma unroll
+  for (int i = 0; i < MT; ++i) live[i] = cols[i] < a.n_valid;
+  float acc[MT];
+#pragma unroll
+  for (int i = 0; i < MT; ++i) acc[i] = 0.f;
+  for (int j0 = 0; j0 < k; j0 += 8) {
+    float v[8][MT];
+    int rr[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int j = j0 + q;
+      rr[q] = __shfl_sync(0xffffffffu, j < 32 ? ra : rb, j & 31);
+      if (j < k) {
+#pragma unroll
+        for (int i = 0; i < MT; ++i) v[q][i] = live[i] ? __ldcg(o + (size_t)rr[q] * a.ld_out + cols[i]) : 0.f;
+      }
+    }
+    for (int s = 1; s < S; ++s) {
+      const float* os = o + (size_t)s * a.split_stride;
+      float p[8][MT];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (j0 + q < k) {
+#pragma unroll
+          for (int i = 0; i < MT; ++i) p[q][i] = live[i] ? __ldcg(os + (size_t)rr[q] * a.ld_out + cols[i]) : 0.f;
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (j0 + q < k) {
+#pragma unroll
+          for (int i = 0; i < MT; ++i) v[q][i] += p[q][i];
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int j = j0 + q;
+      const float wj = __shfl_sync(0xffffffffu, j < 32 ? wa : wb, j & 31);
+      if (j < k) {
+#pragma unroll
+        for (int i = 0; i < MT; ++i) acc[i] = fmaf(wj, v[q][i], acc[i]);
+      }
+    }
+  }
+  __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(a.fin_out) + (size_t)t * a.fin_ld;
+#pragma unroll
+  for (int i = 0; i < MT; ++i) {
+    if (live[i]) {
+      float v = acc[i];
+      if (a.shared) v += __ldg(a.shared + (size_t)t * a.ld_out + cols[i]);
+      y[cols[i]] = __float2bfloat16_rn(v);
+    }
+  }
+}
+
+// One epilogue warp, after storing rows [r0, r0 + nr) of output chunk
+// `chunk`, and after a __syncwarp() and a __threadfence() by every lane
+// since those stores (the release: the stores are visible device-wide before
+// any counter moves): count the arrivals with relaxed atomics and reduce
+// every key this warp completed, after another fence (the acquire: every
+// other warp's stores counted on that key are visible to the loads).
+// Warp-uniform arguments.
+template <int MT, int EPI>
+__device__ __forceinline__ void arrive_rows(const GemmArgs& a, int r0, int nr, int chunk, const int (&cols)[MT]) {
+  const int lane = lane_id();
+  int key = -1;
+  bool fin = false;
+  if (lane < nr) {
+    const int r = r0 + lane;
+    key = r;
+    if constexpr (EPI == EPI_DOWN_COMBINE) {
+      key = __ldg(a.row_token + r);
+      if (key < 0 || key >= a.n_tokens) {
+        raise_error(a.status, MOE_ERR_DEVICE_BOUNDS, SITE_GEMM_EPILOGUE, r);
+        key = -1;
+      }
+    }
+    if (key >= 0) {
+      uint32_t* c = a.arrivals + (size_t)key * a.cnt_stride + chunk;
+      const uint32_t done = atom_add_relaxed_gpu(c, 1u) + 1u;
+      if (done == (uint32_t)a.arrive_target) {
+        fin = true;
+        *c = 0u;  // every arrival has been counted: zero again for the next kernel
+      } else if (done > (uint32_t)a.arrive_target) {
+        raise_error(a.status, MOE_ERR_DEVICE_BOUNDS, SITE_GEMM_EPILOGUE, r);
+      }
+    }
+  }
+  uint32_t m = __ballot_sync(0xffffffffu, fin);
+  if (m == 0u) return;
+  __syncwarp();
+  __threadfence();  // acquire side, before any lane reads other warps' rows
+  while (m) {
+    const int i = __ffs(m) - 1;
+    m &= m - 1u;
+    const int kk = __shfl_sync(0xffffffffu, key, i);
+    if constexpr (EPI == EPI_DOWN_COMBINE) {
+      finish_combine_row<MT>(a, kk, cols);
+    } else {
+      static_assert(EPI != EPI_SWIGLU_SPLIT || MT == 2, "the split SwiGLU needs the gate and the up tile");
+      finish_swiglu_row(a, kk, cols);
+    }
+  }
+}
+
 }  // namespace moe

@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 out[(size_t)(un.row0 + c0 + j) * a.ld_out + col] = __float2bfloat16_rn(silu_f(g[j]) * v[j]);
             }
           }
-        } else {
+        } else {  // fp32 rows (EPI_STORE_F32, and the slabs / rows of the last-arriver reductions)
           // both tiles' 32 rows in one batch of TMEM loads (one wait), then the stores
           float v[MT][32];
           if constexpr (MT == 2) {
@@ -307,6 +307,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&tempty[buf]);
       ++acc_it;
+      if constexpr (EPI == EPI_SWIGLU_SPLIT || EPI == EPI_DOWN_COMBINE) {
+        // TMEM is released; now count this warp's stored rows and reduce the
+        // chunks they complete while the next unit's MMAs run.
+        __syncwarp();
+        __threadfence();
+        int cols[MT];
+        cols[0] = col;
+        if constexpr (MT == 2) cols[1] = col + a.out_col1_off;
+        const int chunk = un.nb * 4 + quarter;
+        for (int c0 = half * 32; c0 < un.rows; c0 += 64)
+          arrive_rows<MT, EPI>(a, un.row0 + c0, min(32, un.rows - c0), chunk, cols);
+      }
     }
   }
 
@@ -338,16 +350,22 @@ int gemm_tiles_per_unit(int tiles, int epilogue) {
   return 2;  // measured: one tile per unit doubles the token-row re-reads and loses more than it overlaps
 }
 
+template <int NT, int ST>
+cudaError_t launch_epi(const CUtensorMap& wmap, const GemmArgs& a, int epilogue, int num_sms, cudaStream_t stream) {
+  switch (epilogue) {
+    case EPI_SWIGLU: return launch_cfg<NT, ST, 2, EPI_SWIGLU>(wmap, a, num_sms, stream);
+    case EPI_SWIGLU_SPLIT: return launch_cfg<NT, ST, 2, EPI_SWIGLU_SPLIT>(wmap, a, num_sms, stream);
+    case EPI_DOWN_COMBINE: return launch_cfg<NT, ST, 2, EPI_DOWN_COMBINE>(wmap, a, num_sms, stream);
+    default: return launch_cfg<NT, ST, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
+  }
+}
+
 cudaError_t launch_grouped_gemm(const CUtensorMap& wmap, const GemmArgs& a, int epilogue, int tiles, int num_sms,
                                 cudaStream_t stream) {
-  if (tiles == MOE_TILES_LARGE) {
-    return epilogue == EPI_SWIGLU ? launch_cfg<256, 3, 2, EPI_SWIGLU>(wmap, a, num_sms, stream)
-                                  : launch_cfg<256, 3, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
-  }
+  if (tiles == MOE_TILES_LARGE) return launch_epi<256, 3>(wmap, a, epilogue, num_sms, stream);
   // Small groups (decode): 128-row passes, 4 stages -- measured ~5% faster
   // than 64-row passes with 5 stages at 1-30 rows per expert.
-  return epilogue == EPI_SWIGLU ? launch_cfg<128, 4, 2, EPI_SWIGLU>(wmap, a, num_sms, stream)
-                                : launch_cfg<128, 4, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
+  return launch_epi<128, 4>(wmap, a, epilogue, num_sms, stream);
 }
 
 }  // namespace moe

@@ -371,7 +371,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 out[(size_t)(un.row0 + c0 + j) * a.ld_out + col] = __float2bfloat16_rn(silu_f(g[j]) * v[j]);
             }
           }
-        } else {
+        } else {  // fp32 rows (EPI_STORE_F32, and the rows of the down-combine reduction)
           // both tiles' 32 rows in one batch of TMEM loads (one wait), then the stores
           float v[MT][32];
           if constexpr (MT == 2) {
@@ -396,6 +396,18 @@ __global__ void __launch_bounds__(kPThreads, 1)
       __syncwarp();
       if (lane == 0) remote_arrive(tempty_leader + buf * 8);
       ++acc_it;
+      if constexpr (EPI == EPI_DOWN_COMBINE) {
+        // TMEM is released; now count this warp's stored rows and reduce the
+        // chunks they complete while the next unit's MMAs run.
+        __syncwarp();
+        __threadfence();
+        int cols[MT];
+        cols[0] = col;
+        if constexpr (MT == 2) cols[1] = col + a.out_col1_off;
+        const int chunk = (un.nb * 2 + (int)rank) * 4 + quarter;
+        for (int c0 = half * 32; c0 < un.rows; c0 += 64)
+          arrive_rows<MT, EPI>(a, un.row0 + c0, min(32, un.rows - c0), chunk, cols);
+      }
     }
   }
 
@@ -462,7 +474,9 @@ cudaError_t launch_grouped_gemm_pair(const CUtensorMap& wmap, const GemmArgs& a,
     // One 256-column tile per unit with a double-buffered accumulator: down
     // 1.03 / 2.35 ms.
     case EPI_SWIGLU: return launch_pair<256, 4, 2, EPI_SWIGLU>(wmap, a, num_sms, stream);
-    default: return launch_pair<256, 4, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
+    case EPI_DOWN_COMBINE: return launch_pair<256, 4, 2, EPI_DOWN_COMBINE>(wmap, a, num_sms, stream);
+    case EPI_STORE_F32: return launch_pair<256, 4, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
+    default: return cudaErrorInvalidValue;  // the K split (and its SwiGLU reduction) runs on single SMs only
   }
 }
 

@@ -68,10 +68,33 @@ struct GemmArgs {
   size_t split_stride; // elements between the partial-result slabs of consecutive K splits
   DevStatus* status;
   uint64_t timeout_ns;
+  // Last-arriver reduction (EPI_SWIGLU_SPLIT, EPI_DOWN_COMBINE).  After a
+  // warp has stored its fp32 rows of a 32-column chunk it adds one to the
+  // counter of every (key, chunk) it covered; the warp that brings a counter
+  // to arrive_target reduces that key's chunk in a fixed order, writes the
+  // result and sets the counter back to zero.  Counters must be zero when
+  // the kernel starts.
+  uint32_t* arrivals;       // [keys][cnt_stride] counters
+  int cnt_stride;           // counters per key (column chunks of the output row)
+  int arrive_target;        // arrivals per (key, chunk): k_splits (gate/up) or topk * k_splits (down)
+  // EPI_SWIGLU_SPLIT: h [rows][fin_ld] bf16 = silu(sum of the gate slabs) * (sum of the up slabs).
+  // EPI_DOWN_COMBINE: y [n_tokens][fin_ld] bf16 = sum_j topk_w[t,j] * (slab-summed o[inv_perm[t,j]]) + shared[t].
+  uint16_t* fin_out;
+  int fin_ld;
+  const int32_t* row_token;  // permuted row -> token (down-combine key)
+  const int32_t* inv_perm;   // [n_tokens][topk] slot -> permuted row
+  const float* topk_w;       // [n_tokens][topk]
+  const float* shared;       // [n_tokens][ld_out] f32 shared-expert rows, or nullptr
+  int topk;
+  int n_tokens;
 };
 
-// SWIGLU: h = bf16(silu(gate) * up); STORE_F32: fp32 rows (K splits to their own slabs).
-enum Epilogue { EPI_SWIGLU = 0, EPI_STORE_F32 = 1 };
+// SWIGLU: h = bf16(silu(gate) * up); STORE_F32: fp32 rows (K splits to their
+// own slabs); SWIGLU_SPLIT: fp32 gate/up slabs of a K split, the last slab
+// of each row chunk to land sums them and writes h; DOWN_COMBINE: fp32
+// expert-output rows (per K slab), the last of a token's k * k_splits row
+// chunks to land writes that chunk of y (weighted slot-order sum + shared).
+enum Epilogue { EPI_SWIGLU = 0, EPI_STORE_F32 = 1, EPI_SWIGLU_SPLIT = 2, EPI_DOWN_COMBINE = 3 };
 
 // MMA tiles (128 weight columns each) per work unit of the given tile
 // policy and epilogue; the caller sets n_blocks/col_stride/out_col_stride
@@ -89,6 +112,19 @@ cudaError_t launch_grouped_gemm_pair(const CUtensorMap& wmap, const GemmArgs& a,
 cudaError_t launch_grouped_gemm(const CUtensorMap& wmap, const GemmArgs& a, int epilogue, int tiles,
                                 int num_sms, cudaStream_t stream);
 
+// A span of device memory a kernel zeroes (grid-stride, 16-byte stores)
+// before its own work: the routing kernels clear the arrival counters of the
+// expert GEMMs' last-arriver epilogues this way, in every layer call.
+struct ZeroSpan {
+  uint4* p;
+  int n16;  // 16-byte words
+};
+__device__ __forceinline__ void zero_span(const ZeroSpan& z) {
+  const int nthreads = gridDim.x * gridDim.y * blockDim.x;
+  const int tid = (blockIdx.y * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x;
+  for (int i = tid; i < z.n16; i += nthreads) z.p[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 // Router.
 cudaError_t launch_router_split(const float* w, int H, int E, uint16_t* planes, cudaStream_t s);
 // fp32 CUDA-core logits into fma_router_splits(T, H) partial slabs [T, E].
@@ -98,7 +134,7 @@ cudaError_t launch_router_logits_fma(const uint16_t* x, const float* w, int T, i
 // logits: nsplit partial slabs of [T, E], split_stride elements apart, summed in slab order;
 // scoring: MOE_SCORE_*.
 cudaError_t launch_topk(const float* logits, int nsplit, size_t split_stride, const float* bias, int T, int E, int k,
-                        int scoring, int32_t* ids, float* w, DevStatus* st, cudaStream_t s);
+                        int scoring, int32_t* ids, float* w, DevStatus* st, ZeroSpan zero, cudaStream_t s);
 
 // Permutation.
 int permute_num_blocks(int T, int k);
@@ -111,6 +147,10 @@ cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* cou
 cudaError_t launch_combine(const float* o, const float* topk_w, const int32_t* inv_perm, const float* shared,
                            int T, int H, int k, int rows, int nsplit, size_t split_stride, uint16_t* y, DevStatus* st,
                            cudaStream_t s);
+
+// row_token[inv_perm[t, j]] = t for every slot, and the counters in `zero` cleared.
+cudaError_t launch_row_tokens(const int32_t* inv_perm, int T, int k, int32_t* row_token, ZeroSpan zero, DevStatus* st,
+                              cudaStream_t s);
 
 // h = bf16(silu(sum_s gate_s) * sum_s up_s) from K-split partial slabs [rows, 2I].
 cudaError_t launch_swiglu_reduce(const float* partials, int nsplit, size_t split_stride, int rows, int I, uint16_t* h,
@@ -145,7 +185,7 @@ int small_router_slabs(int H, int E);
 cudaError_t launch_router_small(const uint16_t* x, const float* w, const float* bias, int T, int H, int E, int k,
                                 int scoring, float* partial, unsigned int* arrivals, int32_t* ids, float* wout,
                                 int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
-                                DevStatus* st, cudaStream_t s);
+                                DevStatus* st, ZeroSpan zero, cudaStream_t s);
 
 cudaError_t launch_selftest_timeout(DevStatus* st, uint64_t timeout_ns, cudaStream_t s);
 

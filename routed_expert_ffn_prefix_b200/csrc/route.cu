@@ -131,7 +131,8 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
                                                              size_t split_stride, const float* __restrict__ bias,
                                                              int T, int E, int k, int scoring,
                                                              int32_t* __restrict__ ids, float* __restrict__ wout,
-                                                             DevStatus* st) {
+                                                             DevStatus* st, ZeroSpan zero) {
+  zero_span(zero);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kTopkWarps + warp;
   if (t >= T) return;
@@ -162,10 +163,10 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
 
 template <int EPL, int UNR, bool QUAD = false>
 cudaError_t launch_topk_t(const float* logits, int nsplit, size_t split_stride, const float* bias, int T, int E,
-                          int k, int scoring, int32_t* ids, float* w, DevStatus* st, cudaStream_t s) {
+                          int k, int scoring, int32_t* ids, float* w, DevStatus* st, ZeroSpan zero, cudaStream_t s) {
   auto kern = scoring == MOE_SCORE_SOFTMAX ? topk_kernel<EPL, UNR, QUAD, false> : topk_kernel<EPL, UNR, QUAD, true>;
   return launch_kernel(kern, dim3((T + kTopkWarps - 1) / kTopkWarps), dim3(kTopkWarps * 32), 0, s, logits, nsplit,
-                       split_stride, bias, T, E, k, scoring, ids, w, st);
+                       split_stride, bias, T, E, k, scoring, ids, w, st, zero);
 }
 
 
@@ -181,7 +182,8 @@ __global__ void __launch_bounds__(kSmallThreads) router_small_kernel(
     int E, int k, int scoring, int chunk, int hs, float* __restrict__ partial, unsigned int* arrivals,
     int32_t* __restrict__ ids,
     float* __restrict__ wout, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-    int32_t* __restrict__ sorted_ids, int32_t* __restrict__ inv_perm, DevStatus* st) {
+    int32_t* __restrict__ sorted_ids, int32_t* __restrict__ inv_perm, DevStatus* st, ZeroSpan zero) {
+  zero_span(zero);
   __shared__ RouterSmem<TT> rsm;
   __shared__ int32_t sel[kSmallMaxSlots];
   __shared__ int32_t cnt[kMaxExperts];
@@ -261,11 +263,11 @@ template <int TT, int EPL>
 cudaError_t launch_router_small_t(const uint16_t* x, const float* w, const float* bias, int T, int H, int E, int k,
                                   int scoring, float* partial, unsigned int* arrivals, int32_t* ids, float* wout,
                                   int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
-                                  DevStatus* st, cudaStream_t s) {
+                                  DevStatus* st, ZeroSpan zero, cudaStream_t s) {
   const SmallGrid g = small_grid(H, E);
   return launch_kernel(router_small_kernel<TT, EPL>, dim3(g.ncs, g.hs), dim3(kSmallThreads), 0, s,
                        reinterpret_cast<const __nv_bfloat16*>(x), w, bias, T, H, E, k, scoring, g.chunk, g.hs,
-                       partial, arrivals, ids, wout, counts, offsets, sorted_ids, inv_perm, st);
+                       partial, arrivals, ids, wout, counts, offsets, sorted_ids, inv_perm, st, zero);
 }
 
 // accumulators for 1, 4 or 16 tokens
@@ -300,23 +302,23 @@ cudaError_t launch_router_logits_fma(const uint16_t* x, const float* w, int T, i
 }
 
 cudaError_t launch_topk(const float* logits, int nsplit, size_t split_stride, const float* bias, int T, int E, int k,
-                        int scoring, int32_t* ids, float* w, DevStatus* st, cudaStream_t s) {
-  if (E <= 32) return launch_topk_t<1, 8>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
-  if (E <= 64) return launch_topk_t<2, 8>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
+                        int scoring, int32_t* ids, float* w, DevStatus* st, ZeroSpan zero, cudaStream_t s) {
+  if (E <= 32) return launch_topk_t<1, 8>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, zero, s);
+  if (E <= 64) return launch_topk_t<2, 8>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, zero, s);
   // E % 4 == 0 (and 16-byte aligned rows): each lane loads 4 experts per 16-byte load
   if (E % 4 == 0) {
     if (E <= 128)
-      return launch_topk_t<4, 8, true>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
+      return launch_topk_t<4, 8, true>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, zero, s);
     if (E <= 256)
-      return launch_topk_t<8, 4, true>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
+      return launch_topk_t<8, 4, true>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, zero, s);
     if (E <= 512)
-      return launch_topk_t<16, 4, true>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
-    return launch_topk_t<32, 2, true>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
+      return launch_topk_t<16, 4, true>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, zero, s);
+    return launch_topk_t<32, 2, true>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, zero, s);
   }
-  if (E <= 128) return launch_topk_t<4, 8>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
-  if (E <= 256) return launch_topk_t<8, 4>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
-  if (E <= 512) return launch_topk_t<16, 4>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
-  return launch_topk_t<32, 2>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, s);
+  if (E <= 128) return launch_topk_t<4, 8>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, zero, s);
+  if (E <= 256) return launch_topk_t<8, 4>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, zero, s);
+  if (E <= 512) return launch_topk_t<16, 4>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, zero, s);
+  return launch_topk_t<32, 2>(logits, nsplit, split_stride, bias, T, E, k, scoring, ids, w, st, zero, s);
 }
 
 int small_router_slabs(int H, int E) { return small_grid(H, E).hs; }
@@ -324,10 +326,10 @@ int small_router_slabs(int H, int E) { return small_grid(H, E).hs; }
 cudaError_t launch_router_small(const uint16_t* x, const float* w, const float* bias, int T, int H, int E, int k,
                                 int scoring, float* partial, unsigned int* arrivals, int32_t* ids, float* wout,
                                 int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
-                                DevStatus* st, cudaStream_t s) {
+                                DevStatus* st, ZeroSpan zero, cudaStream_t s) {
   if (T < 1 || T > kSmallRouterT || E % 4 != 0 || k > 64) return cudaErrorInvalidValue;
 #define MOE_SMALL_ARGS T, x, w, bias, T, H, E, k, scoring, partial, arrivals, ids, wout, counts, offsets, sorted_ids, \
-                       inv_perm, st, s
+                       inv_perm, st, zero, s
   if (E <= 64) return launch_router_small_e<2>(MOE_SMALL_ARGS);
   if (E <= 128) return launch_router_small_e<4>(MOE_SMALL_ARGS);
   if (E <= 256) return launch_router_small_e<8>(MOE_SMALL_ARGS);

@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.moe_abi_version() == 1
+    assert lib.moe_abi_version() == 2
     for code, name in moe.STATUS.items():
         assert lib.moe_status_string(code).decode().startswith(name)
 
@@ -48,7 +48,7 @@ def test_workspace_layout_is_ordered_and_aligned(lib):
     L = moe.workspace_layout(8192, 4096, 512, 1024, 10)
     offs = [L[n] for n in ("status", "topk_ids", "topk_w", "counts", "offsets", "sorted_token_ids",
                            "inv_perm", "block_hist", "logits", "router_split", "h", "o", "h_shared",
-                           "o_shared", "split", "fused", "total")]
+                           "o_shared", "split", "fused", "arrivals", "total")]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
     assert L["o"] - L["h"] >= 81920 * 1024 * 2          # h: [T*k, I] bf16
     assert L["h_shared"] - L["o"] >= 81920 * 4096 * 4   # o: [T*k, H] f32
@@ -56,7 +56,10 @@ def test_workspace_layout_is_ordered_and_aligned(lib):
     Ls = moe.workspace_layout(4096, 8192, 256, 2048, 8, 2048)
     assert Ls["split"] - Ls["o_shared"] >= 4096 * 8192 * 4
     # many tokens: no K split and no one-launch layer, so no partial slabs
-    assert L["total"] == L["fused"] == L["split"] and Ls["total"] == Ls["fused"] == Ls["split"]
+    assert L["arrivals"] == L["fused"] == L["split"] and Ls["arrivals"] == Ls["fused"] == Ls["split"]
+    # arrival counters of the combine in the down GEMM: one per token and 64 output columns
+    assert L["total"] - L["arrivals"] == 8192 * (4096 // 64) * 4
+    assert Ls["total"] - Ls["arrivals"] == 4096 * (8192 // 64) * 4
 
 
 def test_workspace_layout_reserves_k_split_slabs_for_one_token(lib):
@@ -66,7 +69,9 @@ def test_workspace_layout_reserves_k_split_slabs_for_one_token(lib):
     L = moe.workspace_layout(1, 4096, 256, 1536, 8)
     assert L["fused"] - L["split"] == max(3 * 8 * 3072, 2 * 8 * 4096) * 4
     # the one-launch layer (T <= 4): 8 K slices of gate/up (2 x I) and down (H) rows, f32
-    assert L["total"] - L["fused"] == 8 * 8 * (2 * 1536 + 4096) * 4
+    assert L["arrivals"] - L["fused"] == 8 * 8 * (2 * 1536 + 4096) * 4
+    # arrival counters: the K-split gate/up's (8 rows x 1536/32 chunks) outnumber the down's (1 x 4096/64)
+    assert L["total"] - L["arrivals"] == 256 * ((8 * 1536 // 32 * 4 + 255) // 256)
     # the router's partial slabs: one per H slice of the few-token router
     assert L["router_split"] - L["logits"] >= 4 * 1 * 256 * 4
 

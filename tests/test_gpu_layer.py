@@ -206,6 +206,39 @@ def test_forward_bitwise_deterministic():
     assert torch.equal(ys[0], ys[1]) and torch.equal(ys[2], ys[3])
 
 
+def arrivals_zero(ws, cfg):
+    import torch
+    lay = moe.workspace_layout(cfg.T, cfg.H, cfg.E, cfg.I, cfg.k, cfg.I_s)
+    torch.cuda.synchronize()
+    return bool((ws[lay["arrivals"]:lay["total"]] == 0).all().item())
+
+
+@pytest.mark.parametrize("tiles", [moe.TILES_AUTO, moe.TILES_SMALL, moe.TILES_LARGE, moe.TILES_PAIR])
+@pytest.mark.parametrize("name", list(CASES))
+def test_fused_combine_bitwise_equals_separate_kernels(name, tiles):
+    """The combine in the down GEMM's epilogue (and, for a K split, the slab
+    sum + SwiGLU in the gate/up GEMM's) sums in the same order as the
+    separate kernels, so y is bitwise the same whichever warp finishes a
+    token; two fused calls in a row agree, and the arrival counters are
+    back at zero after each call."""
+    import torch
+    cfg, inp, ref = case(name)
+    d = dev_inputs(inp)
+    ws = workspace(cfg)
+    args = (d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws,
+            d["w_sh_gate_up"], d["w_sh_down"])
+    sep = moe.forward(*args, tiles=tiles, combine=moe.COMBINE_SEPARATE).cpu()
+    assert_ok(ws)
+    fused = []
+    for _ in range(2):
+        info = {}
+        fused.append(moe.forward(*args, tiles=tiles, combine=moe.COMBINE_FUSED, info=info).cpu())
+        assert_ok(ws)
+        assert arrivals_zero(ws, cfg)
+    assert torch.equal(fused[0], sep) and torch.equal(fused[1], sep)
+    assert_close_output(host_f64(fused[0]), ref["y"])
+
+
 def test_few_token_router_repeated_calls():
     """The one-launch router's last-block counter returns to zero after each
     launch: back-to-back calls (also through the whole layer) stay correct
@@ -238,9 +271,15 @@ def test_split_k_forward_bitwise_deterministic():
     ys = [moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws,
                       tiles=moe.TILES_SMALL, info=info).cpu() for _ in range(3)]
     assert_ok(ws)
-    assert info["launches"] == 5  # route+permute, gate/up, SwiGLU reduce, down, combine
+    assert info["launches"] == 4  # route+permute, gate/up (slab sum + SwiGLU in its epilogue), down, combine
     assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2])
     assert_close_output(host_f64(ys[0]), ref["y"])
+    moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws,
+                tiles=moe.TILES_SMALL, info=info, combine=moe.COMBINE_FUSED)
+    assert info["launches"] == 3  # route+permute, gate/up, down + combine in its epilogue
+    moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws,
+                tiles=moe.TILES_SMALL, info=info, combine=moe.COMBINE_SEPARATE)
+    assert info["launches"] == 5  # route+permute, gate/up, SwiGLU reduce, down, combine
 
 
 def test_fused_layer_one_launch_repeated_and_deterministic():
