@@ -87,11 +87,16 @@ enum {
   MOE_TILES_LARGE = 2,  /* <= 256 token rows per tile pass, 3-stage ring: prefill */
   MOE_TILES_PAIR = 3,   /* SM pairs (2-SM tcgen05 MMA): 256 weight columns per MMA, 128 per SM; <= 256
                            token rows per pass, half gathered by each SM; 4-stage ring: prefill */
-  MOE_TILES_FUSED = 4   /* moe_forward_ex only, T <= 4: the whole layer (routing, permutation, both
+  MOE_TILES_FUSED = 4,  /* moe_forward_ex only, T <= 4: the whole layer (routing, permutation, both
                            expert matrix-vector products, combine) in one cooperative launch with
                            grid barriers; CUDA-core weight streams.  Needs k <= 16, E % 4 == 0,
                            H, I, I_s multiples of 256, H <= 8192, I, I_s <= 4096.  Never chosen
                            by AUTO (measured slower than SMALL with its K split). */
+  MOE_TILES_PERSISTENT = 5 /* moe_forward_ex only, T <= 16, E % 4 == 0, no shared expert: the whole
+                              layer in one persistent launch on the tensor cores -- the few-token
+                              router, then the gate/up and the down grouped GEMM as one sequence of
+                              work units (a down unit starts once its expert's gate/up units are
+                              done), the weighted combine in the down GEMM's epilogue */
 };
 
 /* Router logits implementation. */

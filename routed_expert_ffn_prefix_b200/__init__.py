@@ -16,7 +16,7 @@ import os
 from . import build as _build
 
 __all__ = [
-    "MoEError", "lib", "TILES_AUTO", "TILES_SMALL", "TILES_LARGE", "TILES_PAIR", "TILES_FUSED",
+    "MoEError", "lib", "TILES_AUTO", "TILES_SMALL", "TILES_LARGE", "TILES_PAIR", "TILES_FUSED", "TILES_PERSISTENT",
     "ROUTER_AUTO", "ROUTER_FMA", "ROUTER_TC", "ROUTER_SMALL",
     "SCORE_SOFTMAX", "SCORE_SOFTMAX_SELECT_BIAS", "SCORE_SIGMOID",
     "COMBINE_AUTO", "COMBINE_FUSED", "COMBINE_SEPARATE",
@@ -25,7 +25,7 @@ __all__ = [
     "STATUS",
 ]
 
-TILES_AUTO, TILES_SMALL, TILES_LARGE, TILES_PAIR, TILES_FUSED = 0, 1, 2, 3, 4
+TILES_AUTO, TILES_SMALL, TILES_LARGE, TILES_PAIR, TILES_FUSED, TILES_PERSISTENT = 0, 1, 2, 3, 4, 5
 ROUTER_AUTO, ROUTER_FMA, ROUTER_TC, ROUTER_SMALL = 0, 1, 2, 3
 SCORE_SOFTMAX, SCORE_SOFTMAX_SELECT_BIAS, SCORE_SIGMOID = 0, 1, 2
 COMBINE_AUTO, COMBINE_FUSED, COMBINE_SEPARATE = 0, 1, 2

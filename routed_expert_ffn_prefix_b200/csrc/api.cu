@@ -82,13 +82,25 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // kernel's 4 per 256.  A multiple of 64 words, so the region has no
 // alignment padding and the routing kernels zero all of it with 16-byte
 // stores.
+// The persistent few-token layer runs both GEMMs at once, so it takes the
+// gate/up counters, the down counters and one done-counter per expert and
+// gate/up column block side by side; the multi-kernel path uses the region from its start for each GEMM.
 inline int down_cnt_stride(int H) { return ((H + 511) / 512) * 8; }
+inline size_t gate_up_cnt_words(int T, int I, int k, const SplitPlan& sp) {
+  return sp.gate_up > 1 ? (size_t)T * k * (I / 128) * 4 : 0;
+}
+inline size_t down_cnt_words(int T, int H) { return (size_t)T * down_cnt_stride(H); }
 inline size_t arrival_words(int T, int H, int E, int I, int k) {
   const SplitPlan sp = split_plan(T, H, E, I, k, MOE_TILES_SMALL);
-  const size_t gu = sp.gate_up > 1 ? (size_t)T * k * (I / 128) * 4 : 0;
-  const size_t dn = (size_t)T * down_cnt_stride(H);
-  const size_t w = gu > dn ? gu : dn;
+  const size_t w = gate_up_cnt_words(T, I, k, sp) + down_cnt_words(T, H) + (size_t)E * (I / 128);
   return (w + 63) & ~size_t(63);
+}
+// K-split partial slabs (f32 elements) of the two GEMMs.
+inline size_t split_gate_up_elems(int T, int I, int k, const SplitPlan& sp) {
+  return sp.gate_up > 1 ? (size_t)sp.gate_up * T * k * 2 * I : 0;
+}
+inline size_t split_down_elems(int T, int H, int k, const SplitPlan& sp) {
+  return sp.down > 1 ? (size_t)sp.down * T * k * H : 0;
 }
 
 // ---------------------------------------------------------------- workspace
@@ -116,10 +128,9 @@ moe_workspace_layout_t make_layout(int T, int H, int E, int I, int k, int I_s) {
   L.h_shared = take((size_t)T * I_s * 2);
   L.o_shared = take(I_s > 0 ? (size_t)T * H * 4 : 0);
   // Sized for SMALL tiles, the only policy that splits K.
+  // gate/up slabs, then down slabs (the persistent few-token layer holds both at once)
   const SplitPlan sp = split_plan(T, H, E, I, k, MOE_TILES_SMALL);
-  const size_t gu = sp.gate_up > 1 ? (size_t)sp.gate_up * tk * 2 * I : 0;
-  const size_t dn = sp.down > 1 ? (size_t)sp.down * tk * H : 0;
-  L.split = take((gu > dn ? gu : dn) * 4);
+  L.split = take((split_gate_up_elems(T, I, k, sp) + split_down_elems(T, H, k, sp)) * 4);
   // slabs of the one-launch few-token layer
   size_t fused = 0;
   if (T <= kFusedMaxT && H > 0 && I > 0) {
@@ -323,16 +334,16 @@ moe_status_t run_route(const uint16_t* x, const float* w_router, const float* bi
   return cuda_status(launch_topk(logits, nsplit, (size_t)T * E, bias, T, E, k, scoring, ids, w, st, zero, s));
 }
 
-// nsplit > 1: K-split into partial slabs [nsplit][rows][2I] f32 at `partials`
-// (gate columns [0, I), up [I, 2I)), reduced into h either by the last slab
-// of each row chunk to land (arrivals != nullptr: zeroed counters, one per
-// row and 32-column chunk) or by a separate reduce + SwiGLU pass.
-moe_status_t run_swiglu(const uint16_t* x, int src_rows, const uint16_t* w_gate_up, const int32_t* offsets,
-                        const int32_t* row_index, int rows, int H, int E, int I, int tiles, uint16_t* h,
-                        DevStatus* st, const DeviceInfo& dev, cudaStream_t s, int nsplit = 1,
-                        float* partials = nullptr, uint32_t* arrivals = nullptr) {
-  CUtensorMap map;
-  if (!make_weight_map(&map, w_gate_up, 2ull * I, (uint64_t)H, (uint64_t)E)) return MOE_ERR_CUDA;
+// Arguments of the gate/up GEMM on single-SM tiles: units of 128
+// intermediate columns, the gate and the up tile of the same columns, SwiGLU
+// into h [rows, I] bf16.  With nsplit > 1 the units cover K slices and store
+// fp32 partial slabs [nsplit][rows][2I] at `partials` (gate columns [0, I),
+// up [I, 2I)); arrivals != nullptr (zeroed counters, one per row and
+// 32-column chunk) lets the last slab of each row chunk to land sum them and
+// write h in its epilogue.
+GemmArgs gate_up_args(const uint16_t* x, int src_rows, const int32_t* offsets, const int32_t* row_index, int rows,
+                      int H, int E, int I, uint16_t* h, DevStatus* st, int nsplit = 1, float* partials = nullptr,
+                      uint32_t* arrivals = nullptr) {
   GemmArgs a{};
   a.offsets = offsets;
   a.row_index = row_index;
@@ -356,12 +367,6 @@ moe_status_t run_swiglu(const uint16_t* x, int src_rows, const uint16_t* w_gate_
   a.split_stride = 0;
   a.status = st;
   a.timeout_ns = kDefaultTimeoutNs;
-  if (tiles == MOE_TILES_PAIR) {  // 256 intermediate columns per unit (128 per SM of the pair)
-    a.n_blocks = (I + 255) / 256;
-    a.col_stride = 256;
-    a.out_col_stride = 256;
-    return cuda_status(launch_grouped_gemm_pair(map, a, EPI_SWIGLU, dev.num_sms, s));
-  }
   if (nsplit > 1) {
     a.out = partials;
     a.ld_out = 2 * I;
@@ -375,8 +380,27 @@ moe_status_t run_swiglu(const uint16_t* x, int src_rows, const uint16_t* w_gate_
       a.arrive_target = nsplit;
       a.fin_out = h;
       a.fin_ld = I;
-      return cuda_status(launch_grouped_gemm(map, a, EPI_SWIGLU_SPLIT, tiles, dev.num_sms, s));
     }
+  }
+  return a;
+}
+
+moe_status_t run_swiglu(const uint16_t* x, int src_rows, const uint16_t* w_gate_up, const int32_t* offsets,
+                        const int32_t* row_index, int rows, int H, int E, int I, int tiles, uint16_t* h,
+                        DevStatus* st, const DeviceInfo& dev, cudaStream_t s, int nsplit = 1,
+                        float* partials = nullptr, uint32_t* arrivals = nullptr) {
+  CUtensorMap map;
+  if (!make_weight_map(&map, w_gate_up, 2ull * I, (uint64_t)H, (uint64_t)E)) return MOE_ERR_CUDA;
+  if (tiles == MOE_TILES_PAIR) {  // 256 intermediate columns per unit (128 per SM of the pair)
+    GemmArgs a = gate_up_args(x, src_rows, offsets, row_index, rows, H, E, I, h, st);
+    a.n_blocks = (I + 255) / 256;
+    a.col_stride = 256;
+    a.out_col_stride = 256;
+    return cuda_status(launch_grouped_gemm_pair(map, a, EPI_SWIGLU, dev.num_sms, s));
+  }
+  const GemmArgs a = gate_up_args(x, src_rows, offsets, row_index, rows, H, E, I, h, st, nsplit, partials, arrivals);
+  if (nsplit > 1) {
+    if (arrivals != nullptr) return cuda_status(launch_grouped_gemm(map, a, EPI_SWIGLU_SPLIT, tiles, dev.num_sms, s));
     MOE_TRY(cuda_status(launch_grouped_gemm(map, a, EPI_STORE_F32, tiles, dev.num_sms, s)));
     return cuda_status(launch_swiglu_reduce(partials, nsplit, a.split_stride, rows, I, h, s));
   }
@@ -390,19 +414,16 @@ struct CombineArgs {
   const float* topk_w;
   const float* shared;  // [T, H] f32 or nullptr
   uint16_t* y;
-  uint32_t* arrivals;  // zeroed, arrival_words() of them
+  uint32_t* arrivals;  // zeroed, down_cnt_stride(H) per token
   int T, k;
 };
 
-// o: fp32 rows; nsplit > 1: K-split into partial slabs [nsplit][rows][H].
-// comb != nullptr: the last of each token's k * nsplit row chunks to land
-// also writes that chunk of y.
-moe_status_t run_down(const uint16_t* h, const uint16_t* w_down, const int32_t* offsets, int rows, int H, int E,
-                      int I, int tiles, float* o, DevStatus* st, const DeviceInfo& dev, cudaStream_t s,
-                      int nsplit = 1, const CombineArgs* comb = nullptr) {
-  CUtensorMap map;
-  if (!make_weight_map(&map, w_down, (uint64_t)H, (uint64_t)I, (uint64_t)E)) return MOE_ERR_CUDA;
-  const int cols = 128 * gemm_tiles_per_unit(tiles, EPI_STORE_F32);  // output columns per work unit
+// Arguments of the down GEMM on single-SM tiles: units of 256 output
+// columns (two 128-column tiles), fp32 rows o [rows, H]; nsplit > 1: K slices
+// into partial slabs [nsplit][rows][H] at o.  comb != nullptr: the last of
+// each token's k * nsplit row chunks to land also writes that chunk of y.
+GemmArgs down_args(const uint16_t* h, const int32_t* offsets, int rows, int H, int E, int I, float* o, DevStatus* st,
+                   int nsplit = 1, const CombineArgs* comb = nullptr) {
   GemmArgs a{};
   a.offsets = offsets;
   a.row_index = nullptr;
@@ -413,12 +434,12 @@ moe_status_t run_down(const uint16_t* h, const uint16_t* w_down, const int32_t* 
   a.K = I;
   a.krep = 1;
   a.a_dim2_rep = 0;
-  a.n_blocks = H / cols;
-  a.col_stride = cols;
+  a.n_blocks = H / 256;
+  a.col_stride = 256;
   a.col1_off = 128;
   a.out = o;
   a.ld_out = H;
-  a.out_col_stride = cols;
+  a.out_col_stride = 256;
   a.out_col1_off = 128;
   a.n_valid = H;
   a.rows_cap = rows;
@@ -426,9 +447,7 @@ moe_status_t run_down(const uint16_t* h, const uint16_t* w_down, const int32_t* 
   a.split_stride = nsplit > 1 ? (size_t)rows * H : 0;
   a.status = st;
   a.timeout_ns = kDefaultTimeoutNs;
-  int epi = EPI_STORE_F32;
   if (comb != nullptr) {
-    epi = EPI_DOWN_COMBINE;
     a.arrivals = comb->arrivals;
     a.cnt_stride = down_cnt_stride(H);
     a.arrive_target = comb->k * nsplit;
@@ -441,6 +460,16 @@ moe_status_t run_down(const uint16_t* h, const uint16_t* w_down, const int32_t* 
     a.topk = comb->k;
     a.n_tokens = comb->T;
   }
+  return a;
+}
+
+moe_status_t run_down(const uint16_t* h, const uint16_t* w_down, const int32_t* offsets, int rows, int H, int E,
+                      int I, int tiles, float* o, DevStatus* st, const DeviceInfo& dev, cudaStream_t s,
+                      int nsplit = 1, const CombineArgs* comb = nullptr) {
+  CUtensorMap map;
+  if (!make_weight_map(&map, w_down, (uint64_t)H, (uint64_t)I, (uint64_t)E)) return MOE_ERR_CUDA;
+  GemmArgs a = down_args(h, offsets, rows, H, E, I, o, st, nsplit, comb);
+  const int epi = comb != nullptr ? EPI_DOWN_COMBINE : EPI_STORE_F32;
   if (tiles == MOE_TILES_PAIR) {  // 2 x 256 output columns per unit (128 of each per SM of the pair)
     if (nsplit > 1) return MOE_ERR_INVALID_ARG;
     a.n_blocks = (H + 511) / 512;
@@ -630,7 +659,7 @@ moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const floa
   const int scoring = options ? options->scoring : MOE_SCORE_SOFTMAX;
   const int combine = options ? options->combine : MOE_COMBINE_AUTO;
   if (combine < MOE_COMBINE_AUTO || combine > MOE_COMBINE_SEPARATE) return MOE_ERR_INVALID_ARG;
-  if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_FUSED) return MOE_ERR_INVALID_ARG;
+  if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_PERSISTENT) return MOE_ERR_INVALID_ARG;
   if (router_impl < MOE_ROUTER_AUTO || router_impl > MOE_ROUTER_SMALL) return MOE_ERR_INVALID_ARG;
   if (!valid_scoring(scoring)) return MOE_ERR_INVALID_ARG;
   if (!all_aligned(x, w_router, w_gate_up, w_down, y) || (bias && !aligned16(bias))) return MOE_ERR_ALIGNMENT;
@@ -672,6 +701,49 @@ moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const floa
                                             shared ? I_s : 0, T, H, E, I, k,
                                             at<float>(ws, L.logits), gslabs, dslabs, ids, tw, counts, offs, sids, inv,
                                             y, st, kDefaultTimeoutNs, dev.num_sms, s)));
+    for (int i = 1; i < 7; ++i) MOE_TRY(mark(i));
+    if (options) options->launches = 1;
+    return MOE_OK;
+  }
+
+  // A few tokens, on request: the whole layer in one persistent launch on the tensor cores.
+  if (tile_policy == MOE_TILES_PERSISTENT) {
+    if (!layer_small_supported(T, E, shared ? I_s : 0)) return MOE_ERR_INVALID_ARG;
+    if (router_impl != MOE_ROUTER_AUTO && router_impl != MOE_ROUTER_SMALL) return MOE_ERR_INVALID_ARG;
+    const SplitPlan sp = split_plan(T, H, E, I, k, MOE_TILES_SMALL);
+    CUtensorMap gmap, dmap;
+    if (!make_weight_map(&gmap, w_gate_up, 2ull * I, (uint64_t)H, (uint64_t)E) ||
+        !make_weight_map(&dmap, w_down, (uint64_t)H, (uint64_t)I, (uint64_t)E))
+      return MOE_ERR_CUDA;
+    uint32_t* arr = at<uint32_t>(ws, L.arrivals);
+    const size_t gu_cnt = gate_up_cnt_words(T, I, k, sp), dn_cnt = down_cnt_words(T, H);
+    float* gu_slabs = at<float>(ws, L.split);
+    float* dn_slabs = gu_slabs + split_gate_up_elems(T, I, k, sp);
+    LayerParams p{};
+    p.x = x;
+    p.w_router = w_router;
+    p.bias = bias;
+    p.scoring = scoring;
+    p.T = T;
+    p.H = H;
+    p.E = E;
+    p.k = k;
+    p.partial = at<float>(ws, L.logits);
+    p.ids = ids;
+    p.counts = counts;
+    p.offsets = offs;
+    p.sids = sids;
+    p.inv = inv;
+    p.tw = tw;
+    p.expert_done = arr + gu_cnt + dn_cnt;
+    p.zero = ZeroSpan{reinterpret_cast<uint4*>(arr), (int)(arrival_words(T, H, E, I, k) / 4)};
+    p.gu = gate_up_args(x, T, offs, sids, rows, H, E, I, h, st, sp.gate_up, gu_slabs, arr);
+    const CombineArgs comb{sids, inv, tw, nullptr, y, arr + gu_cnt, T, k};
+    p.dn = down_args(h, offs, rows, H, E, I, sp.down > 1 ? dn_slabs : o, st, sp.down, &comb);
+    p.st = st;
+    p.timeout_ns = kDefaultTimeoutNs;
+    MOE_TRY(mark(0));
+    MOE_TRY(cuda_status(launch_layer_small(gmap, dmap, p, dev.num_sms, s)));
     for (int i = 1; i < 7; ++i) MOE_TRY(mark(i));
     if (options) options->launches = 1;
     return MOE_OK;

@@ -21,7 +21,8 @@ struct DevStatus {
   int32_t aux;
   uint32_t arrivals;  // block counter of the few-token router: zero between its launches
   uint32_t grid_bar;  // grid-barrier counter of the one-launch few-token layer: zero between launches
-  uint32_t reserved[3];
+  uint32_t exits;     // persistent few-token layer: blocks done; zero between launches
+  uint32_t reserved[2];
 };
 
 // Where an error was raised (DevStatus::site).
@@ -37,6 +38,7 @@ enum Site : int32_t {
   SITE_SELFTEST = 8,
   SITE_TOPK = 9,
   SITE_FUSED = 10,
+  SITE_LAYER = 11,
 };
 
 __device__ __forceinline__ void raise_error(DevStatus* st, int code, int site, int aux) {
@@ -55,6 +57,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 // ---------------------------------------------------------------- mbarrier

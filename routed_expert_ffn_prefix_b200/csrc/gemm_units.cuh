@@ -14,17 +14,22 @@ namespace moe {
 
 constexpr int kBK = 64;  // k per pipeline stage (one 128-byte swizzle row of bf16)
 
+
 struct Unit {
   int group, nb, row0, rows, ks, kb, ke;  // ks: K split; [kb, ke): its k-steps (of kBK)
   int passes;                             // row passes of this group (units re-streaming the same weights)
 };
 
-__device__ __forceinline__ int group_rows_begin(const GemmArgs& a, int g) {
-  return a.offsets ? __ldg(a.offsets + g) : 0;
-}
-__device__ __forceinline__ int group_rows_end(const GemmArgs& a, int g) {
-  return a.offsets ? __ldg(a.offsets + g + 1) : a.single_rows;
-}
+// Routing metadata (offsets, row indices, slot rows and weights) is read
+// with generic loads, never the read-only path: the persistent few-token
+// layer computes it in the same launch and keeps it in each block's shared
+// memory.
+
+// The unit prefix of a GEMM in shared memory: ustart[g] (g < ngroups) is the
+// first unit of group g; ustart[kPrefixRows + g] (g <= ngroups) the first
+// permuted row of group g, so decoding a unit reads no global memory.
+constexpr int kPrefixRows = kMaxExperts + 1;
+constexpr int kPrefixInts = 2 * kPrefixRows;
 
 template <int NT>
 __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, const int* ustart, int ngroups, int u) {
@@ -34,7 +39,7 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, const int* ustart
     if (ustart[mid] <= u) lo = mid; else hi = mid - 1;
   }
   const int g = lo;
-  const int b = group_rows_begin(a, g), e = group_rows_end(a, g);
+  const int b = ustart[kPrefixRows + g], e = ustart[kPrefixRows + g + 1];
   const int passes = (e - b + NT - 1) / NT;
   const int S = a.k_splits;
   const int local = u - ustart[g];
@@ -53,16 +58,40 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, const int* ustart
   return r;
 }
 
-// Warp 0: per-group unit counts -> exclusive prefix in shared memory, with
-// the row ranges checked.  Returns the total unit count (0 on bad metadata).
+// One warp: per-group unit counts -> exclusive prefix and the groups' row
+// ranges in shared memory (kPrefixInts ints at ustart), with the ranges
+// checked.  The group boundaries come from `soffsets` (shared memory, when
+// the caller already holds them) or else from a.offsets in global memory,
+// all loaded at once (one round trip, not one per group).  Returns the total
+// unit count in *total_out (0 on bad metadata).
 template <int NT>
-__device__ void build_unit_prefix(const GemmArgs& a, int ngroups, int* ustart, int* total_out) {
+__device__ void build_unit_prefix(const GemmArgs& a, int ngroups, int* ustart, int* total_out,
+                                  const int* soffsets = nullptr) {
   const int lane = lane_id();
+  int* rbeg = ustart + kPrefixRows;
+  constexpr int kPer = (kPrefixRows + 31) / 32;
+  int v[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int i = lane + 32 * j;
+    v[j] = 0;
+    if (i <= ngroups) {
+      if (soffsets != nullptr) v[j] = soffsets[i];
+      else if (a.offsets != nullptr) v[j] = __ldcg(a.offsets + i);
+      else v[j] = i == 0 ? 0 : a.single_rows;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int i = lane + 32 * j;
+    if (i <= ngroups) rbeg[i] = v[j];
+  }
+  __syncwarp();
   const int per = (ngroups + 31) / 32;
   const int g0 = min(ngroups, lane * per), g1 = min(ngroups, g0 + per);
   int sum = 0, bad = -1;
   for (int g = g0; g < g1; ++g) {
-    const int b = group_rows_begin(a, g), e = group_rows_end(a, g);
+    const int b = rbeg[g], e = rbeg[g + 1];
     if (b < 0 || e < b || e > a.rows_cap) bad = g;
     ustart[g] = sum;
     sum += (e > b && bad < 0) ? ((e - b + NT - 1) / NT) * a.n_blocks * a.k_splits : 0;
@@ -70,8 +99,8 @@ __device__ void build_unit_prefix(const GemmArgs& a, int ngroups, int* ustart, i
   int incl = sum;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, d);
-    if (lane >= d) incl += v;
+    const int w = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += w;
   }
   const int base = incl - sum;
   for (int g = g0; g < g1; ++g) ustart[g] += base;
@@ -84,6 +113,7 @@ __device__ void build_unit_prefix(const GemmArgs& a, int ngroups, int* ustart, i
       *total_out = incl;
     }
   }
+  __syncwarp();
 }
 
 // silu(g) = g * sigmoid(g); h is rounded to bf16 right after, so the fast
@@ -142,12 +172,12 @@ __device__ __forceinline__ void finish_combine_row(const GemmArgs& a, int t, con
   int ra = 0, rb = 0;
   float wa = 0.f, wb = 0.f;
   if (lane < k) {
-    ra = __ldg(a.inv_perm + (size_t)t * k + lane);
-    wa = __ldg(a.topk_w + (size_t)t * k + lane);
+    ra = a.inv_perm[(size_t)t * k + lane];
+    wa = a.topk_w[(size_t)t * k + lane];
   }
   if (lane + 32 < k) {
-    rb = __ldg(a.inv_perm + (size_t)t * k + lane + 32);
-    wb = __ldg(a.topk_w + (size_t)t * k + lane + 32);
+    rb = a.inv_perm[(size_t)t * k + lane + 32];
+    wb = a.topk_w[(size_t)t * k + lane + 32];
   }
   const bool bad = (lane < k && (ra < 0 || ra >= a.rows_cap)) || (lane + 32 < k && (rb < 0 || rb >= a.rows_cap));
   if (__any_sync(0xffffffffu, bad)) {
@@ -206,7 +236,7 @@ __device__ __forceinline__ void finish_combine_row(const GemmArgs& a, int t, con
   for (int i = 0; i < MT; ++i) {
     if (live[i]) {
       float v = acc[i];
-      if (a.shared) v += __ldg(a.shared + (size_t)t * a.ld_out + cols[i]);
+      if (a.shared) v += __ldcg(a.shared + (size_t)t * a.ld_out + cols[i]);
       y[cols[i]] = __float2bfloat16_rn(v);
     }
   }
@@ -228,7 +258,7 @@ __device__ __forceinline__ void arrive_rows(const GemmArgs& a, int r0, int nr, i
     const int r = r0 + lane;
     key = r;
     if constexpr (EPI == EPI_DOWN_COMBINE) {
-      key = __ldg(a.row_token + r);
+      key = a.row_token[r];
       if (key < 0 || key >= a.n_tokens) {
         raise_error(a.status, MOE_ERR_DEVICE_BOUNDS, SITE_GEMM_EPILOGUE, r);
         key = -1;

@@ -36,297 +36,35 @@
 //
 // Warp roles (416 threads): warps 0-7 epilogue, warps 8-11 producers,
 // warp 12 TMEM allocation + MMA issue.
-#include "gemm_units.cuh"
+#include "gemm_pipeline.cuh"
 
 namespace moe {
 
 namespace {
 
-constexpr int kEpiWarps = 8;
-constexpr int kProdWarps = 4;
-constexpr int kMmaWarp = kEpiWarps + kProdWarps;
-constexpr int kThreads = (kMmaWarp + 1) * 32;
-constexpr int kProdThreads = kProdWarps * 32;
-constexpr int kEpiThreads = kEpiWarps * 32;
-template <int NT, int ST, int MT, int BK>
-struct Cfg {
-  // A stage holds BK of K: MT weight tiles of 128 columns (two 64-column TMA
-  // boxes each, MN-major) and NT token rows (K-major, BK*2 bytes per row).
-  static constexpr int ROW_BYTES = BK * 2;
-  static constexpr int BOX_BYTES = 64 * BK * 2;
-  static constexpr int ATILE_BYTES = 2 * BOX_BYTES;
-  static constexpr int CHUNKS = ROW_BYTES / 16;  // 16-byte chunks per token row
-  static constexpr uint32_t ROW_LAYOUT = BK == 64 ? kLayoutSw128 : kLayoutSw64;
-  static constexpr uint32_t ROW_SBO = 8 * ROW_BYTES;  // one swizzle atom = 8 rows
-  static constexpr int SUB = kBK / BK;  // stages per 64-wide k-step of the unit schedule
-  static constexpr int B_BYTES = NT * ROW_BYTES;
-  static constexpr int A_BYTES = MT * ATILE_BYTES;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int NBUF = (2 * MT * NT <= 512) ? 2 : 1;
-  static constexpr int ACC_COLS = NBUF * MT * NT;
-  static constexpr int TMEM_COLS = ACC_COLS <= 32 ? 32 : ACC_COLS <= 64 ? 64 : ACC_COLS <= 128 ? 128
-                                   : ACC_COLS <= 256 ? 256 : 512;
-  // ring + barriers/flags (256) + unit prefix (kMaxExperts+1 ints) + alignment slack
-  static constexpr int SMEM_BYTES = ST * STAGE_BYTES + 256 + 4 * (kMaxExperts + 1) + 1024;
-  static_assert(NT % 32 == 0 && NT >= 32 && NT <= 256, "row pass must be 32..256, multiple of 32");
-  static_assert(MT == 1 || MT == 2, "one or two MMA tiles per unit");
-  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte swizzle alignment");
-  static_assert(BK == 64 || BK == 32, "stage depth: one 128-byte or 64-byte swizzle row");
-};
-
-// Physical 16-byte chunk of logical chunk `chunk` in row `row` of a K-major
-// tile: the swizzle XORs the chunk index with row bits (128-byte: row % 8;
-// 64-byte: (row / 2) % 4), matching what the MMA descriptor expects.
-template <int BK>
-__device__ __forceinline__ int swizzled_chunk(int chunk, int row) {
-  return BK == 64 ? (chunk ^ (row & 7)) : (chunk ^ ((row >> 1) & 3));
-}
-
 template <int NT, int ST, int MT, int EPI, int BK>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap wmap, const GemmArgs a) {
-  using C = Cfg<NT, ST, MT, BK>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * C::STAGE_BYTES);
-  uint64_t* empty = full + ST;
-  uint64_t* tfull = empty + ST;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* mma_done = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
-  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-  int* total_units = abort_flag + 1;
-  int* ustart = reinterpret_cast<int*>(smem + ST * C::STAGE_BYTES + 256);
-
+  const PipeSmem<NT, ST, MT, BK> sm = PipeSmem<NT, ST, MT, BK>::carve(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ngroups = a.offsets ? a.groups : 1;
-
-  if (tid == 0) {
-    for (int s = 0; s < ST; ++s) {
-      mbar_init(full + s, kProdThreads + 1);  // producer cp.async arrivals + 1 expect_tx arrival
-      mbar_init(empty + s, 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(tfull + b, 1);
-      mbar_init(tempty + b, kEpiThreads);
-    }
-    mbar_init(mma_done, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == kMmaWarp) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
-  }
+  sm.init(tid, warp);
   if (warp == kEpiWarps && lane == 0) prefetch_tmap(&wmap);
-  if (warp == 0) build_unit_prefix<NT>(a, ngroups, ustart, total_units);
+  if (warp == 0) build_unit_prefix<NT>(a, ngroups, sm.ustart, sm.total_units);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const int total = *total_units;
-
-  if (warp >= kEpiWarps && warp < kMmaWarp) {
-    // ------------------------------------------------------------ producers
-    const WaitCtx wc{a.status, abort_flag, a.timeout_ns, SITE_GEMM_PRODUCER};
-    const int pt = tid - kEpiThreads;
-    const int chunk = pt % C::CHUNKS, rsub = pt / C::CHUNKS;  // 16-byte chunk of a row; first row
-    constexpr int kRowStep = kProdThreads / C::CHUNKS;
-    constexpr int kRowsPerThread = NT / kRowStep;
-    // Weight tiles are streamed past L2 (evict-first): keeping them (even for
-    // groups with several row passes) measured slower, because it displaces
-    // the token rows, which every column block of the group reads again.
-    const uint64_t pol_w = policy_evict_first();
-    const uint64_t pol_rows = a.rows_evict_last ? policy_evict_last() : policy_evict_normal();
-    const __nv_bfloat16* bsrc = reinterpret_cast<const __nv_bfloat16*>(a.b_src);
-    int stage = 0;
-    uint32_t phase = 0;
-    uint32_t issued_mask = 0, issued_par = 0;  // per stage: loads issued / parity of the last issue
-    bool ok = true;
-    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-      const Unit un = decode_unit<NT>(a, ustart, ngroups, u);
-      int src[kRowsPerThread];
-#pragma unroll
-      for (int i = 0; i < kRowsPerThread; ++i) {
-        const int c = rsub + kRowStep * i;
-        int sr = -1;
-        if (c < un.rows) {
-          const int r = un.row0 + c;
-          sr = a.row_index ? __ldg(a.row_index + r) : r;
-          if (sr < 0 || sr >= a.src_rows) {
-            raise_error(a.status, MOE_ERR_DEVICE_BOUNDS, SITE_GEMM_GATHER, r);
-            sr = -1;
-          }
-        }
-        src[i] = sr;
-      }
-      const int col0 = un.nb * a.col_stride;
-      const int nk = (un.ke - un.kb) * C::SUB, kiters = nk * a.krep;  // stages per repeat, total
-      for (int it = 0; it < kiters; ++it) {
-        const int rep = it / nk;
-        const int k0 = un.kb * kBK + (it - rep * nk) * BK;
-        if (!mbar_wait(&empty[stage], phase ^ 1u, wc, 100 + stage)) { ok = false; break; }
-        uint8_t* sA = smem + stage * C::STAGE_BYTES;
-        const uint32_t sB = smem_u32(sA + C::A_BYTES);
-#pragma unroll
-        for (int i = 0; i < kRowsPerThread; ++i) {
-          if (src[i] >= 0) {
-            const int c = rsub + kRowStep * i;
-            cp_async_16(sB + c * C::ROW_BYTES + (swizzled_chunk<BK>(chunk, c) << 4),
-                        bsrc + (size_t)src[i] * a.K + k0 + chunk * 8, pol_rows);
-          }
-        }
-        cp_async_arrive_noinc(&full[stage]);
-        if (pt == 0) {
-          mbar_arrive_expect_tx(&full[stage], C::A_BYTES);
-          const int d2 = a.a_dim2_rep ? rep : un.group;
-#pragma unroll
-          for (int t = 0; t < MT; ++t) {
-            const int c = col0 + t * a.col1_off;
-            tma_load_3d(sA + t * C::ATILE_BYTES, &wmap, &full[stage], c, k0, d2, pol_w);
-            tma_load_3d(sA + t * C::ATILE_BYTES + C::BOX_BYTES, &wmap, &full[stage], c + 64, k0, d2, pol_w);
-          }
-        }
-        issued_mask |= 1u << stage;
-        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-        if (++stage == ST) { stage = 0; phase ^= 1u; }
-      }
-    }
-    cp_async_wait_all();
-    if (!ok && pt == 0) {
-      // Aborted: let every load still in flight land before the block exits.
-      for (int s = 0; s < ST; ++s) {
-        if (!(issued_mask >> s & 1u)) continue;
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(&full[s], (issued_par >> s) & 1u) && globaltimer_ns() - t0 < a.timeout_ns) {
-        }
-      }
-    }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const WaitCtx wc{a.status, abort_flag, a.timeout_ns, SITE_GEMM_MMA};
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc_it = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-        const Unit un = decode_unit<NT>(a, ustart, ngroups, u);
-        const int buf = C::NBUF == 2 ? (acc_it & 1) : 0;
-        const uint32_t apar = C::NBUF == 2 ? ((acc_it >> 1) & 1) : (acc_it & 1);
-        if (!mbar_wait(&tempty[buf], apar ^ 1u, wc, 200 + buf)) break;
-        tc_fence_after();
-        const uint32_t d0 = tmem + buf * MT * NT;
-        const int N = (un.rows + 15) & ~15;
-        const uint32_t idesc = idesc_bf16_f32(128, N, /*A MN-major*/ true, /*B K-major*/ false);
-        const int kiters = (un.ke - un.kb) * C::SUB * a.krep;
-        uint32_t acc = 0;
-        for (int it = 0; it < kiters; ++it) {
-          if (!mbar_wait(&full[stage], phase, wc, 300 + stage)) { ok = false; break; }
-          tc_fence_after();
-          fence_proxy_async_smem();
-          const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
-          const uint32_t sB = sA + C::A_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            // B (rows, K-major): +16 k = 32 B inside the swizzled row.
-            const uint64_t bd = smem_desc(sB + kk * 32, 16, C::ROW_SBO, C::ROW_LAYOUT);
-#pragma unroll
-            for (int t = 0; t < MT; ++t) {
-              // A (weights, MN-major): +16 k = two 8-row groups = 2048 B; the two
-              // 64-column halves of a tile sit one TMA box apart.
-              const uint64_t ad = smem_desc_sw128(sA + t * C::ATILE_BYTES + kk * 2048, C::BOX_BYTES, 1024);
-              mma_bf16(d0 + t * NT, ad, bd, idesc, acc);
-            }
-            acc = 1;
-          }
-          mma_commit(&empty[stage]);
-          if (++stage == ST) { stage = 0; phase ^= 1u; }
-        }
-        if (!ok) break;
-        mma_commit(&tfull[buf]);
-        ++acc_it;
-      }
-      // Every MMA issued by this thread has finished once mma_done flips.
-      mma_commit(mma_done);
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(mma_done, 0) && globaltimer_ns() - t0 < a.timeout_ns) {
-      }
-    }
-    __syncwarp();
-  } else {
-    // ------------------------------------------------------------ epilogue (warps 0-7)
-    // Warp w reads TMEM lanes 32*(w%4).. (one weight column per thread) and
-    // handles the 32-row chunks c0 = 32*(w/4) + 64*j of the unit's rows.
-    const WaitCtx wc{a.status, abort_flag, a.timeout_ns, SITE_GEMM_EPILOGUE};
-    const int quarter = warp & 3, half = warp >> 2;
-    int acc_it = 0;
-    for (int u = blockIdx.x; u < total; u += gridDim.x) {
-      const Unit un = decode_unit<NT>(a, ustart, ngroups, u);
-      const int buf = C::NBUF == 2 ? (acc_it & 1) : 0;
-      const uint32_t apar = C::NBUF == 2 ? ((acc_it >> 1) & 1) : (acc_it & 1);
-      if (!mbar_wait(&tfull[buf], apar, wc, 400 + buf)) break;
-      tc_fence_after();
-      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * MT * NT;
-      const int col = un.nb * a.out_col_stride + quarter * 32 + lane;
-      for (int c0 = half * 32; c0 < un.rows; c0 += 64) {
-        const int nr = min(32, un.rows - c0);
-        if (EPI == EPI_SWIGLU) {
-          float g[32], v[32];
-          tmem_ld_4x16(tbase + c0, tbase + c0 + 16, tbase + NT + c0, tbase + NT + c0 + 16, g, g + 16, v, v + 16);
-          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
-          if (col < a.n_valid) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (j < nr)
-                out[(size_t)(un.row0 + c0 + j) * a.ld_out + col] = __float2bfloat16_rn(silu_f(g[j]) * v[j]);
-            }
-          }
-        } else {  // fp32 rows (EPI_STORE_F32, and the slabs / rows of the last-arriver reductions)
-          // both tiles' 32 rows in one batch of TMEM loads (one wait), then the stores
-          float v[MT][32];
-          if constexpr (MT == 2) {
-            tmem_ld_4x16(tbase + c0, tbase + c0 + 16, tbase + NT + c0, tbase + NT + c0 + 16, v[0], v[0] + 16, v[1],
-                         v[1] + 16);
-          } else {
-            tmem_ld_2x16(tbase + c0, tbase + c0 + 16, v[0], v[0] + 16);
-          }
-#pragma unroll
-          for (int t = 0; t < MT; ++t) {
-            const int ct = col + t * a.out_col1_off;
-            if (ct < a.n_valid) {
-              float* out = reinterpret_cast<float*>(a.out) + (size_t)un.ks * a.split_stride;
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (j < nr) out[(size_t)(un.row0 + c0 + j) * a.ld_out + ct] = v[t][j];
-            }
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&tempty[buf]);
-      ++acc_it;
-      if constexpr (EPI == EPI_SWIGLU_SPLIT || EPI == EPI_DOWN_COMBINE) {
-        // TMEM is released; now count this warp's stored rows and reduce the
-        // chunks they complete while the next unit's MMAs run.
-        __syncwarp();
-        __threadfence();
-        int cols[MT];
-        cols[0] = col;
-        if constexpr (MT == 2) cols[1] = col + a.out_col1_off;
-        const int chunk = un.nb * 4 + quarter;
-        for (int c0 = half * 32; c0 < un.rows; c0 += 64)
-          arrive_rows<MT, EPI>(a, un.row0 + c0, min(32, un.rows - c0), chunk, cols);
-      }
-    }
-  }
-
+  const uint32_t tmem = *sm.tmem_slot;
+  const OnePhase<NT> sched{&a, &wmap, sm.ustart, ngroups};
+  gemm_roles<NT, ST, MT, BK, EPI, EPI>(sm, sched, tmem, blockIdx.x, gridDim.x, *sm.total_units, a.status,
+                                       a.timeout_ns);
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    tmem_dealloc(tmem, Cfg<NT, ST, MT, BK>::TMEM_COLS);
   }
 }
 
@@ -339,7 +77,7 @@ cudaError_t launch_cfg(const CUtensorMap& wmap, const GemmArgs& a, int num_sms, 
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (err != cudaSuccess) return err;
-  return launch_kernel(kern, dim3(num_sms), dim3(kThreads), C::SMEM_BYTES, stream, wmap, a);
+  return launch_kernel(kern, dim3(num_sms), dim3(kGemmThreads), C::SMEM_BYTES, stream, wmap, a);
 }
 
 }  // namespace

@@ -58,7 +58,7 @@ struct PCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int NBUF = (2 * MT * NT <= 512) ? 2 : 1;  // accumulators double-buffered if they fit
   static constexpr int TMEM_COLS = 512;
-  static constexpr int SMEM_BYTES = ST * STAGE_BYTES + 512 + 4 * (kMaxExperts + 1) + 1024;
+  static constexpr int SMEM_BYTES = ST * STAGE_BYTES + 512 + 4 * kPrefixInts + 1024;
   static_assert(NT % 32 == 0 && NT >= 32 && NT <= 256, "row pass must be 32..256, multiple of 32");
   static_assert(MT == 1 || MT == 2, "one or two MMA tiles per unit");
   static_assert(MT * NT * NBUF <= TMEM_COLS, "accumulators must fit in TMEM");

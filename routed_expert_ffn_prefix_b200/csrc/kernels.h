@@ -187,6 +187,29 @@ cudaError_t launch_router_small(const uint16_t* x, const float* w, const float* 
                                 int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
                                 DevStatus* st, ZeroSpan zero, cudaStream_t s);
 
+// The whole layer for T <= kSmallRouterT tokens in one persistent launch on
+// the tensor cores (layer_small.cu): the few-token router, then the gate/up
+// and the down grouped GEMM as one sequence of work units, the combine in the
+// down GEMM's epilogue.  E % 4 == 0, no shared expert.
+struct LayerParams {
+  const uint16_t* x;
+  const float* w_router;
+  const float* bias;
+  int scoring;
+  int T, H, E, k;
+  float* partial;  // router partial slabs [small_router_slabs(H, E)][T][E]
+  int32_t *ids, *counts, *offsets, *sids, *inv;
+  float* tw;
+  uint32_t* expert_done;  // [E][I/128]: epilogue warps done with each gate/up column block of each expert
+  ZeroSpan zero;          // the arrival counters of both GEMMs and expert_done, cleared in the launch
+  GemmArgs gu, dn;        // the two GEMMs (gate/up: SwiGLU, or K-split slabs + SwiGLU; down: combine)
+  DevStatus* st;
+  uint64_t timeout_ns;
+};
+bool layer_small_supported(int T, int E, int I_s);
+cudaError_t launch_layer_small(const CUtensorMap& gu_map, const CUtensorMap& dn_map, const LayerParams& p,
+                               int num_sms, cudaStream_t s);
+
 cudaError_t launch_selftest_timeout(DevStatus* st, uint64_t timeout_ns, cudaStream_t s);
 
 }  // namespace moe

@@ -198,64 +198,9 @@ __global__ void __launch_bounds__(kSmallThreads) router_small_kernel(
   if (!is_last) return;
   __threadfence();
 
-  // ---- last block: slab sum in slab order, scoring, top-k (one warp per token)
-  for (int t = warp; t < T; t += kSmallThreads / 32)
-    router_select<EPL>(partial, hs, bias, T, E, k, scoring, t, ids + (size_t)t * k, wout + (size_t)t * k,
-                       sel + t * k, st);
-  if (counts != nullptr) {
-    // ---- permutation of the n = T*k slots, stable counting sort by expert
-    const int n = T * k;
-    for (int e = tid; e < E; e += kSmallThreads) cnt[e] = 0;
-    __syncthreads();
-    for (int s = tid; s < n; s += kSmallThreads) atomicAdd(&cnt[sel[s]], 1);
-    __syncthreads();
-    constexpr int EPT = kMaxExperts / kSmallThreads;  // experts per thread in the scan
-    int loc[EPT], tot = 0;
-#pragma unroll
-    for (int j = 0; j < EPT; ++j) {
-      const int e = tid * EPT + j;
-      loc[j] = e < E ? cnt[e] : 0;
-      tot += loc[j];
-    }
-    int incl = tot;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const int o = __shfl_up_sync(0xffffffffu, incl, d);
-      if (lane >= d) incl += o;
-    }
-    if (lane == 31) warp_sums[warp] = incl;
-    __syncthreads();
-    int base = incl - tot;
-    for (int v = 0; v < warp; ++v) base += warp_sums[v];
-#pragma unroll
-    for (int j = 0; j < EPT; ++j) {
-      const int e = tid * EPT + j;
-      if (e < E) {
-        counts[e] = loc[j];
-        offsets[e] = base;
-        cnt[e] = base;  // running position of expert e
-      }
-      base += loc[j];
-    }
-    if (tid == 0) offsets[E] = n;
-    __syncthreads();
-    if (warp == 0) {
-      for (int s0 = 0; s0 < n; s0 += 32) {
-        const int s = s0 + lane;
-        const int e = s < n ? sel[s] : -1;
-        const uint32_t peers = __match_any_sync(0xffffffffu, e);
-        const int rank = __popc(peers & ((1u << lane) - 1u));
-        const int pos = e >= 0 ? cnt[e] + rank : -1;
-        __syncwarp();
-        if (e >= 0 && rank == 0) cnt[e] += __popc(peers);
-        __syncwarp();
-        if (e >= 0) {
-          sorted_ids[pos] = s / k;
-          inv_perm[s] = pos;
-        }
-      }
-    }
-  }
+  // ---- last block: slab sum, scoring, top-k and (in the layer) the permutation
+  router_finish<EPL>(partial, hs, bias, T, E, k, scoring, ids, wout, counts, offsets, sorted_ids, inv_perm, st, sel,
+                     cnt, warp_sums);
   if (tid == 0) *arrivals = 0u;  // every block has arrived: ready for the next launch
 }
 

@@ -28,6 +28,17 @@ __device__ __forceinline__ bool topk_better(float av, int ai, float bv, int bi) 
   return av > bv || (av == bv && ai < bi);
 }
 
+// Non-NaN float -> unsigned integer with the same order (larger float,
+// larger integer; -0 taken as +0, as the float comparison does; -inf the
+// smallest value above 0), and back.  0 is left for "no candidate".
+__device__ __forceinline__ uint32_t ordered_key(float f) {
+  const uint32_t u = f == 0.f ? 0u : __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 // Expert held in entry i of a lane's EPL logits: scalar layout e = lane + 32 i;
 // quad layout (16-byte loads, E % 4 == 0) e = 128 (i / 4) + 4 lane + i % 4.
 template <bool QUAD>
@@ -57,7 +68,7 @@ __device__ __forceinline__ void warp_topk(const float (&vin)[EPL], const float (
     id[i] = ok ? e : kNoExpert;
   }
   float lead = 0.f, sum = 0.f;
-  float held0 = 0.f, held1 = 0.f;  // SEL: source values of slots lane and lane + 32
+  float held0 = 0.f, held1 = 0.f;  // values of slots lane and lane + 32 (SEL: sources; else numerators)
   for (int j = 0; j < k; ++j) {
     float tv[EPL];
     int ti[EPL];
@@ -68,14 +79,13 @@ __device__ __forceinline__ void warp_topk(const float (&vin)[EPL], const float (
 #pragma unroll
       for (int i = 0; i + w < EPL; i += 2 * w)
         if (topk_better(tv[i + w], ti[i + w], tv[i], ti[i])) { tv[i] = tv[i + w]; ti[i] = ti[i + w]; }
-    float bv = tv[0];
-    int bi = ti[0];
-#pragma unroll
-    for (int d = 16; d >= 1; d >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, d);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, d);
-      if (topk_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-    }
+    // The warp's best: the largest key by one warp reduction over an
+    // order-preserving unsigned encoding of the lanes' bests, then the lowest
+    // expert id among the lanes holding that key by a second one.
+    const uint32_t lane_key = ti[0] == kNoExpert ? 0u : ordered_key(tv[0]);
+    const uint32_t best_key = __reduce_max_sync(0xffffffffu, lane_key);
+    int bi = (int)__reduce_min_sync(0xffffffffu, lane_key == best_key ? (uint32_t)ti[0] : (uint32_t)kNoExpert);
+    float bv = key_value(best_key);
     if (bi == kNoExpert) {  // no candidate left: the keys were NaN
       if (lane == 0) raise_error(st, MOE_ERR_DEVICE_BOUNDS, SITE_TOPK, t);
       bi = 0;
@@ -103,9 +113,12 @@ __device__ __forceinline__ void warp_topk(const float (&vin)[EPL], const float (
       if (j == 0) lead = bv;
       const float z = expf(bv - lead);
       sum += z;
+      if (lane == (j & 31)) {  // slot j's numerator stays in a register of lane j % 32
+        if (j < 32) held0 = z;
+        else held1 = z;
+      }
       if (lane == 0) {
         idrow[j] = bi;
-        wrow[j] = z;
         if (sel) sel[j] = bi;
       }
     }
@@ -127,9 +140,9 @@ __device__ __forceinline__ void warp_topk(const float (&vin)[EPL], const float (
     if (h0) wrow[lane] = z0 / tot;  // a division: one selected expert gets exactly 1
     if (h1) wrow[lane + 32] = z1 / tot;
   } else {
-    __syncwarp();
     const float inv = 1.0f / sum;
-    for (int j = lane; j < k; j += 32) wrow[j] = wrow[j] * inv;
+    if (lane < k) wrow[lane] = held0 * inv;
+    if (lane + 32 < k) wrow[lane + 32] = held1 * inv;
   }
 }
 
@@ -168,7 +181,7 @@ struct SmallGrid {
   int ncs, hs, chunk;
 };
 
-inline SmallGrid small_grid(int H, int E) {
+__host__ __device__ inline SmallGrid small_grid(int H, int E) {
   SmallGrid g;
   g.ncs = (E + kSmallCols - 1) / kSmallCols;
   int hs = 148 / g.ncs;
@@ -178,6 +191,19 @@ inline SmallGrid small_grid(int H, int E) {
   g.chunk = (((H + hs - 1) / hs) + 15) & ~15;
   g.hs = (H + g.chunk - 1) / g.chunk;
   return g;
+}
+
+// Barrier among the kSmallThreads threads running a router piece: the whole
+// block (BAR = 0, a block of kSmallThreads), or named barrier BAR among
+// threads [0, kSmallThreads) of a larger block (the persistent layer kernel,
+// whose other warps skip the router pieces).
+template <int BAR>
+__device__ __forceinline__ void router_sync() {
+  if constexpr (BAR == 0) {
+    __syncthreads();
+  } else {
+    asm volatile("bar.sync %0, %1;" ::"n"(BAR), "n"(kSmallThreads) : "memory");
+  }
 }
 
 // Shared memory of one partial-logits item (TT tokens).
@@ -190,7 +216,7 @@ struct RouterSmem {
 // Partial logits of item (cs, hy) for T <= TT tokens into slab hy of
 // partial [hs][T][E].  Called by all kSmallThreads threads of a block;
 // ends with the partial written (no fence).
-template <int TT>
+template <int TT, int BAR = 0>
 __device__ __forceinline__ void router_partial(const __nv_bfloat16* __restrict__ x, const float* __restrict__ w,
                                                int T, int H, int E, int chunk, int cs, int hy,
                                                float* __restrict__ partial, RouterSmem<TT>& sm) {
@@ -215,7 +241,7 @@ __device__ __forceinline__ void router_partial(const __nv_bfloat16* __restrict__
     if (t < T && h < h1) val = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H + h));
     reinterpret_cast<uint4*>(&sm.xs[t][0])[v] = val;
   }
-  __syncthreads();
+  router_sync<BAR>();
   float acc[TT][4];
 #pragma unroll
   for (int t = 0; t < TT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
@@ -244,7 +270,7 @@ __device__ __forceinline__ void router_partial(const __nv_bfloat16* __restrict__
 #pragma unroll
       for (int j = 0; j < 4; ++j) sm.red[warp][t][q * 4 + j] = acc[t][j];
   }
-  __syncthreads();
+  router_sync<BAR>();
   if (tid < TT * kSmallCols) {
     const int t = tid / kSmallCols, c = tid - t * kSmallCols;
     float sum = 0.f;
@@ -298,6 +324,79 @@ __device__ __forceinline__ void router_select(const float* partial, int hs, cons
     warp_topk<EPL, false, false>(v, v, true, E, k, t, idrow, wrow, sel, st);
   else
     warp_topk<EPL, false, true>(v, src, scoring == MOE_SCORE_SOFTMAX_SELECT_BIAS, E, k, t, idrow, wrow, sel, st);
+}
+
+// The last block of the few-token router (kSmallThreads threads, barrier
+// BAR): sums the partial slabs in slab order, selects each token's top-k
+// under the scoring rule (one warp per token) and, if offsets != nullptr,
+// writes the expert-contiguous permutation of the n = T*k slots (a stable
+// counting sort: experts ascending, slot order within an expert), as the
+// permutation kernels do; counts may be nullptr.  The outputs may be global
+// or shared memory.  sel [T*k], cnt [E] and warp_sums [kSmallThreads/32]
+// are shared memory of the caller.
+template <int EPL, int BAR = 0>
+__device__ __forceinline__ void router_finish(const float* partial, int hs, const float* __restrict__ bias, int T,
+                                              int E, int k, int scoring, int32_t* ids, float* wout,
+                                              int32_t* counts, int32_t* offsets, int32_t* sorted_ids,
+                                              int32_t* inv_perm, DevStatus* st, int32_t* sel, int32_t* cnt,
+                                              int32_t* warp_sums) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int t = warp; t < T; t += kSmallThreads / 32)
+    router_select<EPL>(partial, hs, bias, T, E, k, scoring, t, ids + (size_t)t * k, wout + (size_t)t * k,
+                       sel + t * k, st);
+  if (offsets == nullptr) return;
+  // ---- permutation of the n = T*k slots, stable counting sort by expert
+  const int n = T * k;
+  for (int e = tid; e < E; e += kSmallThreads) cnt[e] = 0;
+  router_sync<BAR>();
+  for (int s = tid; s < n; s += kSmallThreads) atomicAdd(&cnt[sel[s]], 1);
+  router_sync<BAR>();
+  constexpr int EPT = kMaxExperts / kSmallThreads;  // experts per thread in the scan
+  int loc[EPT], tot = 0;
+#pragma unroll
+  for (int j = 0; j < EPT; ++j) {
+    const int e = tid * EPT + j;
+    loc[j] = e < E ? cnt[e] : 0;
+    tot += loc[j];
+  }
+  int incl = tot;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += o;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  router_sync<BAR>();
+  int base = incl - tot;
+  for (int v = 0; v < warp; ++v) base += warp_sums[v];
+#pragma unroll
+  for (int j = 0; j < EPT; ++j) {
+    const int e = tid * EPT + j;
+    if (e < E) {
+      if (counts) counts[e] = loc[j];
+      offsets[e] = base;
+      cnt[e] = base;  // running position of expert e
+    }
+    base += loc[j];
+  }
+  if (tid == 0) offsets[E] = n;
+  router_sync<BAR>();
+  if (warp == 0) {
+    for (int s0 = 0; s0 < n; s0 += 32) {
+      const int s = s0 + lane;
+      const int e = s < n ? sel[s] : -1;
+      const uint32_t peers = __match_any_sync(0xffffffffu, e);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      const int pos = e >= 0 ? cnt[e] + rank : -1;
+      __syncwarp();
+      if (e >= 0 && rank == 0) cnt[e] += __popc(peers);
+      __syncwarp();
+      if (e >= 0) {
+        sorted_ids[pos] = s / k;
+        inv_perm[s] = pos;
+      }
+    }
+  }
 }
 
 }  // namespace moe

@@ -57,21 +57,24 @@ def test_workspace_layout_is_ordered_and_aligned(lib):
     assert Ls["split"] - Ls["o_shared"] >= 4096 * 8192 * 4
     # many tokens: no K split and no one-launch layer, so no partial slabs
     assert L["arrivals"] == L["fused"] == L["split"] and Ls["arrivals"] == Ls["fused"] == Ls["split"]
-    # arrival counters of the combine in the down GEMM: one per token and 64 output columns
-    assert L["total"] - L["arrivals"] == 8192 * (4096 // 64) * 4
-    assert Ls["total"] - Ls["arrivals"] == 4096 * (8192 // 64) * 4
+    # arrival counters of the combine in the down GEMM (one per token and 64 output columns) and one
+    # done-counter per expert and 128-column gate/up block, rounded up to 256 bytes
+    assert L["total"] - L["arrivals"] == (8192 * (4096 // 64) + 512 * 8 + 63) // 64 * 256
+    assert Ls["total"] - Ls["arrivals"] == (4096 * (8192 // 64) + 256 * 16 + 63) // 64 * 256
 
 
 def test_workspace_layout_reserves_k_split_slabs_for_one_token(lib):
     """One token, 8 of 256 experts, H = 4096, I = 1536: 8 active experts give
     96 gate/up units (-> 3 K slices) and 128 down units (-> 2 slices) for
-    148 SMs.  The split region holds the larger: 3 x 8 rows x 3072 f32."""
+    148 SMs.  The split region holds both: 3 x 8 rows x 3072 and 2 x 8 rows x 4096 f32."""
     L = moe.workspace_layout(1, 4096, 256, 1536, 8)
-    assert L["fused"] - L["split"] == max(3 * 8 * 3072, 2 * 8 * 4096) * 4
+    # gate/up slabs, then down slabs (the persistent few-token layer holds both)
+    assert L["fused"] - L["split"] == (3 * 8 * 3072 + 2 * 8 * 4096) * 4
     # the one-launch layer (T <= 4): 8 K slices of gate/up (2 x I) and down (H) rows, f32
     assert L["arrivals"] - L["fused"] == 8 * 8 * (2 * 1536 + 4096) * 4
-    # arrival counters: the K-split gate/up's (8 rows x 1536/32 chunks) outnumber the down's (1 x 4096/64)
-    assert L["total"] - L["arrivals"] == 256 * ((8 * 1536 // 32 * 4 + 255) // 256)
+    # arrival counters: the K-split gate/up's (8 rows x 1536/32 chunks), the down's (1 x 4096/64) and one
+    # per expert and 128-column gate/up block, side by side, rounded up to 256 bytes
+    assert L["total"] - L["arrivals"] == (8 * 1536 // 32 + 4096 // 64 + 256 * 12 + 63) // 64 * 256
     # the router's partial slabs: one per H slice of the few-token router
     assert L["router_split"] - L["logits"] >= 4 * 1 * 256 * 4
 

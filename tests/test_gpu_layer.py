@@ -167,14 +167,21 @@ def fused_ok(cfg):
             and cfg.I_s % 256 == 0)
 
 
+def persistent_ok(cfg):
+    return cfg.T <= 16 and cfg.E % 4 == 0 and cfg.I_s == 0
+
+
 @pytest.mark.parametrize("router", [moe.ROUTER_FMA, moe.ROUTER_TC, moe.ROUTER_SMALL])
-@pytest.mark.parametrize("tiles", [moe.TILES_SMALL, moe.TILES_LARGE, moe.TILES_PAIR, moe.TILES_FUSED])
+@pytest.mark.parametrize("tiles", [moe.TILES_SMALL, moe.TILES_LARGE, moe.TILES_PAIR, moe.TILES_FUSED,
+                                   moe.TILES_PERSISTENT])
 @pytest.mark.parametrize("name", list(CASES))
 def test_forward_matches_oracle(name, tiles, router):
     cfg, inp, ref = case(name)
     router_skip(cfg, router)
     if tiles == moe.TILES_FUSED and (router != moe.ROUTER_SMALL or not fused_ok(cfg)):
         pytest.skip("one-launch layer: T <= 4 and 256-multiple shapes (its router is the few-token one)")
+    if tiles == moe.TILES_PERSISTENT and (router != moe.ROUTER_SMALL or not persistent_ok(cfg)):
+        pytest.skip("persistent layer: T <= 16, E % 4 == 0, no shared expert (its router is the few-token one)")
     d = dev_inputs(inp)
     ws = workspace(cfg)
     y = moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws,
@@ -310,6 +317,45 @@ def test_fused_layer_one_launch_repeated_and_deterministic():
         assert_close_output(host_f64(ys[0]), ref["y"])
         torch.cuda.synchronize()
         assert ws[:32].view(torch.int32).cpu().tolist() == [0] * 8
+
+
+@pytest.mark.parametrize("name", [n for n, c in CASES.items() if persistent_ok(c)])
+def test_persistent_layer_bitwise_equals_kernel_sequence(name):
+    """The persistent layer runs the same tiles, K split, epilogue arithmetic
+    and router as the multi-kernel path with SMALL tiles and the few-token
+    router, so y is bitwise the same; three calls in a row agree, the
+    routing is bit-exact against the oracle, and the status block (router,
+    plan and exit words) is all zero afterwards."""
+    import torch
+    cfg, inp, ref = case(name)
+    d = dev_inputs(inp)
+    ws = workspace(cfg)
+    args = (d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws)
+    want = moe.forward(*args, tiles=moe.TILES_SMALL, router=moe.ROUTER_SMALL).cpu()
+    assert_ok(ws)
+    info = {}
+    for _ in range(3):
+        got = moe.forward(*args, tiles=moe.TILES_PERSISTENT, info=info).cpu()
+        assert_ok(ws)
+        assert info["launches"] == 1
+        assert torch.equal(got, want)
+        torch.cuda.synchronize()
+        assert ws[:32].view(torch.int32).cpu().tolist() == [0] * 8
+    v = moe.workspace_view(ws, cfg.T, cfg.H, cfg.E, cfg.I, cfg.k, cfg.I_s)
+    np.testing.assert_array_equal(v["topk_ids"].cpu().numpy(), ref["ids"])
+    np.testing.assert_array_equal(v["offsets"].cpu().numpy(), ref["offsets"])
+    np.testing.assert_array_equal(v["sorted_token_ids"].cpu().numpy(), ref["sorted_token_ids"])
+    np.testing.assert_array_equal(v["inv_perm"].cpu().numpy(), ref["inv_perm"])
+    assert_close_output(host_f64(got), ref["y"])
+
+
+def test_persistent_layer_rejects_unsupported_shapes():
+    for name in ("tiny", "three_shared"):  # 64 tokens; a shared expert
+        cfg, inp, ref = case(name)
+        d = dev_inputs(inp)
+        with pytest.raises(moe.MoEError):
+            moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, workspace(cfg),
+                        d["w_sh_gate_up"], d["w_sh_down"], tiles=moe.TILES_PERSISTENT)
 
 
 def test_fused_policy_rejects_unsupported_shapes():
