@@ -184,6 +184,41 @@ def device_inputs(cfg, rank):
     return d, x
 
 
+def device_inputs_mx(cfg, rank):
+    """The same workload with block-scaled FP8 expert weights (seeded random
+    E4M3 codes and E8M0 scales, synth.mx_expert_weights) instead of bf16."""
+    import torch
+    from concurrent.futures import ThreadPoolExecutor
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+    t0 = time.time()
+    inp = synth.make_inputs(cfg.with_(seed=cfg.seed), experts=False)
+    x = inp.x if rank == 0 else synth.make_x(cfg.with_(seed=cfg.seed + rank))
+    E, H, I = cfg.E, cfg.H, cfg.I
+    # codes of W^T [E, N, K] (K contiguous), scales [E, K/32, N]
+    out = {"gate_up": (torch.empty(E, 2 * I, H, dtype=torch.uint8, device="cuda"),
+                       torch.empty(E, H // 32, 2 * I, dtype=torch.uint8, device="cuda")),
+           "down": (torch.empty(E, H, I, dtype=torch.uint8, device="cuda"),
+                    torch.empty(E, I // 32, H, dtype=torch.uint8, device="cuda"))}
+    with ThreadPoolExecutor(min(16, os.cpu_count() or 4)) as ex:
+        for which in ("gate_up", "down"):
+            for e0 in range(0, E, 32):
+                e1 = min(E, e0 + 32)
+                parts = list(ex.map(lambda e: synth.mx_expert_weights(cfg, e, which), range(e0, e1)))
+                out[which][0][e0:e1].copy_(torch.from_numpy(np.stack([c for c, _ in parts])).transpose(1, 2))
+                out[which][1][e0:e1].copy_(torch.from_numpy(np.stack([sc for _, sc in parts])))
+    d = dict(x=bf(x), w_router=torch.from_numpy(inp.w_router).cuda(),
+             bias=None if inp.bias is None else torch.from_numpy(inp.bias).cuda(),
+             mx=(out["gate_up"][0], out["gate_up"][1], out["down"][0], out["down"][1]),
+             w_sh_gate_up=None if inp.w_sh_gate_up is None else bf(inp.w_sh_gate_up),
+             w_sh_down=None if inp.w_sh_down is None else bf(inp.w_sh_down))
+    torch.cuda.synchronize()
+    log(f"[bench] rank {rank}: FP8 inputs for {cfg.name} ready in {time.time() - t0:.1f}s")
+    return d
+
+
 class _Shift:
     """Array view indexed by absolute expert id (e - e0)."""
 
@@ -195,14 +230,17 @@ class _Shift:
 
 
 # ---------------------------------------------------------------- accounting
-def layer_accounting(cfg, counts):
-    """Algorithmic FLOPs and bytes of one step (activated experts only)."""
+def layer_accounting(cfg, counts, mx=False):
+    """Algorithmic FLOPs and bytes of one step (activated experts only).  With
+    mx, the routed experts' weights take 1 byte each plus one scale byte per
+    32 (block-scaled FP8); the shared expert stays bf16."""
     touched = int((counts > 0).sum())
     H, I, T, k = cfg.H, cfg.I, cfg.T, cfg.k
+    wb = (1.0 + 1.0 / 32) if mx else 2.0  # bytes per routed expert weight
     flops = 6.0 * k * H * I * T + (6.0 * H * cfg.I_s * T if cfg.I_s else 0.0)
-    w_bytes = touched * 3 * H * I * 2 + (3 * H * cfg.I_s * 2 if cfg.I_s else 0)
+    w_bytes = touched * 3 * H * I * wb + (3 * H * cfg.I_s * 2 if cfg.I_s else 0)
     layer_bytes = w_bytes + T * H * 2 + H * cfg.E * 4 + T * H * 2
-    gate_up_bytes = touched * H * 2 * I * 2 + T * H * 2 + T * k * I * 2
+    gate_up_bytes = touched * H * 2 * I * wb + T * H * 2 + T * k * I * 2
     return dict(touched=touched, flops=flops, layer_bytes=layer_bytes, gate_up_bytes=gate_up_bytes)
 
 
@@ -233,7 +271,8 @@ TILES = {"auto": 0, "small": 1, "large": 2, "pair": 3, "fused": 4, "persistent":
 COMBINE = {"auto": 0, "fused": 1, "separate": 2}
 # further workloads timed with the default workload, reported under "extra" (their weights
 # replace the decode ones after the decode and prefill measurements)
-DEFAULT_EXTRA = "ling_skewed_t4096,sweep_decode_t1,sweep_decode_t4,sweep_decode_t16,sweep_decode_t64"
+DEFAULT_EXTRA = ("ling_skewed_t4096,sweep_decode_t1,sweep_decode_t4,sweep_decode_t16,sweep_decode_t64,"
+                 "qwen_decode_t512:mx,qwen_prefill_t8192:mx")
 # router scoring rules (an extra workload "name:rule" is timed under that rule)
 SCORING = {"softmax": 0, "softmax_select_bias": 1, "sigmoid": 2}
 
@@ -249,6 +288,10 @@ def time_workload(cfg, d, ws, steps, warmup, rank, world, flush, moe, gpu_index,
     out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
 
     def step(evs=None, info=None):
+        if "mx" in d:
+            return moe.forward_mx(d["x"], d["w_router"], d["bias"], *d["mx"], cfg.k, ws, d["w_sh_gate_up"],
+                                  d["w_sh_down"], stage_events=evs, info=info, tiles=tiles, out=out,
+                                  scoring=scoring, combine=combine)
         return moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws,
                            d["w_sh_gate_up"], d["w_sh_down"], stage_events=evs, info=info, tiles=tiles, out=out,
                            scoring=scoring, combine=combine)
@@ -477,13 +520,14 @@ def run_ours(args):
         loaded = None
         for spec in args.extra.split(","):
             name, _, sc_name = spec.partition(":")
-            scoring = SCORING[sc_name or "softmax"]
+            mx = sc_name == "mx"
+            scoring = SCORING["softmax" if mx or not sc_name else sc_name]
             ecfg = synth.CONFIGS[name]
-            key = (ecfg.H, ecfg.E, ecfg.I, ecfg.I_s, ecfg.bias)
+            key = (ecfg.H, ecfg.E, ecfg.I, ecfg.I_s, ecfg.bias, mx)
             if loaded is None or loaded[0] != key:
                 loaded = None
                 torch.cuda.empty_cache()
-                loaded = (key, device_inputs(ecfg, rank)[0])
+                loaded = (key, device_inputs_mx(ecfg, rank) if mx else device_inputs(ecfg, rank)[0])
             de = dict(loaded[1])
             de["x"] = torch.from_numpy(synth.make_x(ecfg.with_(seed=ecfg.seed + rank)).view(np.int16)).view(
                 torch.bfloat16).cuda()
@@ -493,10 +537,13 @@ def run_ours(args):
             gres = time_workload(ecfg, de, wse, args.steps, args.warmup, rank, world, flush, moe, gpu_index,
                                  sample_clocks=False, tiles=tiles, graph=True, scoring=scoring, combine=comb)
             ecounts = moe.workspace_view(wse, ecfg.T, ecfg.H, ecfg.E, ecfg.I, ecfg.k, ecfg.I_s)["counts"]
-            eacc = layer_accounting(ecfg, ecounts.cpu().numpy())
+            eacc = layer_accounting(ecfg, ecounts.cpu().numpy(), mx=mx)
             extra[spec] = {"value": round(gres["value"], 1), "unit": "tokens/s",
                            "ms_per_step": round(gres["ms_per_step"], 4), "eager": eager_of(eres),
                            **roof(ecfg, eres, eacc, gres["ms_per_step"])}
+            if mx:
+                extra[spec]["weights"] = "block-scaled FP8: E4M3 codes, one E8M0 scale per 32 along K"
+                extra[spec]["roofline"]["traffic"] = None
             del wse
 
     cpu = None
@@ -584,9 +631,9 @@ def main():
                     help="weighted combine in the down GEMM's epilogue (fused) or its own kernel (separate)")
     ap.add_argument("--extra", default=None,
                     help="comma-separated further workloads to time (default with the default workload: the "
-                         "Ling-like skewed prefill and the small-batch decode sweep; otherwise none); "
-                         "name:sigmoid or name:softmax_select_bias times it under that router scoring rule; "
-                         "'' for none")
+                         "Ling-like skewed prefill, the small-batch decode sweep and the decode and prefill steps on "
+                         "block-scaled FP8 weights; otherwise none); name:sigmoid or name:softmax_select_bias "
+                         "times it under that router scoring rule, name:mx on FP8 weights; '' for none")
     args = ap.parse_args()
     if args.extra is None:
         args.extra = DEFAULT_EXTRA if args.workload == ap.get_default("workload") else ""

@@ -326,6 +326,35 @@ moe_status_t moe_forward_ex(const uint16_t *x, const float *w_router, const floa
                             uint16_t *y, void *workspace, size_t workspace_bytes,
                             moe_forward_options_t *options, void *stream);
 
+/* The layer on block-scaled FP8 expert weights.  Each routed expert matrix
+ * W [E, K, N] (W_gate_up: K = H, N = 2I; W_down: K = I, N = H) is given as
+ * OCP FP8 E4M3 codes of its transpose, [E, N, K] u8 with K contiguous (1
+ * sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent 0 =
+ * subnormals; 0x7F/0xFF = NaN; largest 448), and one OCP E8M0 scale per 32
+ * consecutive weights along K of each column, [E, K/32, N] u8
+ * (2^(code - 127); 0xFF = NaN): the weight W[e, k, n] is
+ * e4m3(code[e, n, k]) * 2^(scale[e, k/32, n] - 127).  Token rows, h and the
+ * shared expert stay bf16.  Passage: Qwen 3.5-397B MoE on Ironwood (TPU
+ * v7x), sec. 6 "numerical validation" (accumulation across FP8 scaling
+ * blocks); the Ironwood systems handbook page runs Microscaling formats.
+ * Every such weight with scale code 3 or above is an exact bf16 value (4
+ * significant bits times a power of two, within bf16's range), so the layer
+ * computes exactly what moe_forward_ex computes on the dequantised weights,
+ * with the same rounding points; only the expert-weight bytes halve (plus
+ * 1/32 for the scales).  Below scale code 3 a weight smaller than bf16's
+ * least subnormal step is rounded to nearest bf16.  Everything else as moe_forward_ex, except: tile policies FUSED
+ * and PERSISTENT and MOE_COMBINE_FUSED are not available
+ * (MOE_ERR_INVALID_ARG), and PAIR runs as LARGE (single-SM 256-row passes).
+ * The two E4M3 NaN patterns are not supported as weights (they decode as
+ * +-480, not NaN).  Codes and scales pointers 16-byte aligned. */
+moe_status_t moe_forward_mx(const uint16_t *x, const float *w_router, const float *bias,
+                            const uint8_t *w_gate_up_codes, const uint8_t *w_gate_up_scales,
+                            const uint8_t *w_down_codes, const uint8_t *w_down_scales,
+                            const uint16_t *w_sh_gate_up, const uint16_t *w_sh_down, int I_s,
+                            int T, int H, int E, int I, int k,
+                            uint16_t *y, void *workspace, size_t workspace_bytes,
+                            moe_forward_options_t *options, void *stream);
+
 /* Failure-detection self test: launches one block that waits, with the
  * library's bounded wait, on a barrier nothing will complete.  After
  * timeout_ns the wait gives up, the kernel records MOE_ERR_DEVICE_TIMEOUT

@@ -21,7 +21,7 @@ __all__ = [
     "SCORE_SOFTMAX", "SCORE_SOFTMAX_SELECT_BIAS", "SCORE_SIGMOID",
     "COMBINE_AUTO", "COMBINE_FUSED", "COMBINE_SEPARATE",
     "workspace_size", "workspace_layout", "alloc_workspace", "route", "permute", "grouped_swiglu",
-    "grouped_down", "down_combine", "forward", "device_status", "clear_device_status", "selftest_timeout",
+    "grouped_down", "down_combine", "forward", "forward_mx", "device_status", "clear_device_status", "selftest_timeout",
     "STATUS",
 ]
 
@@ -71,6 +71,8 @@ _SIGS = {
     "moe_down_combine": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _Z, _P], _I),
     "moe_forward": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _Z, _P], _I),
     "moe_forward_ex": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _Z,
+                        ctypes.POINTER(_Options), _P], _I),
+    "moe_forward_mx": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _Z,
                         ctypes.POINTER(_Options), _P], _I),
     "moe_selftest_timeout": ([_P, _Z, _U64, _P], _I),
 }
@@ -304,6 +306,49 @@ def forward(x, w_router, bias, w_gate_up, w_down, k, ws, w_sh_gate_up=None, w_sh
     _check(lib().moe_forward_ex(_ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate_up), _ptr(w_down),
                                 _ptr(w_sh_gate_up), _ptr(w_sh_down), I_s, T, H, E, I, k, _ptr(y), _ptr(ws),
                                 ws.numel(), ctypes.byref(opt), _stream()), "moe_forward")
+    if info is not None:
+        info["launches"] = opt.launches
+    return y
+
+
+def forward_mx(x, w_router, bias, w_gate_up_codes, w_gate_up_scales, w_down_codes, w_down_scales, k, ws,
+               w_sh_gate_up=None, w_sh_down=None, tiles=TILES_AUTO, router=ROUTER_AUTO, out=None,
+               stage_events=None, info=None, scoring=SCORE_SOFTMAX, combine=COMBINE_AUTO):
+    """The layer on block-scaled FP8 expert weights W [E, K, N]: codes of the
+    transpose uint8 [E, N, K] (OCP E4M3, K contiguous) and scales uint8
+    [E, K/32, N] (OCP E8M0) for W_gate_up (K = H, N = 2I) and W_down (K = I,
+    N = H); y [T,H] bf16 (include/moe.h)."""
+    import torch
+    T, H = _dims(x, 2, "x")
+    E, I2, _ = _dims(w_gate_up_codes, 3, "w_gate_up_codes")
+    I = I2 // 2
+    I_s = 0
+    if (w_sh_gate_up is None) != (w_sh_down is None):
+        raise TypeError("the shared expert needs both w_sh_gate_up and w_sh_down")
+    if w_sh_gate_up is not None:
+        I_s = _dims(w_sh_gate_up, 2, "w_sh_gate_up")[1] // 2
+    if H % 32 or I % 32:
+        raise ValueError("H and I must be multiples of the 32-weight scale block")
+    _check_args([(x, torch.bfloat16, "x", (T, H)), (w_router, torch.float32, "w_router", (H, E)),
+                 (bias, torch.float32, "bias", (E,)),
+                 (w_gate_up_codes, torch.uint8, "w_gate_up_codes", (E, 2 * I, H)),
+                 (w_gate_up_scales, torch.uint8, "w_gate_up_scales", (E, H // 32, 2 * I)),
+                 (w_down_codes, torch.uint8, "w_down_codes", (E, H, I)),
+                 (w_down_scales, torch.uint8, "w_down_scales", (E, I // 32, H)),
+                 (w_sh_gate_up, torch.bfloat16, "w_sh_gate_up", (H, 2 * I_s)),
+                 (w_sh_down, torch.bfloat16, "w_sh_down", (I_s, H)), (out, torch.bfloat16, "out", (T, H))], ws)
+    y = out if out is not None else torch.empty(T, H, dtype=torch.bfloat16, device=x.device)
+    opt = _Options(tiles, router)
+    opt.scoring = scoring
+    opt.combine = combine
+    if stage_events is not None:
+        for i, ev in enumerate(stage_events):
+            if ev is not None:
+                opt.stage_events[i] = ev.cuda_event
+    _check(lib().moe_forward_mx(_ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate_up_codes), _ptr(w_gate_up_scales),
+                                _ptr(w_down_codes), _ptr(w_down_scales), _ptr(w_sh_gate_up), _ptr(w_sh_down), I_s,
+                                T, H, E, I, k, _ptr(y), _ptr(ws), ws.numel(), ctypes.byref(opt), _stream()),
+           "moe_forward_mx")
     if info is not None:
         info["launches"] = opt.launches
     return y

@@ -162,12 +162,19 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor [d2][d1][d0] (d0 contiguous), box 64 x 64 x 1, 128-byte swizzle.
-// A descriptor depends only on (address, extents), so the last few are
-// memoised: a steady stream of calls on the same weights skips the encode.
+// Tensor maps of the weight matrices, [d2][d1][d0] with d0 contiguous:
+//   kMapBf16:  bf16, box 64 x 64 x 1, 128-byte swizzle (the bf16 kernels);
+//   kMapCodes: u8 FP8 codes [E][N][K], box 64*kMxRawSteps x 128 x 1, swizzled
+//              over the box row (64 or 128 bytes);
+//   kMapScales: u8 E8M0 scales, box 128 x 2*kMxRawSteps x 1, no swizzle.
+// A descriptor depends only on (kind, address, extents), so the last few
+// are memoised: a steady stream of calls on the same weights skips the
+// encode.
+enum MapKind { kMapBf16 = 0, kMapCodes = 1, kMapScales = 2 };
 struct MapCacheEntry {
   const void* base;
   uint64_t d0, d1, d2;
+  int kind;
   CUtensorMap map;
 };
 constexpr int kMapCache = 16;
@@ -175,35 +182,52 @@ std::mutex g_map_mutex;
 MapCacheEntry g_map_cache[kMapCache];
 int g_map_next = 0;
 
-bool encode_weight_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2);
+bool encode_map(CUtensorMap* m, int kind, const void* base, uint64_t d0, uint64_t d1, uint64_t d2) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const uint64_t esz = kind == kMapBf16 ? 2 : 1;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * esz, d0 * d1 * esz};
+  cuuint32_t box[3] = {kind == kMapBf16 ? 64u : kind == kMapScales ? 128u : 64u * kMxRawSteps,
+                       kind == kMapBf16 ? 64u : kind == kMapScales ? 2u * kMxRawSteps : 128u, 1};
+  const CUtensorMapSwizzle code_swizzle = kMxRawSteps == 1 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, kind == kMapBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+             const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             kind == kMapBf16 ? CU_TENSOR_MAP_SWIZZLE_128B
+                              : kind == kMapCodes ? code_swizzle : CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
-bool make_weight_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2) {
+bool make_map(CUtensorMap* m, int kind, const void* base, uint64_t d0, uint64_t d1, uint64_t d2) {
   {
     std::lock_guard<std::mutex> lock(g_map_mutex);
     for (const MapCacheEntry& e : g_map_cache) {
-      if (e.base == base && e.d0 == d0 && e.d1 == d1 && e.d2 == d2) {
+      if (e.base == base && e.d0 == d0 && e.d1 == d1 && e.d2 == d2 && e.kind == kind) {
         *m = e.map;
         return true;
       }
     }
   }
-  if (!encode_weight_map(m, base, d0, d1, d2)) return false;
+  if (!encode_map(m, kind, base, d0, d1, d2)) return false;
   std::lock_guard<std::mutex> lock(g_map_mutex);
-  g_map_cache[g_map_next] = MapCacheEntry{base, d0, d1, d2, *m};
+  g_map_cache[g_map_next] = MapCacheEntry{base, d0, d1, d2, kind, *m};
   g_map_next = (g_map_next + 1) % kMapCache;
   return true;
 }
 
-bool encode_weight_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {d0, d1, d2};
-  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
-  cuuint32_t box[3] = {64, 64, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+bool make_weight_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2) {
+  return make_map(m, kMapBf16, base, d0, d1, d2);
+}
+
+// Block-scaled FP8 weights of one expert matrix W [E, K, N]: codes of W^T
+// [E, N, K] and their scales [E, K/32, N].
+struct MxWeights {
+  const uint8_t* codes;
+  const uint8_t* scales;
+};
+bool make_mx_maps(CUtensorMap* cm, CUtensorMap* sm, const MxWeights& w, uint64_t N, uint64_t K, uint64_t E) {
+  return make_map(cm, kMapCodes, w.codes, K, N, E) && make_map(sm, kMapScales, w.scales, N, K / 32, E);
 }
 
 struct DeviceInfo {
@@ -388,7 +412,19 @@ GemmArgs gate_up_args(const uint16_t* x, int src_rows, const int32_t* offsets, c
 moe_status_t run_swiglu(const uint16_t* x, int src_rows, const uint16_t* w_gate_up, const int32_t* offsets,
                         const int32_t* row_index, int rows, int H, int E, int I, int tiles, uint16_t* h,
                         DevStatus* st, const DeviceInfo& dev, cudaStream_t s, int nsplit = 1,
-                        float* partials = nullptr, uint32_t* arrivals = nullptr) {
+                        float* partials = nullptr, uint32_t* arrivals = nullptr, const MxWeights* mx = nullptr) {
+  if (mx != nullptr) {  // block-scaled FP8 weights: single-SM tiles of the FP8 kernel
+    CUtensorMap cm, sm;
+    if (!make_mx_maps(&cm, &sm, *mx, 2ull * I, (uint64_t)H, (uint64_t)E)) return MOE_ERR_CUDA;
+    const int xt = tiles == MOE_TILES_SMALL ? MOE_TILES_SMALL : MOE_TILES_LARGE;
+    const GemmArgs a = gate_up_args(x, src_rows, offsets, row_index, rows, H, E, I, h, st, nsplit, partials, arrivals);
+    if (nsplit > 1) {
+      if (arrivals != nullptr) return cuda_status(launch_grouped_gemm_mx(cm, sm, a, EPI_SWIGLU_SPLIT, xt, dev.num_sms, s));
+      MOE_TRY(cuda_status(launch_grouped_gemm_mx(cm, sm, a, EPI_STORE_F32, xt, dev.num_sms, s)));
+      return cuda_status(launch_swiglu_reduce(partials, nsplit, a.split_stride, rows, I, h, s));
+    }
+    return cuda_status(launch_grouped_gemm_mx(cm, sm, a, EPI_SWIGLU, xt, dev.num_sms, s));
+  }
   CUtensorMap map;
   if (!make_weight_map(&map, w_gate_up, 2ull * I, (uint64_t)H, (uint64_t)E)) return MOE_ERR_CUDA;
   if (tiles == MOE_TILES_PAIR) {  // 256 intermediate columns per unit (128 per SM of the pair)
@@ -465,7 +501,15 @@ GemmArgs down_args(const uint16_t* h, const int32_t* offsets, int rows, int H, i
 
 moe_status_t run_down(const uint16_t* h, const uint16_t* w_down, const int32_t* offsets, int rows, int H, int E,
                       int I, int tiles, float* o, DevStatus* st, const DeviceInfo& dev, cudaStream_t s,
-                      int nsplit = 1, const CombineArgs* comb = nullptr) {
+                      int nsplit = 1, const CombineArgs* comb = nullptr, const MxWeights* mx = nullptr) {
+  if (mx != nullptr) {  // block-scaled FP8 weights: fp32 rows (the combine kernel follows)
+    if (comb != nullptr) return MOE_ERR_INVALID_ARG;
+    CUtensorMap cm, sm;
+    if (!make_mx_maps(&cm, &sm, *mx, (uint64_t)H, (uint64_t)I, (uint64_t)E)) return MOE_ERR_CUDA;
+    const int xt = tiles == MOE_TILES_SMALL ? MOE_TILES_SMALL : MOE_TILES_LARGE;
+    const GemmArgs a = down_args(h, offsets, rows, H, E, I, o, st, nsplit);
+    return cuda_status(launch_grouped_gemm_mx(cm, sm, a, EPI_STORE_F32, xt, dev.num_sms, s));
+  }
   CUtensorMap map;
   if (!make_weight_map(&map, w_down, (uint64_t)H, (uint64_t)I, (uint64_t)E)) return MOE_ERR_CUDA;
   GemmArgs a = down_args(h, offsets, rows, H, E, I, o, st, nsplit, comb);
@@ -480,6 +524,191 @@ moe_status_t run_down(const uint16_t* h, const uint16_t* w_down, const int32_t* 
     return cuda_status(launch_grouped_gemm_pair(map, a, epi, dev.num_sms, s));
   }
   return cuda_status(launch_grouped_gemm(map, a, epi, tiles, dev.num_sms, s));
+}
+
+// The layer (moe_forward_ex, moe_forward_mx): bf16 expert weights, or with
+// mx_gu/mx_dn block-scaled FP8 ones (w_gate_up/w_down unused then).
+moe_status_t forward_impl(const uint16_t* x, const float* w_router, const float* bias, const uint16_t* w_gate_up,
+                          const uint16_t* w_down, const MxWeights* mx_gu, const MxWeights* mx_dn,
+                          const uint16_t* w_sh_gate_up, const uint16_t* w_sh_down, int I_s, int T, int H, int E,
+                          int I, int k, uint16_t* y, void* workspace, size_t workspace_bytes,
+                          moe_forward_options_t* options, void* stream) {
+  const bool mx = mx_gu != nullptr;
+  if (!all_nonnull(x, w_router, y)) return MOE_ERR_INVALID_ARG;
+  if (mx ? !(mx_dn && all_nonnull(mx_gu->codes, mx_gu->scales, mx_dn->codes, mx_dn->scales))
+         : !all_nonnull(w_gate_up, w_down))
+    return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_shapes(T, H, E, I, k, true));
+  const bool shared = w_sh_gate_up != nullptr || w_sh_down != nullptr || I_s != 0;
+  if (shared) {
+    if (!all_nonnull(w_sh_gate_up, w_sh_down) || I_s < 1) return MOE_ERR_INVALID_ARG;
+    if (I_s % 128 != 0) return MOE_ERR_ALIGNMENT;
+    if (!all_aligned(w_sh_gate_up, w_sh_down)) return MOE_ERR_ALIGNMENT;
+  }
+  const int tile_policy = options ? options->tile_policy : MOE_TILES_AUTO;
+  const int router_impl = options ? options->router_impl : MOE_ROUTER_AUTO;
+  const int scoring = options ? options->scoring : MOE_SCORE_SOFTMAX;
+  const int combine = options ? options->combine : MOE_COMBINE_AUTO;
+  if (combine < MOE_COMBINE_AUTO || combine > MOE_COMBINE_SEPARATE) return MOE_ERR_INVALID_ARG;
+  if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_PERSISTENT) return MOE_ERR_INVALID_ARG;
+  if (router_impl < MOE_ROUTER_AUTO || router_impl > MOE_ROUTER_SMALL) return MOE_ERR_INVALID_ARG;
+  if (!valid_scoring(scoring)) return MOE_ERR_INVALID_ARG;
+  if (mx && (tile_policy == MOE_TILES_FUSED || tile_policy == MOE_TILES_PERSISTENT || combine == MOE_COMBINE_FUSED))
+    return MOE_ERR_INVALID_ARG;  // the FP8 kernel runs the multi-kernel layer with the combine kernel
+  if (!all_aligned(x, w_router, y) || (bias && !aligned16(bias))) return MOE_ERR_ALIGNMENT;
+  if (mx ? !all_aligned(mx_gu->codes, mx_gu->scales, mx_dn->codes, mx_dn->scales) : !all_aligned(w_gate_up, w_down))
+    return MOE_ERR_ALIGNMENT;
+  const moe_workspace_layout_t L = make_layout(T, H, E, I, k, shared ? I_s : 0);
+  MOE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  DeviceInfo dev;
+  MOE_TRY(check_device(&dev));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* ws = workspace;
+  DevStatus* st = status_of(ws);
+  int32_t* ids = at<int32_t>(ws, L.topk_ids);
+  float* tw = at<float>(ws, L.topk_w);
+  int32_t* counts = at<int32_t>(ws, L.counts);
+  int32_t* offs = at<int32_t>(ws, L.offsets);
+  int32_t* sids = at<int32_t>(ws, L.sorted_token_ids);
+  int32_t* inv = at<int32_t>(ws, L.inv_perm);
+  uint16_t* h = at<uint16_t>(ws, L.h);
+  float* o = at<float>(ws, L.o);
+  const int rows = T * k;
+
+  void* const* ev = options ? options->stage_events : nullptr;
+  auto mark = [&](int i) -> moe_status_t {
+    if (ev && ev[i]) return cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s));
+    return MOE_OK;
+  };
+  int launches = 0;
+
+  // A few tokens, on request: the whole layer in one cooperative launch.
+  if (tile_policy == MOE_TILES_FUSED) {
+    if (!fused_decode_supported(T, H, E, I, k, shared ? I_s : 0)) return MOE_ERR_INVALID_ARG;
+    float* slabs = at<float>(ws, L.fused);
+    const size_t frows = (size_t)rows + (shared ? (size_t)T : 0);
+    const int imax = I > I_s ? I : I_s;
+    float* gslabs = slabs;
+    float* dslabs = slabs + (size_t)kFusedMaxSplit * frows * 2 * imax;
+    MOE_TRY(mark(0));
+    MOE_TRY(cuda_status(launch_fused_decode(x, w_router, bias, scoring, w_gate_up, w_down,
+                                            shared ? w_sh_gate_up : nullptr, shared ? w_sh_down : nullptr,
+                                            shared ? I_s : 0, T, H, E, I, k,
+                                            at<float>(ws, L.logits), gslabs, dslabs, ids, tw, counts, offs, sids, inv,
+                                            y, st, kDefaultTimeoutNs, dev.num_sms, s)));
+    for (int i = 1; i < 7; ++i) MOE_TRY(mark(i));
+    if (options) options->launches = 1;
+    return MOE_OK;
+  }
+
+  // A few tokens, on request: the whole layer in one persistent launch on the tensor cores.
+  if (tile_policy == MOE_TILES_PERSISTENT) {
+    if (!layer_small_supported(T, E, shared ? I_s : 0)) return MOE_ERR_INVALID_ARG;
+    if (router_impl != MOE_ROUTER_AUTO && router_impl != MOE_ROUTER_SMALL) return MOE_ERR_INVALID_ARG;
+    const SplitPlan sp = split_plan(T, H, E, I, k, MOE_TILES_SMALL);
+    CUtensorMap gmap, dmap;
+    if (!make_weight_map(&gmap, w_gate_up, 2ull * I, (uint64_t)H, (uint64_t)E) ||
+        !make_weight_map(&dmap, w_down, (uint64_t)H, (uint64_t)I, (uint64_t)E))
+      return MOE_ERR_CUDA;
+    uint32_t* arr = at<uint32_t>(ws, L.arrivals);
+    const size_t gu_cnt = gate_up_cnt_words(T, I, k, sp), dn_cnt = down_cnt_words(T, H);
+    float* gu_slabs = at<float>(ws, L.split);
+    float* dn_slabs = gu_slabs + split_gate_up_elems(T, I, k, sp);
+    LayerParams p{};
+    p.x = x;
+    p.w_router = w_router;
+    p.bias = bias;
+    p.scoring = scoring;
+    p.T = T;
+    p.H = H;
+    p.E = E;
+    p.k = k;
+    p.partial = at<float>(ws, L.logits);
+    p.ids = ids;
+    p.counts = counts;
+    p.offsets = offs;
+    p.sids = sids;
+    p.inv = inv;
+    p.tw = tw;
+    p.expert_done = arr + gu_cnt + dn_cnt;
+    p.zero = ZeroSpan{reinterpret_cast<uint4*>(arr), (int)(arrival_words(T, H, E, I, k) / 4)};
+    p.gu = gate_up_args(x, T, offs, sids, rows, H, E, I, h, st, sp.gate_up, gu_slabs, arr);
+    const CombineArgs comb{sids, inv, tw, nullptr, y, arr + gu_cnt, T, k};
+    p.dn = down_args(h, offs, rows, H, E, I, sp.down > 1 ? dn_slabs : o, st, sp.down, &comb);
+    p.st = st;
+    p.timeout_ns = kDefaultTimeoutNs;
+    MOE_TRY(mark(0));
+    MOE_TRY(cuda_status(launch_layer_small(gmap, dmap, p, dev.num_sms, s)));
+    for (int i = 1; i < 7; ++i) MOE_TRY(mark(i));
+    if (options) options->launches = 1;
+    return MOE_OK;
+  }
+
+  const int ri = resolve_router(router_impl, T, E);
+  int tiles = choose_tiles(tile_policy, rows, E);
+  if (mx) {
+    // The FP8 kernel runs on single SMs; its small tiles are 32-row passes,
+    // which AUTO takes while the mean expert holds at most 24 rows.
+    if (tile_policy == MOE_TILES_AUTO) tiles = rows <= 24ll * E ? MOE_TILES_SMALL : MOE_TILES_LARGE;
+    if (tiles == MOE_TILES_PAIR) tiles = MOE_TILES_LARGE;
+  }
+  const SplitPlan sp = split_plan(T, H, E, I, k, tiles);
+  // Last-arriver epilogues: the K-split gate/up GEMM sums its slabs in its
+  // epilogue unless SEPARATE is asked for; the down GEMM combines in its
+  // epilogue only on request (FUSED), because a separate combine kernel
+  // measured faster at every size (see the combine options in moe.h).
+  const bool fuse_swiglu = combine != MOE_COMBINE_SEPARATE && sp.gate_up > 1;
+  const bool fuse_combine = combine == MOE_COMBINE_FUSED;
+  uint32_t* arrivals = at<uint32_t>(ws, L.arrivals);
+  // the routing kernel zeroes the arrival counters of the fused epilogues
+  const bool need_zero = fuse_swiglu || fuse_combine;
+  const ZeroSpan zero{need_zero ? reinterpret_cast<uint4*>(arrivals) : nullptr,
+                      need_zero ? (int)(arrival_words(T, H, E, I, k) / 4) : 0};
+  MOE_TRY(mark(0));
+  if (ri == MOE_ROUTER_SMALL) {
+    const PermOut perm{counts, offs, sids, inv};
+    MOE_TRY(run_route(x, w_router, bias, T, H, E, k, scoring, ids, tw, ri, ws, L, dev, s, &perm, zero));
+    launches += 1;
+    MOE_TRY(mark(1));
+  } else {
+    MOE_TRY(run_route(x, w_router, bias, T, H, E, k, scoring, ids, tw, ri, ws, L, dev, s, nullptr, zero));
+    launches += ri == MOE_ROUTER_TC ? 3 : 2;
+    MOE_TRY(mark(1));
+    MOE_TRY(cuda_status(
+        launch_permute(ids, T, E, k, counts, offs, sids, inv, at<int32_t>(ws, L.block_hist), st, s)));
+    launches += rows <= 8192 ? 1 : 3;
+  }
+  MOE_TRY(mark(2));
+  float* split = at<float>(ws, L.split);
+  float* o_sh = nullptr;
+  if (shared) {
+    uint16_t* h_sh = at<uint16_t>(ws, L.h_shared);
+    o_sh = at<float>(ws, L.o_shared);
+    const int sh_tiles = choose_tiles(tile_policy, T, 1);
+    MOE_TRY(run_swiglu(x, T, w_sh_gate_up, nullptr, nullptr, T, H, 1, I_s, sh_tiles, h_sh, st, dev, s));
+    MOE_TRY(run_down(h_sh, w_sh_down, nullptr, T, H, 1, I_s, sh_tiles, o_sh, st, dev, s));
+    launches += 2;
+  }
+  MOE_TRY(mark(3));
+  MOE_TRY(run_swiglu(x, T, w_gate_up, offs, sids, rows, H, E, I, tiles, h, st, dev, s, sp.gate_up, split,
+                     fuse_swiglu ? arrivals : nullptr, mx_gu));
+  launches += (sp.gate_up > 1 && !fuse_swiglu) ? 2 : 1;
+  MOE_TRY(mark(4));
+  float* od = sp.down > 1 ? split : o;
+  if (fuse_combine) {
+    const CombineArgs comb{sids, inv, tw, o_sh, y, arrivals, T, k};
+    MOE_TRY(run_down(h, w_down, offs, rows, H, E, I, tiles, od, st, dev, s, sp.down, &comb));
+    launches += 1;
+    MOE_TRY(mark(5));
+  } else {
+    MOE_TRY(run_down(h, w_down, offs, rows, H, E, I, tiles, od, st, dev, s, sp.down, nullptr, mx_dn));
+    MOE_TRY(mark(5));
+    MOE_TRY(cuda_status(launch_combine(od, tw, inv, o_sh, T, H, k, rows, sp.down, (size_t)rows * H, y, st, s)));
+    launches += 2;  // down GEMM, combine
+  }
+  MOE_TRY(mark(6));
+  if (options) options->launches = launches;
+  return MOE_OK;
 }
 
 }  // namespace
@@ -646,168 +875,19 @@ moe_status_t moe_forward_ex(const uint16_t* x, const float* w_router, const floa
                             const uint16_t* w_down, const uint16_t* w_sh_gate_up, const uint16_t* w_sh_down, int I_s,
                             int T, int H, int E, int I, int k, uint16_t* y, void* workspace,
                             size_t workspace_bytes, moe_forward_options_t* options, void* stream) {
-  if (!all_nonnull(x, w_router, w_gate_up, w_down, y)) return MOE_ERR_INVALID_ARG;
-  MOE_TRY(check_shapes(T, H, E, I, k, true));
-  const bool shared = w_sh_gate_up != nullptr || w_sh_down != nullptr || I_s != 0;
-  if (shared) {
-    if (!all_nonnull(w_sh_gate_up, w_sh_down) || I_s < 1) return MOE_ERR_INVALID_ARG;
-    if (I_s % 128 != 0) return MOE_ERR_ALIGNMENT;
-    if (!all_aligned(w_sh_gate_up, w_sh_down)) return MOE_ERR_ALIGNMENT;
-  }
-  const int tile_policy = options ? options->tile_policy : MOE_TILES_AUTO;
-  const int router_impl = options ? options->router_impl : MOE_ROUTER_AUTO;
-  const int scoring = options ? options->scoring : MOE_SCORE_SOFTMAX;
-  const int combine = options ? options->combine : MOE_COMBINE_AUTO;
-  if (combine < MOE_COMBINE_AUTO || combine > MOE_COMBINE_SEPARATE) return MOE_ERR_INVALID_ARG;
-  if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_PERSISTENT) return MOE_ERR_INVALID_ARG;
-  if (router_impl < MOE_ROUTER_AUTO || router_impl > MOE_ROUTER_SMALL) return MOE_ERR_INVALID_ARG;
-  if (!valid_scoring(scoring)) return MOE_ERR_INVALID_ARG;
-  if (!all_aligned(x, w_router, w_gate_up, w_down, y) || (bias && !aligned16(bias))) return MOE_ERR_ALIGNMENT;
-  const moe_workspace_layout_t L = make_layout(T, H, E, I, k, shared ? I_s : 0);
-  MOE_TRY(check_ws(workspace, workspace_bytes, L.total));
-  DeviceInfo dev;
-  MOE_TRY(check_device(&dev));
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  void* ws = workspace;
-  DevStatus* st = status_of(ws);
-  int32_t* ids = at<int32_t>(ws, L.topk_ids);
-  float* tw = at<float>(ws, L.topk_w);
-  int32_t* counts = at<int32_t>(ws, L.counts);
-  int32_t* offs = at<int32_t>(ws, L.offsets);
-  int32_t* sids = at<int32_t>(ws, L.sorted_token_ids);
-  int32_t* inv = at<int32_t>(ws, L.inv_perm);
-  uint16_t* h = at<uint16_t>(ws, L.h);
-  float* o = at<float>(ws, L.o);
-  const int rows = T * k;
+  return forward_impl(x, w_router, bias, w_gate_up, w_down, nullptr, nullptr, w_sh_gate_up, w_sh_down, I_s, T, H, E,
+                      I, k, y, workspace, workspace_bytes, options, stream);
+}
 
-  void* const* ev = options ? options->stage_events : nullptr;
-  auto mark = [&](int i) -> moe_status_t {
-    if (ev && ev[i]) return cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s));
-    return MOE_OK;
-  };
-  int launches = 0;
-
-  // A few tokens, on request: the whole layer in one cooperative launch.
-  if (tile_policy == MOE_TILES_FUSED) {
-    if (!fused_decode_supported(T, H, E, I, k, shared ? I_s : 0)) return MOE_ERR_INVALID_ARG;
-    float* slabs = at<float>(ws, L.fused);
-    const size_t frows = (size_t)rows + (shared ? (size_t)T : 0);
-    const int imax = I > I_s ? I : I_s;
-    float* gslabs = slabs;
-    float* dslabs = slabs + (size_t)kFusedMaxSplit * frows * 2 * imax;
-    MOE_TRY(mark(0));
-    MOE_TRY(cuda_status(launch_fused_decode(x, w_router, bias, scoring, w_gate_up, w_down,
-                                            shared ? w_sh_gate_up : nullptr, shared ? w_sh_down : nullptr,
-                                            shared ? I_s : 0, T, H, E, I, k,
-                                            at<float>(ws, L.logits), gslabs, dslabs, ids, tw, counts, offs, sids, inv,
-                                            y, st, kDefaultTimeoutNs, dev.num_sms, s)));
-    for (int i = 1; i < 7; ++i) MOE_TRY(mark(i));
-    if (options) options->launches = 1;
-    return MOE_OK;
-  }
-
-  // A few tokens, on request: the whole layer in one persistent launch on the tensor cores.
-  if (tile_policy == MOE_TILES_PERSISTENT) {
-    if (!layer_small_supported(T, E, shared ? I_s : 0)) return MOE_ERR_INVALID_ARG;
-    if (router_impl != MOE_ROUTER_AUTO && router_impl != MOE_ROUTER_SMALL) return MOE_ERR_INVALID_ARG;
-    const SplitPlan sp = split_plan(T, H, E, I, k, MOE_TILES_SMALL);
-    CUtensorMap gmap, dmap;
-    if (!make_weight_map(&gmap, w_gate_up, 2ull * I, (uint64_t)H, (uint64_t)E) ||
-        !make_weight_map(&dmap, w_down, (uint64_t)H, (uint64_t)I, (uint64_t)E))
-      return MOE_ERR_CUDA;
-    uint32_t* arr = at<uint32_t>(ws, L.arrivals);
-    const size_t gu_cnt = gate_up_cnt_words(T, I, k, sp), dn_cnt = down_cnt_words(T, H);
-    float* gu_slabs = at<float>(ws, L.split);
-    float* dn_slabs = gu_slabs + split_gate_up_elems(T, I, k, sp);
-    LayerParams p{};
-    p.x = x;
-    p.w_router = w_router;
-    p.bias = bias;
-    p.scoring = scoring;
-    p.T = T;
-    p.H = H;
-    p.E = E;
-    p.k = k;
-    p.partial = at<float>(ws, L.logits);
-    p.ids = ids;
-    p.counts = counts;
-    p.offsets = offs;
-    p.sids = sids;
-    p.inv = inv;
-    p.tw = tw;
-    p.expert_done = arr + gu_cnt + dn_cnt;
-    p.zero = ZeroSpan{reinterpret_cast<uint4*>(arr), (int)(arrival_words(T, H, E, I, k) / 4)};
-    p.gu = gate_up_args(x, T, offs, sids, rows, H, E, I, h, st, sp.gate_up, gu_slabs, arr);
-    const CombineArgs comb{sids, inv, tw, nullptr, y, arr + gu_cnt, T, k};
-    p.dn = down_args(h, offs, rows, H, E, I, sp.down > 1 ? dn_slabs : o, st, sp.down, &comb);
-    p.st = st;
-    p.timeout_ns = kDefaultTimeoutNs;
-    MOE_TRY(mark(0));
-    MOE_TRY(cuda_status(launch_layer_small(gmap, dmap, p, dev.num_sms, s)));
-    for (int i = 1; i < 7; ++i) MOE_TRY(mark(i));
-    if (options) options->launches = 1;
-    return MOE_OK;
-  }
-
-  const int ri = resolve_router(router_impl, T, E);
-  const int tiles = choose_tiles(tile_policy, rows, E);
-  const SplitPlan sp = split_plan(T, H, E, I, k, tiles);
-  // Last-arriver epilogues: the K-split gate/up GEMM sums its slabs in its
-  // epilogue unless SEPARATE is asked for; the down GEMM combines in its
-  // epilogue only on request (FUSED), because a separate combine kernel
-  // measured faster at every size (see the combine options in moe.h).
-  const bool fuse_swiglu = combine != MOE_COMBINE_SEPARATE && sp.gate_up > 1;
-  const bool fuse_combine = combine == MOE_COMBINE_FUSED;
-  uint32_t* arrivals = at<uint32_t>(ws, L.arrivals);
-  // the routing kernel zeroes the arrival counters of the fused epilogues
-  const bool need_zero = fuse_swiglu || fuse_combine;
-  const ZeroSpan zero{need_zero ? reinterpret_cast<uint4*>(arrivals) : nullptr,
-                      need_zero ? (int)(arrival_words(T, H, E, I, k) / 4) : 0};
-  MOE_TRY(mark(0));
-  if (ri == MOE_ROUTER_SMALL) {
-    const PermOut perm{counts, offs, sids, inv};
-    MOE_TRY(run_route(x, w_router, bias, T, H, E, k, scoring, ids, tw, ri, ws, L, dev, s, &perm, zero));
-    launches += 1;
-    MOE_TRY(mark(1));
-  } else {
-    MOE_TRY(run_route(x, w_router, bias, T, H, E, k, scoring, ids, tw, ri, ws, L, dev, s, nullptr, zero));
-    launches += ri == MOE_ROUTER_TC ? 3 : 2;
-    MOE_TRY(mark(1));
-    MOE_TRY(cuda_status(
-        launch_permute(ids, T, E, k, counts, offs, sids, inv, at<int32_t>(ws, L.block_hist), st, s)));
-    launches += rows <= 8192 ? 1 : 3;
-  }
-  MOE_TRY(mark(2));
-  float* split = at<float>(ws, L.split);
-  float* o_sh = nullptr;
-  if (shared) {
-    uint16_t* h_sh = at<uint16_t>(ws, L.h_shared);
-    o_sh = at<float>(ws, L.o_shared);
-    const int sh_tiles = choose_tiles(tile_policy, T, 1);
-    MOE_TRY(run_swiglu(x, T, w_sh_gate_up, nullptr, nullptr, T, H, 1, I_s, sh_tiles, h_sh, st, dev, s));
-    MOE_TRY(run_down(h_sh, w_sh_down, nullptr, T, H, 1, I_s, sh_tiles, o_sh, st, dev, s));
-    launches += 2;
-  }
-  MOE_TRY(mark(3));
-  MOE_TRY(run_swiglu(x, T, w_gate_up, offs, sids, rows, H, E, I, tiles, h, st, dev, s, sp.gate_up, split,
-                     fuse_swiglu ? arrivals : nullptr));
-  launches += (sp.gate_up > 1 && !fuse_swiglu) ? 2 : 1;
-  MOE_TRY(mark(4));
-  float* od = sp.down > 1 ? split : o;
-  if (fuse_combine) {
-    const CombineArgs comb{sids, inv, tw, o_sh, y, arrivals, T, k};
-    MOE_TRY(run_down(h, w_down, offs, rows, H, E, I, tiles, od, st, dev, s, sp.down, &comb));
-    launches += 1;
-    MOE_TRY(mark(5));
-  } else {
-    MOE_TRY(run_down(h, w_down, offs, rows, H, E, I, tiles, od, st, dev, s, sp.down));
-    MOE_TRY(mark(5));
-    MOE_TRY(cuda_status(launch_combine(od, tw, inv, o_sh, T, H, k, rows, sp.down, (size_t)rows * H, y, st, s)));
-    launches += 2;  // down GEMM, combine
-  }
-  MOE_TRY(mark(6));
-  if (options) options->launches = launches;
-  return MOE_OK;
+moe_status_t moe_forward_mx(const uint16_t* x, const float* w_router, const float* bias,
+                            const uint8_t* w_gate_up_codes, const uint8_t* w_gate_up_scales,
+                            const uint8_t* w_down_codes, const uint8_t* w_down_scales,
+                            const uint16_t* w_sh_gate_up, const uint16_t* w_sh_down, int I_s, int T, int H, int E,
+                            int I, int k, uint16_t* y, void* workspace, size_t workspace_bytes,
+                            moe_forward_options_t* options, void* stream) {
+  const MxWeights gu{w_gate_up_codes, w_gate_up_scales}, dn{w_down_codes, w_down_scales};
+  return forward_impl(x, w_router, bias, nullptr, nullptr, &gu, &dn, w_sh_gate_up, w_sh_down, I_s, T, H, E, I, k, y,
+                      workspace, workspace_bytes, options, stream);
 }
 
 moe_status_t moe_forward(const uint16_t* x, const float* w_router, const float* bias, const uint16_t* w_gate_up,

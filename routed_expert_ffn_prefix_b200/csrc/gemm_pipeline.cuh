@@ -133,11 +133,11 @@ struct OnePhase {
 };
 
 // Epilogue of one unit by one epilogue warp: drain its TMEM lane quarter
-// (one weight column per thread) for the 32-row chunks c0 = 32*half + 64*j
-// and store them (SwiGLU -> bf16, or fp32 rows / K slabs); for the
+// (one weight column per thread) for the 32-row chunks c0 = 32*half +
+// 32*HALVES*j (HALVES warps per lane quarter) and store them (SwiGLU -> bf16, or fp32 rows / K slabs); for the
 // last-arriver epilogues, release TMEM first, then count the stored rows and
 // reduce the chunks they complete while the next unit's MMAs run.
-template <int NT, int MT, int EPI>
+template <int NT, int MT, int EPI, int HALVES = 2>
 __device__ __forceinline__ void epilogue_unit(const GemmArgs& a, const Unit& un, uint32_t tbase, int quarter,
                                               int half, uint64_t* tempty_buf) {
   const int lane = lane_id();
@@ -146,7 +146,7 @@ __device__ __forceinline__ void epilogue_unit(const GemmArgs& a, const Unit& un,
   const int col = un.nb * a.out_col_stride + quarter * 32 + lane;
   __nv_bfloat16* const hout = reinterpret_cast<__nv_bfloat16*>(a.out);
   float* const fout = reinterpret_cast<float*>(a.out) + (size_t)un.ks * a.split_stride;
-  for (int c0 = half * 32; c0 < un.rows; c0 += 64) {
+  for (int c0 = half * 32; c0 < un.rows; c0 += 32 * HALVES) {
     const int nr = min(32, un.rows - c0);
     if constexpr (EPI == EPI_SWIGLU) {
       float g[32], v[32];
@@ -186,7 +186,7 @@ __device__ __forceinline__ void epilogue_unit(const GemmArgs& a, const Unit& un,
     cols[0] = col;
     if constexpr (MT == 2) cols[1] = col + out_col1_off;
     const int chunk = un.nb * 4 + quarter;
-    for (int c0 = half * 32; c0 < un.rows; c0 += 64)
+    for (int c0 = half * 32; c0 < un.rows; c0 += 32 * HALVES)
       arrive_rows<MT, EPI>(a, un.row0 + c0, min(32, un.rows - c0), chunk, cols);
   }
 }

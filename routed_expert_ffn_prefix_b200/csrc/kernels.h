@@ -14,6 +14,7 @@ namespace moe {
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxK = 64;          // largest top-k any entry point accepts
 constexpr int kPermuteChunk = 1024; // slots per block of the multi-block permutation (histogram rows)
+constexpr int kMxRawSteps = 2;      // k-steps of 64 per TMA box of FP8 codes (box rows of 64 * this bytes)
 constexpr int kMaxDevices = 64;
 
 // Runs `setup` once per (call site, device): kernel attributes and occupancy
@@ -100,6 +101,18 @@ enum Epilogue { EPI_SWIGLU = 0, EPI_STORE_F32 = 1, EPI_SWIGLU_SPLIT = 2, EPI_DOW
 // policy and epilogue; the caller sets n_blocks/col_stride/out_col_stride
 // for units of 128 * that many columns.
 int gemm_tiles_per_unit(int tiles, int epilogue);
+
+// The grouped GEMM on block-scaled FP8 weights (grouped_gemm_mx.cu): code_map
+// covers the E4M3 codes of W^T [E, N, K] u8 (boxes of kMxRawSteps * 64 codes
+// x 128 columns, swizzled over the box row: 64-byte swizzle for one k-step,
+// 128-byte for two), scale_map the E8M0 scales [E, K/32, N] u8 (boxes of 128
+// columns x 2 * kMxRawSteps rows).  Units of 128-column tiles as in the
+// single-SM kernel (two tiles per unit, col_stride and col1_off multiples of
+// 128, krep 1); epilogue EPI_SWIGLU, EPI_SWIGLU_SPLIT or EPI_STORE_F32;
+// tiles MOE_TILES_SMALL (32-row passes, decoded weights in TMEM) or anything
+// else (256-row passes).
+cudaError_t launch_grouped_gemm_mx(const CUtensorMap& code_map, const CUtensorMap& scale_map, const GemmArgs& a,
+                                   int epilogue, int tiles, int num_sms, cudaStream_t stream);
 
 // Large-row groups on SM pairs (grouped_gemm_pair.cu): 256 token rows per
 // unit, two 128-column weight tiles per unit (the same n_blocks/col_stride/
