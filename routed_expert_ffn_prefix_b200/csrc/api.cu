@@ -166,11 +166,12 @@ EncodeTiledFn encode_fn() {
 //   kMapBf16:  bf16, box 64 x 64 x 1, 128-byte swizzle (the bf16 kernels);
 //   kMapCodes: u8 FP8 codes [E][N][K], box 64*kMxRawSteps x 128 x 1, swizzled
 //              over the box row (64 or 128 bytes);
-//   kMapScales: u8 E8M0 scales, box 128 x 2*kMxRawSteps x 1, no swizzle.
+//   kMapScales: u8 E8M0 scales, box 128 x 2*kMxRawSteps x 1, no swizzle;
+//   kMapRows:  bf16 rows [rows][K] (K contiguous), box 64 x 128 x 1, 128-byte swizzle.
 // A descriptor depends only on (kind, address, extents), so the last few
 // are memoised: a steady stream of calls on the same weights skips the
 // encode.
-enum MapKind { kMapBf16 = 0, kMapCodes = 1, kMapScales = 2 };
+enum MapKind { kMapBf16 = 0, kMapCodes = 1, kMapScales = 2, kMapRows = 3 };
 struct MapCacheEntry {
   const void* base;
   uint64_t d0, d1, d2;
@@ -185,16 +186,17 @@ int g_map_next = 0;
 bool encode_map(CUtensorMap* m, int kind, const void* base, uint64_t d0, uint64_t d1, uint64_t d2) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  const uint64_t esz = kind == kMapBf16 ? 2 : 1;
+  const bool bf16 = kind == kMapBf16 || kind == kMapRows;
+  const uint64_t esz = bf16 ? 2 : 1;
   cuuint64_t dims[3] = {d0, d1, d2};
   cuuint64_t strides[2] = {d0 * esz, d0 * d1 * esz};
-  cuuint32_t box[3] = {kind == kMapBf16 ? 64u : kind == kMapScales ? 128u : 64u * kMxRawSteps,
+  cuuint32_t box[3] = {bf16 ? 64u : kind == kMapScales ? 128u : 64u * kMxRawSteps,
                        kind == kMapBf16 ? 64u : kind == kMapScales ? 2u * kMxRawSteps : 128u, 1};
   const CUtensorMapSwizzle code_swizzle = kMxRawSteps == 1 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, kind == kMapBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+  return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             kind == kMapBf16 ? CU_TENSOR_MAP_SWIZZLE_128B
+             bf16 ? CU_TENSOR_MAP_SWIZZLE_128B
                               : kind == kMapCodes ? code_swizzle : CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -432,7 +434,7 @@ moe_status_t run_swiglu(const uint16_t* x, int src_rows, const uint16_t* w_gate_
     a.n_blocks = (I + 255) / 256;
     a.col_stride = 256;
     a.out_col_stride = 256;
-    return cuda_status(launch_grouped_gemm_pair(map, a, EPI_SWIGLU, dev.num_sms, s));
+    return cuda_status(launch_grouped_gemm_pair(map, nullptr, a, EPI_SWIGLU, dev.num_sms, s));
   }
   const GemmArgs a = gate_up_args(x, src_rows, offsets, row_index, rows, H, E, I, h, st, nsplit, partials, arrivals);
   if (nsplit > 1) {
@@ -514,14 +516,20 @@ moe_status_t run_down(const uint16_t* h, const uint16_t* w_down, const int32_t* 
   if (!make_weight_map(&map, w_down, (uint64_t)H, (uint64_t)I, (uint64_t)E)) return MOE_ERR_CUDA;
   GemmArgs a = down_args(h, offsets, rows, H, E, I, o, st, nsplit, comb);
   const int epi = comb != nullptr ? EPI_DOWN_COMBINE : EPI_STORE_F32;
-  if (tiles == MOE_TILES_PAIR) {  // 2 x 256 output columns per unit (128 of each per SM of the pair)
+  if (tiles == MOE_TILES_PAIR) {
     if (nsplit > 1) return MOE_ERR_INVALID_ARG;
+    // 2 x 256 output columns per unit (128 of each per SM of the pair); the
+    // h rows are contiguous, so with the fp32 store epilogue they come by TMA
+    // (boxes of 128 rows, when there are that many)
     a.n_blocks = (H + 511) / 512;
     a.col_stride = 512;
     a.col1_off = 256;
     a.out_col_stride = 512;
     a.out_col1_off = 256;
-    return cuda_status(launch_grouped_gemm_pair(map, a, epi, dev.num_sms, s));
+    CUtensorMap rmap;
+    const bool rows_tma = epi == EPI_STORE_F32 && rows >= 128;
+    if (rows_tma && !make_map(&rmap, kMapRows, h, (uint64_t)I, (uint64_t)rows, 1)) return MOE_ERR_CUDA;
+    return cuda_status(launch_grouped_gemm_pair(map, rows_tma ? &rmap : nullptr, a, epi, dev.num_sms, s));
   }
   return cuda_status(launch_grouped_gemm(map, a, epi, tiles, dev.num_sms, s));
 }

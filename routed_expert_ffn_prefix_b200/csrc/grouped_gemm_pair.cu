@@ -17,6 +17,11 @@
 //     intermediate units (128 per SM), so SwiGLU stays thread-local;
 //   * down: the two tiles are 2 x 256 adjacent output columns.
 //
+// Rows by TMA (RTMA, the down GEMM): the operand rows are h, already in
+// expert order, so each SM loads its half of a unit's rows with one 2D TMA
+// box per stage (128 rows; rows past the unit's are loaded but not read by
+// the MMA) instead of gathering them row by row.
+//
 // Synchronisation (cluster of 2; rank 0 = leader issues every MMA):
 //   full[s]  (leader): 128 cp.async arrivals of the leader's rows, the
 //            leader's expect_tx for both SMs' weight bytes, and one relayed
@@ -25,6 +30,9 @@
 //   xfull[s] (peer):   the peer's 128 cp.async arrivals; the peer's relay
 //            thread waits on it, fences the writes into the async proxy and
 //            arrives on the leader's full[s].
+//            With RTMA both SMs' row boxes complete their bytes on the
+//            leader's full[s] as the weights do: its only arrival is the
+//            leader's expect_tx, and there is no relay.
 //   empty[s], tfull (both): arrived by the leader's commits, multicast to
 //            both SMs of the pair.
 //   tempty (leader): one arrival per epilogue warp of both SMs.
@@ -147,10 +155,12 @@ __device__ __forceinline__ void mma_commit_pair_leader(uint64_t* bar) {
       : "memory");
 }
 
-template <int NT, int ST, int MT, int EPI>
+template <int NT, int ST, int MT, int EPI, bool RTMA>
 __global__ void __launch_bounds__(kPThreads, 1)
-    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap wmap, const GemmArgs a) {
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap rmap,
+                             const GemmArgs a) {
   using C = PCfg<NT, ST, MT>;
+  static_assert(!RTMA || C::ROWS == 128, "row boxes of 128 rows");
   static_assert(EPI != EPI_SWIGLU || MT == 2, "SwiGLU needs the gate and the up tile");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -173,7 +183,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
 
   if (tid == 0) {
     for (int s = 0; s < ST; ++s) {
-      mbar_init(full + s, kPProdThreads + 2);  // leader rows + leader expect_tx + peer relay
+      mbar_init(full + s, RTMA ? 1 : kPProdThreads + 2);  // (leader rows +) leader expect_tx (+ peer relay)
       mbar_init(xfull + s, kPProdThreads);     // peer rows
       mbar_init(empty + s, 1);
     }
@@ -189,7 +199,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
     tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
     tmem_relinquish_pair();
   }
-  if (warp == kPEpiWarps && lane == 0) prefetch_tmap(&wmap);
+  if (warp == kPEpiWarps && lane == 0) {
+    prefetch_tmap(&wmap);
+    if (RTMA) prefetch_tmap(&rmap);
+  }
   if (warp == 0) build_unit_prefix<NT>(a, ngroups, ustart, total_units);
   tc_fence_before();
   cluster_sync();  // barriers of both SMs initialised before any remote arrive
@@ -240,6 +253,23 @@ __global__ void __launch_bounds__(kPThreads, 1)
         if (!mbar_wait(&empty[stage], phase ^ 1u, wc, 100 + stage)) { ok = false; break; }
         uint8_t* sA = smem + stage * C::STAGE_BYTES;
         const uint32_t sb = smem_u32(sA + C::A_BYTES);
+        if (pt == 0) {  // the weight tiles first: they come from HBM, the rows mostly from L2
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (C::A_BYTES + (RTMA ? C::B_BYTES : 0)));
+          const int d2 = a.a_dim2_rep ? rep : un.group;
+          const uint32_t fb = full_leader + stage * 8;
+#pragma unroll
+          for (int t = 0; t < MT; ++t) {
+            const int c = wcol + t * a.col1_off;
+            tma_load_3d_pair(sA + t * kPATileBytes, &wmap, fb, c, kt * kBK, d2, pol_w);
+            tma_load_3d_pair(sA + t * kPATileBytes + kPBoxBytes, &wmap, fb, c + 64, kt * kBK, d2, pol_w);
+          }
+          // rows map: 3D [1][src_rows][K], like the weight maps
+          if constexpr (RTMA) tma_load_3d_pair(sA + C::A_BYTES, &rmap, fb, kt * kBK, un.row0 + my0, 0, pol_rows);
+        }
+        if constexpr (RTMA) {
+          if (++stage == ST) { stage = 0; phase ^= 1u; }
+          continue;
+        }
 #pragma unroll
         for (int i = 0; i < kRowsPerThread; ++i) {
           if (src[i] >= 0) {
@@ -249,17 +279,6 @@ __global__ void __launch_bounds__(kPThreads, 1)
           }
         }
         cp_async_arrive_noinc(&rows_bar_base[stage]);
-        if (pt == 0) {
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::A_BYTES);
-          const int d2 = a.a_dim2_rep ? rep : un.group;
-          const uint32_t fb = full_leader + stage * 8;
-#pragma unroll
-          for (int t = 0; t < MT; ++t) {
-            const int c = wcol + t * a.col1_off;
-            tma_load_3d_pair(sA + t * kPATileBytes, &wmap, fb, c, kt * kBK, d2, pol_w);
-            tma_load_3d_pair(sA + t * kPATileBytes + kPBoxBytes, &wmap, fb, c + 64, kt * kBK, d2, pol_w);
-          }
-        }
         if (++stage == ST) { stage = 0; phase ^= 1u; }
       }
     }
@@ -281,6 +300,13 @@ __global__ void __launch_bounds__(kPThreads, 1)
         uint32_t phase = 0;
         int acc_it = 0;
         bool ok = true;
+        // Descriptors of stage 0; a stage, a k slice and a tile add to the
+        // start-address field (address / 16, below 2^14 in shared memory).
+        // A = weights (MN-major): +16 k = two 8-row groups = 2048 B, the two
+        // 64-column halves of a tile one TMA box apart; B = rows (K-major):
+        // +16 k = 32 B inside the swizzled row.
+        const uint64_t ad0 = smem_desc_sw128(smem_u32(smem), kPBoxBytes, 1024);
+        const uint64_t bd0 = smem_desc(smem_u32(smem) + C::A_BYTES, 16, 1024, kLayoutSw128);
         for (int u = pair; u < total && ok; u += npairs) {
           const Unit un = decode_unit<NT>(a, ustart, ngroups, u);
           const int buf = C::NBUF == 2 ? (acc_it & 1) : 0;
@@ -297,16 +323,13 @@ __global__ void __launch_bounds__(kPThreads, 1)
             if (!mbar_wait(&full[stage], phase, wc, 300 + stage)) { ok = false; break; }
             tc_fence_after();
             fence_proxy_async_smem();
-            const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES), sb = sa + C::A_BYTES;
+            const uint64_t soff = (uint32_t)(stage * C::STAGE_BYTES) >> 4;
+            const uint64_t ads = ad0 + soff, bds = bd0 + soff;
 #pragma unroll
             for (int kk = 0; kk < kBK / 16; ++kk) {
-              const uint64_t bd = smem_desc(sb + kk * 32, 16, 1024, kLayoutSw128);  // rows: +16 k = 32 B
 #pragma unroll
-              for (int t = 0; t < MT; ++t) {
-                // weights: +16 k = two 8-row groups = 2048 B; 64-column halves one box apart
-                const uint64_t ad = smem_desc_sw128(sa + t * kPATileBytes + kk * 2048, kPBoxBytes, 1024);
-                mma_bf16_pair(d0 + t * NT, ad, bd, idesc, acc);
-              }
+              for (int t = 0; t < MT; ++t)
+                mma_bf16_pair(d0 + t * NT, ads + ((t * kPATileBytes + kk * 2048) >> 4), bds + 2 * kk, idesc, acc);
               acc = 1;
             }
             mma_commit_pair(&empty[stage]);
@@ -329,7 +352,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int u = pair; u < total && ok; u += npairs) {
+      for (int u = pair; u < total && ok && !RTMA; u += npairs) {
         const Unit un = decode_unit<NT>(a, ustart, ngroups, u);
         const int kiters = (un.ke - un.kb) * a.krep;
         for (int it = 0; it < kiters; ++it) {
@@ -422,10 +445,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
   }
 }
 
-template <int NT, int ST, int MT, int EPI>
-cudaError_t launch_pair(const CUtensorMap& wmap, const GemmArgs& a, int num_sms, cudaStream_t stream) {
+template <int NT, int ST, int MT, int EPI, bool RTMA = false>
+cudaError_t launch_pair(const CUtensorMap& wmap, const CUtensorMap* rmap, const GemmArgs& a, int num_sms,
+                        cudaStream_t stream) {
   using C = PCfg<NT, ST, MT>;
-  auto kern = grouped_gemm_pair_kernel<NT, ST, MT, EPI>;
+  auto kern = grouped_gemm_pair_kernel<NT, ST, MT, EPI, RTMA>;
   static std::atomic<int> configured[kMaxDevices];
   cudaError_t err = once_per_device(configured, [&] {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -457,25 +481,35 @@ cudaError_t launch_pair(const CUtensorMap& wmap, const GemmArgs& a, int num_sms,
     });
     if (slots[dev] > 0 && 2 * slots[dev] < (int)cfg.gridDim.x) cfg.gridDim = dim3(2 * slots[dev], 1, 1);
   }
-  return cudaLaunchKernelEx(&cfg, kern, wmap, a);
+  return cudaLaunchKernelEx(&cfg, kern, wmap, RTMA ? *rmap : wmap, a);
 }
 
 }  // namespace
 
-cudaError_t launch_grouped_gemm_pair(const CUtensorMap& wmap, const GemmArgs& a, int epilogue, int num_sms,
-                                     cudaStream_t stream) {
+cudaError_t launch_grouped_gemm_pair(const CUtensorMap& wmap, const CUtensorMap* rows_map, const GemmArgs& a,
+                                     int epilogue, int num_sms, cudaStream_t stream) {
+  // 256-row passes.  Measured alternatives with gathered rows (isolated
+  // kernel, in one process; 8192-token prefill shape / Zipf-skewed
+  // 4096-token shape):
+  //   gate/up 256/4: 1.58 / 3.58 ms; 192/5: 1.62 / 3.73 ms; 128/5: 2.56 / 4.52 ms
+  //   down    256/4: 1.12 / 2.07 ms; 192/5: 0.98 / 2.11 ms; 128/5: 1.45 / 2.33 ms
+  // but inside the layer, where h was just written and partly sits in L2,
+  // the 192/5 down GEMM measured slower (1.11 vs 1.07 ms; 2.32 vs 2.24 ms).
+  // One 256-column tile per unit with a double-buffered accumulator and
+  // gathered rows: down 1.03 / 2.35 ms.
+  // rows_map (the down GEMM's rows, contiguous): the rows by TMA, one box per
+  // stage and SM instead of 1024 row-chunk copies; in the layer, down
+  // 1.07-1.10 vs 1.12-1.16 ms (prefill) and 2.19-2.24 vs 2.22-2.23 ms
+  // (skewed).  With one 256-column tile per unit and double-buffered
+  // accumulators on top, the skewed shape lost 10% (h read twice as often).
+  if (rows_map != nullptr) {
+    if (a.row_index != nullptr || epilogue != EPI_STORE_F32) return cudaErrorInvalidValue;
+    return launch_pair<256, 4, 2, EPI_STORE_F32, true>(wmap, rows_map, a, num_sms, stream);
+  }
   switch (epilogue) {
-    // 256-row passes, 4 stages.  Measured alternatives (isolated kernel, in
-    // one process; 8192-token prefill shape / Zipf-skewed 4096-token shape):
-    //   gate/up 256/4: 1.58 / 3.58 ms; 192/5: 1.62 / 3.73 ms; 128/5: 2.56 / 4.52 ms
-    //   down    256/4: 1.12 / 2.07 ms; 192/5: 0.98 / 2.11 ms; 128/5: 1.45 / 2.33 ms
-    // but inside the layer, where h was just written and partly sits in L2,
-    // the 192/5 down GEMM measured slower (1.11 vs 1.07 ms; 2.32 vs 2.24 ms).
-    // One 256-column tile per unit with a double-buffered accumulator: down
-    // 1.03 / 2.35 ms.
-    case EPI_SWIGLU: return launch_pair<256, 4, 2, EPI_SWIGLU>(wmap, a, num_sms, stream);
-    case EPI_DOWN_COMBINE: return launch_pair<256, 4, 2, EPI_DOWN_COMBINE>(wmap, a, num_sms, stream);
-    case EPI_STORE_F32: return launch_pair<256, 4, 2, EPI_STORE_F32>(wmap, a, num_sms, stream);
+    case EPI_SWIGLU: return launch_pair<256, 4, 2, EPI_SWIGLU>(wmap, nullptr, a, num_sms, stream);
+    case EPI_DOWN_COMBINE: return launch_pair<256, 4, 2, EPI_DOWN_COMBINE>(wmap, nullptr, a, num_sms, stream);
+    case EPI_STORE_F32: return launch_pair<256, 4, 2, EPI_STORE_F32>(wmap, nullptr, a, num_sms, stream);
     default: return cudaErrorInvalidValue;  // the K split (and its SwiGLU reduction) runs on single SMs only
   }
 }

@@ -118,8 +118,12 @@ cudaError_t launch_grouped_gemm_mx(const CUtensorMap& code_map, const CUtensorMa
 // unit, two 128-column weight tiles per unit (the same n_blocks/col_stride/
 // col1_off/out_col_stride as the single-SM kernel with two tiles per unit);
 // output columns must come in whole chunks of 32 (n_valid % 32 == 0).
-cudaError_t launch_grouped_gemm_pair(const CUtensorMap& wmap, const GemmArgs& a, int epilogue, int num_sms,
-                                     cudaStream_t stream);
+// rows_map != nullptr: the rows are contiguous (a.row_index == nullptr) and
+// rows_map covers them (bf16 [1][src_rows][K], boxes of 64 x 128 x 1,
+// 128-byte swizzle); each SM then loads its half of a unit's rows with one
+// TMA box per stage (EPI_STORE_F32 only).
+cudaError_t launch_grouped_gemm_pair(const CUtensorMap& wmap, const CUtensorMap* rows_map, const GemmArgs& a,
+                                     int epilogue, int num_sms, cudaStream_t stream);
 
 // tiles: MOE_TILES_SMALL or MOE_TILES_LARGE.
 cudaError_t launch_grouped_gemm(const CUtensorMap& wmap, const GemmArgs& a, int epilogue, int tiles,
