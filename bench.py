@@ -246,7 +246,8 @@ def layer_accounting(cfg, counts, mx=False):
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for f in ("grouped_gemm.cu", "grouped_gemm_pair.cu", "gemm_units.cuh", "common.cuh", "kernels.h"):
+    for f in ("grouped_gemm.cu", "grouped_gemm_pair.cu", "gemm_pipeline.cuh", "gemm_units.cuh", "common.cuh",
+              "kernels.h"):
         h.update(open(os.path.join(ROOT, "routed_expert_ffn_prefix_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
