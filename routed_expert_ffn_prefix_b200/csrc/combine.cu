@@ -40,8 +40,12 @@ struct Vec<float> {
     }
   }
 };
-template <typename OT>
-__global__ void __launch_bounds__(kThreads) combine_kernel(const OT* __restrict__ o, const float* __restrict__ w,
+// SPLIT: the down GEMM's K was split (nsplit > 1 slabs).  The plain path is
+// compiled for four resident blocks per SM (its loads in flight are what
+// paces it); the slab path keeps its registers.
+template <typename OT, bool SPLIT>
+__global__ void __launch_bounds__(kThreads, SPLIT ? 1 : 4)
+    combine_kernel(const OT* __restrict__ o, const float* __restrict__ w,
                                                          const int32_t* __restrict__ inv_perm,
                                                          const float* __restrict__ shared, int H, int k, int rows,
                                                          int nsplit, size_t split_stride,
@@ -69,7 +73,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const OT* __restrict_
     float acc[V];
 #pragma unroll
     for (int i = 0; i < V; ++i) acc[i] = 0.f;
-    if (nsplit == 1) {
+    if (!SPLIT) {
       // k independent row loads in flight together, then the slot-order sum
       int j = 0;
       for (; j + 8 <= k; j += 8) {
@@ -247,8 +251,10 @@ cudaError_t launch_combine_t(const OT* o, const float* topk_w, const int32_t* in
   for (int t0 = 0; t0 < T; t0 += 65535) {  // grid.y limit
     const dim3 grid(slices, T - t0 < 65535 ? T - t0 : 65535);
     const cudaError_t err =
-        launch_kernel(combine_kernel<OT>, grid, dim3(threads), 0, s, o, topk_w, inv_perm, shared, H, k, rows, nsplit,
-                      split_stride, reinterpret_cast<__nv_bfloat16*>(y), st, t0);
+        nsplit > 1 ? launch_kernel(combine_kernel<OT, true>, grid, dim3(threads), 0, s, o, topk_w, inv_perm, shared,
+                                   H, k, rows, nsplit, split_stride, reinterpret_cast<__nv_bfloat16*>(y), st, t0)
+                   : launch_kernel(combine_kernel<OT, false>, grid, dim3(threads), 0, s, o, topk_w, inv_perm, shared,
+                                   H, k, rows, nsplit, split_stride, reinterpret_cast<__nv_bfloat16*>(y), st, t0);
     if (err != cudaSuccess) return err;
   }
   return cudaSuccess;

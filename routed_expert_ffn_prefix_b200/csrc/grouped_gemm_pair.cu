@@ -18,9 +18,14 @@
 //   * down: the two tiles are 2 x 256 adjacent output columns.
 //
 // Rows by TMA (RTMA, the down GEMM): the operand rows are h, already in
-// expert order, so each SM loads its half of a unit's rows with one 2D TMA
-// box per stage (128 rows; rows past the unit's are loaded but not read by
-// the MMA) instead of gathering them row by row.
+// expert order, so each SM loads its half of a unit's rows with one TMA box
+// per stage (128 rows; rows past the unit's are loaded but not read by the
+// MMA) instead of gathering them row by row.  Its fp32 output rows leave by
+// TMA too: each epilogue warp stages 16 rows x 32 columns at a time in
+// shared memory and issues a bulk tensor store, so TMEM is released once the
+// rows are staged and the 164 KB per unit and SM drain while the next
+// unit's MMAs run (written by plain stores, all SMs' epilogues contended for
+// the write bandwidth at once and held the MMAs for ~8K cycles per unit).
 //
 // Synchronisation (cluster of 2; rank 0 = leader issues every MMA):
 //   full[s]  (leader): 128 cp.async arrivals of the leader's rows, the
@@ -66,7 +71,9 @@ struct PCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int NBUF = (2 * MT * NT <= 512) ? 2 : 1;  // accumulators double-buffered if they fit
   static constexpr int TMEM_COLS = 512;
-  static constexpr int SMEM_BYTES = ST * STAGE_BYTES + 512 + 4 * kPrefixInts + 1024;
+  static constexpr int OSTAGE_OFF = (ST * STAGE_BYTES + 512 + 4 * kPrefixInts + 1023) & ~1023;  // fp32 row staging
+  static constexpr int OSTAGE_BYTES = kPEpiWarps * 16 * 32 * 4;                // 16 rows x 32 columns per warp
+  static constexpr int SMEM_BYTES = OSTAGE_OFF + OSTAGE_BYTES + 1024;
   static_assert(NT % 32 == 0 && NT >= 32 && NT <= 256, "row pass must be 32..256, multiple of 32");
   static_assert(MT == 1 || MT == 2, "one or two MMA tiles per unit");
   static_assert(MT * NT * NBUF <= TMEM_COLS, "accumulators must fit in TMEM");
@@ -90,10 +97,6 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ void remote_arrive(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-
 // Relayed "rows landed" signal.  The rows were written to this SM's own
 // shared memory and are read by this SM's own tensor core (each SM computes
 // its half of M from its own A tile), and they have fully landed before the
@@ -103,6 +106,21 @@ __device__ __forceinline__ void remote_arrive(uint32_t cluster_addr) {
 __device__ __forceinline__ void remote_arrive_relaxed(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
+
+// Bulk tensor store of a shared-memory box (fp32 rows), tracked by this
+// thread's bulk-async group.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(map),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// this thread's bulk stores have finished reading their shared-memory sources
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// ... and are complete
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // TMA tile load whose completion is signalled on a barrier of either SM of the pair.
 __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
@@ -158,9 +176,11 @@ __device__ __forceinline__ void mma_commit_pair_leader(uint64_t* bar) {
 template <int NT, int ST, int MT, int EPI, bool RTMA>
 __global__ void __launch_bounds__(kPThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap rmap,
-                             const GemmArgs a) {
+                             const __grid_constant__ CUtensorMap omap, const GemmArgs a) {
   using C = PCfg<NT, ST, MT>;
   static_assert(!RTMA || C::ROWS == 128, "row boxes of 128 rows");
+  static_assert(!RTMA || EPI == EPI_STORE_F32, "rows and fp32 output rows by TMA: the down GEMM's store epilogue");
+  static_assert(C::OSTAGE_OFF % 1024 == 0, "staging aligned for bulk copies");
   static_assert(EPI != EPI_SWIGLU || MT == 2, "SwiGLU needs the gate and the up tile");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -201,7 +221,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
   }
   if (warp == kPEpiWarps && lane == 0) {
     prefetch_tmap(&wmap);
-    if (RTMA) prefetch_tmap(&rmap);
+    if (RTMA) {
+      prefetch_tmap(&rmap);
+      prefetch_tmap(&omap);
+    }
   }
   if (warp == 0) build_unit_prefix<NT>(a, ngroups, ustart, total_units);
   tc_fence_before();
@@ -266,19 +289,17 @@ __global__ void __launch_bounds__(kPThreads, 1)
           // rows map: 3D [1][src_rows][K], like the weight maps
           if constexpr (RTMA) tma_load_3d_pair(sA + C::A_BYTES, &rmap, fb, kt * kBK, un.row0 + my0, 0, pol_rows);
         }
-        if constexpr (RTMA) {
-          if (++stage == ST) { stage = 0; phase ^= 1u; }
-          continue;
-        }
+        if constexpr (!RTMA) {
 #pragma unroll
-        for (int i = 0; i < kRowsPerThread; ++i) {
-          if (src[i] >= 0) {
-            const int c = rsub + 16 * i;
-            cp_async_16(sb + c * 128 + ((chunk ^ (c & 7)) << 4), bsrc + (size_t)src[i] * a.K + kt * kBK + chunk * 8,
-                        pol_rows);
+          for (int i = 0; i < kRowsPerThread; ++i) {
+            if (src[i] >= 0) {
+              const int c = rsub + 16 * i;
+              cp_async_16(sb + c * 128 + ((chunk ^ (c & 7)) << 4),
+                          bsrc + (size_t)src[i] * a.K + kt * kBK + chunk * 8, pol_rows);
+            }
           }
+          cp_async_arrive_noinc(&rows_bar_base[stage]);
         }
-        cp_async_arrive_noinc(&rows_bar_base[stage]);
         if (++stage == ST) { stage = 0; phase ^= 1u; }
       }
     }
@@ -403,6 +424,32 @@ __global__ void __launch_bounds__(kPThreads, 1)
           } else {
             tmem_ld_2x16(tbase + c0, tbase + c0 + 16, v[0], v[0] + 16);
           }
+          if constexpr (RTMA) {
+            // whole 32-row chunks of in-range columns by bulk tensor stores (a
+            // box must not reach past the unit's rows: they are another
+            // expert's); a partial chunk by plain stores below
+            const int cb = col - lane;  // this warp's first column
+            if (nr == 32 && cb + (MT - 1) * a.out_col1_off + 32 <= a.n_valid) {
+              float* stg = reinterpret_cast<float*>(smem + C::OSTAGE_OFF) + warp * (16 * 32);
+#pragma unroll
+              for (int t = 0; t < MT; ++t) {
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                  if (lane == 0) bulk_wait_read_all();  // the previous box has left the buffer
+                  __syncwarp();
+#pragma unroll
+                  for (int j = 0; j < 16; ++j) stg[j * 32 + lane] = v[t][hh * 16 + j];
+                  fence_proxy_async_smem();
+                  __syncwarp();
+                  if (lane == 0) {
+                    tma_store_3d(&omap, stg, cb + t * a.out_col1_off, un.row0 + c0 + hh * 16, 0);
+                    bulk_commit();
+                  }
+                }
+              }
+              continue;
+            }
+          }
 #pragma unroll
           for (int t = 0; t < MT; ++t) {
             const int ct = col + t * a.out_col1_off;
@@ -415,9 +462,13 @@ __global__ void __launch_bounds__(kPThreads, 1)
           }
         }
       }
+      // TMEM is free once this warp's loads are done (tcgen05.wait::ld inside
+      // the loads), whatever its stores: a release at cluster scope would
+      // also wait for every global store above to drain (~1,200 cycles per
+      // unit, measured) while the next unit's MMAs wait for this arrival.
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) remote_arrive(tempty_leader + buf * 8);
+      if (lane == 0) remote_arrive_relaxed(tempty_leader + buf * 8);
       ++acc_it;
       if constexpr (EPI == EPI_DOWN_COMBINE) {
         // TMEM is released; now count this warp's stored rows and reduce the
@@ -431,6 +482,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
         for (int c0 = half * 32; c0 < un.rows; c0 += 64)
           arrive_rows<MT, EPI>(a, un.row0 + c0, min(32, un.rows - c0), chunk, cols);
       }
+    }
+    if constexpr (RTMA) {  // every bulk store of this warp complete before the block leaves
+      if (lane == 0) bulk_wait_all();
+      __syncwarp();
     }
   }
 
@@ -446,8 +501,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
 }
 
 template <int NT, int ST, int MT, int EPI, bool RTMA = false>
-cudaError_t launch_pair(const CUtensorMap& wmap, const CUtensorMap* rmap, const GemmArgs& a, int num_sms,
-                        cudaStream_t stream) {
+cudaError_t launch_pair(const CUtensorMap& wmap, const CUtensorMap* rmap, const CUtensorMap* omap, const GemmArgs& a,
+                        int num_sms, cudaStream_t stream) {
   using C = PCfg<NT, ST, MT>;
   auto kern = grouped_gemm_pair_kernel<NT, ST, MT, EPI, RTMA>;
   static std::atomic<int> configured[kMaxDevices];
@@ -481,13 +536,13 @@ cudaError_t launch_pair(const CUtensorMap& wmap, const CUtensorMap* rmap, const 
     });
     if (slots[dev] > 0 && 2 * slots[dev] < (int)cfg.gridDim.x) cfg.gridDim = dim3(2 * slots[dev], 1, 1);
   }
-  return cudaLaunchKernelEx(&cfg, kern, wmap, RTMA ? *rmap : wmap, a);
+  return cudaLaunchKernelEx(&cfg, kern, wmap, RTMA ? *rmap : wmap, RTMA ? *omap : wmap, a);
 }
 
 }  // namespace
 
-cudaError_t launch_grouped_gemm_pair(const CUtensorMap& wmap, const CUtensorMap* rows_map, const GemmArgs& a,
-                                     int epilogue, int num_sms, cudaStream_t stream) {
+cudaError_t launch_grouped_gemm_pair(const CUtensorMap& wmap, const CUtensorMap* rows_map, const CUtensorMap* out_map,
+                                     const GemmArgs& a, int epilogue, int num_sms, cudaStream_t stream) {
   // 256-row passes.  Measured alternatives with gathered rows (isolated
   // kernel, in one process; 8192-token prefill shape / Zipf-skewed
   // 4096-token shape):
@@ -503,13 +558,15 @@ cudaError_t launch_grouped_gemm_pair(const CUtensorMap& wmap, const CUtensorMap*
   // (skewed).  With one 256-column tile per unit and double-buffered
   // accumulators on top, the skewed shape lost 10% (h read twice as often).
   if (rows_map != nullptr) {
-    if (a.row_index != nullptr || epilogue != EPI_STORE_F32) return cudaErrorInvalidValue;
-    return launch_pair<256, 4, 2, EPI_STORE_F32, true>(wmap, rows_map, a, num_sms, stream);
+    if (a.row_index != nullptr || epilogue != EPI_STORE_F32 || out_map == nullptr || a.k_splits != 1)
+      return cudaErrorInvalidValue;
+    return launch_pair<256, 4, 2, EPI_STORE_F32, true>(wmap, rows_map, out_map, a, num_sms, stream);
   }
   switch (epilogue) {
-    case EPI_SWIGLU: return launch_pair<256, 4, 2, EPI_SWIGLU>(wmap, nullptr, a, num_sms, stream);
-    case EPI_DOWN_COMBINE: return launch_pair<256, 4, 2, EPI_DOWN_COMBINE>(wmap, nullptr, a, num_sms, stream);
-    case EPI_STORE_F32: return launch_pair<256, 4, 2, EPI_STORE_F32>(wmap, nullptr, a, num_sms, stream);
+    case EPI_SWIGLU: return launch_pair<256, 4, 2, EPI_SWIGLU>(wmap, nullptr, nullptr, a, num_sms, stream);
+    case EPI_DOWN_COMBINE:
+      return launch_pair<256, 4, 2, EPI_DOWN_COMBINE>(wmap, nullptr, nullptr, a, num_sms, stream);
+    case EPI_STORE_F32: return launch_pair<256, 4, 2, EPI_STORE_F32>(wmap, nullptr, nullptr, a, num_sms, stream);
     default: return cudaErrorInvalidValue;  // the K split (and its SwiGLU reduction) runs on single SMs only
   }
 }

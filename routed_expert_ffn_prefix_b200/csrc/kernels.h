@@ -121,9 +121,11 @@ cudaError_t launch_grouped_gemm_mx(const CUtensorMap& code_map, const CUtensorMa
 // rows_map != nullptr: the rows are contiguous (a.row_index == nullptr) and
 // rows_map covers them (bf16 [1][src_rows][K], boxes of 64 x 128 x 1,
 // 128-byte swizzle); each SM then loads its half of a unit's rows with one
-// TMA box per stage (EPI_STORE_F32 only).
-cudaError_t launch_grouped_gemm_pair(const CUtensorMap& wmap, const CUtensorMap* rows_map, const GemmArgs& a,
-                                     int epilogue, int num_sms, cudaStream_t stream);
+// TMA box per stage, and writes its fp32 output rows through out_map (fp32
+// [1][rows][ld_out], boxes of 32 x 16 x 1, no swizzle) by bulk tensor
+// stores (EPI_STORE_F32, no K split).
+cudaError_t launch_grouped_gemm_pair(const CUtensorMap& wmap, const CUtensorMap* rows_map, const CUtensorMap* out_map,
+                                     const GemmArgs& a, int epilogue, int num_sms, cudaStream_t stream);
 
 // tiles: MOE_TILES_SMALL or MOE_TILES_LARGE.
 cudaError_t launch_grouped_gemm(const CUtensorMap& wmap, const GemmArgs& a, int epilogue, int tiles,
