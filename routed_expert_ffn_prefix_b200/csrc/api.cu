@@ -168,11 +168,12 @@ EncodeTiledFn encode_fn() {
 //              over the box row (64 or 128 bytes);
 //   kMapScales: u8 E8M0 scales, box 128 x 2*kMxRawSteps x 1, no swizzle;
 //   kMapRows:  bf16 rows [rows][K] (K contiguous), box 64 x 128 x 1, 128-byte swizzle;
-//   kMapOutF32: fp32 rows [rows][N] (N contiguous), box 32 x 16 x 1, no swizzle (bulk stores).
+//   kMapOutF32: fp32 rows [rows][N] (N contiguous), box 32 x 16 x 1, no swizzle (bulk stores);
+//   kMapOutBf16: bf16 rows [rows][N], box 32 x 16 x 1, no swizzle (bulk stores).
 // A descriptor depends only on (kind, address, extents), so the last few
 // are memoised: a steady stream of calls on the same weights skips the
 // encode.
-enum MapKind { kMapBf16 = 0, kMapCodes = 1, kMapScales = 2, kMapRows = 3, kMapOutF32 = 4 };
+enum MapKind { kMapBf16 = 0, kMapCodes = 1, kMapScales = 2, kMapRows = 3, kMapOutF32 = 4, kMapOutBf16 = 5 };
 struct MapCacheEntry {
   const void* base;
   uint64_t d0, d1, d2;
@@ -187,13 +188,14 @@ int g_map_next = 0;
 bool encode_map(CUtensorMap* m, int kind, const void* base, uint64_t d0, uint64_t d1, uint64_t d2) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  const bool bf16 = kind == kMapBf16 || kind == kMapRows;
+  const bool out = kind == kMapOutF32 || kind == kMapOutBf16;  // bulk-store boxes of 32 x 16, no swizzle
+  const bool bf16 = kind == kMapBf16 || kind == kMapRows || kind == kMapOutBf16;
   const bool f32 = kind == kMapOutF32;
   const uint64_t esz = bf16 ? 2 : f32 ? 4 : 1;
   cuuint64_t dims[3] = {d0, d1, d2};
   cuuint64_t strides[2] = {d0 * esz, d0 * d1 * esz};
-  cuuint32_t box[3] = {bf16 ? 64u : f32 ? 32u : kind == kMapScales ? 128u : 64u * kMxRawSteps,
-                       kind == kMapBf16 ? 64u : f32 ? 16u : kind == kMapScales ? 2u * kMxRawSteps : 128u, 1};
+  cuuint32_t box[3] = {out ? 32u : bf16 ? 64u : kind == kMapScales ? 128u : 64u * kMxRawSteps,
+                       out ? 16u : kind == kMapBf16 ? 64u : kind == kMapScales ? 2u * kMxRawSteps : 128u, 1};
   const CUtensorMapSwizzle code_swizzle = kMxRawSteps == 1 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m,
@@ -201,8 +203,9 @@ bool encode_map(CUtensorMap* m, int kind, const void* base, uint64_t d0, uint64_
              : f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                    : CU_TENSOR_MAP_DATA_TYPE_UINT8,
              3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             bf16 ? CU_TENSOR_MAP_SWIZZLE_128B
-                              : kind == kMapCodes ? code_swizzle : CU_TENSOR_MAP_SWIZZLE_NONE,
+             out    ? CU_TENSOR_MAP_SWIZZLE_NONE
+             : bf16 ? CU_TENSOR_MAP_SWIZZLE_128B
+                    : kind == kMapCodes ? code_swizzle : CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -439,7 +442,11 @@ moe_status_t run_swiglu(const uint16_t* x, int src_rows, const uint16_t* w_gate_
     a.n_blocks = (I + 255) / 256;
     a.col_stride = 256;
     a.out_col_stride = 256;
-    return cuda_status(launch_grouped_gemm_pair(map, nullptr, nullptr, a, EPI_SWIGLU, dev.num_sms, s));
+    // h [rows, I] bf16 leaves by bulk tensor stores (boxes of 16 rows)
+    CUtensorMap hmap;
+    const bool h_tma = rows >= 16;
+    if (h_tma && !make_map(&hmap, kMapOutBf16, h, (uint64_t)I, (uint64_t)rows, 1)) return MOE_ERR_CUDA;
+    return cuda_status(launch_grouped_gemm_pair(map, nullptr, h_tma ? &hmap : nullptr, a, EPI_SWIGLU, dev.num_sms, s));
   }
   const GemmArgs a = gate_up_args(x, src_rows, offsets, row_index, rows, H, E, I, h, st, nsplit, partials, arrivals);
   if (nsplit > 1) {

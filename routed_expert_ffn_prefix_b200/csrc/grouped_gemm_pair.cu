@@ -20,12 +20,13 @@
 // Rows by TMA (RTMA, the down GEMM): the operand rows are h, already in
 // expert order, so each SM loads its half of a unit's rows with one TMA box
 // per stage (128 rows; rows past the unit's are loaded but not read by the
-// MMA) instead of gathering them row by row.  Its fp32 output rows leave by
-// TMA too: each epilogue warp stages 16 rows x 32 columns at a time in
+// MMA) instead of gathering them row by row.
+// Output rows by TMA (OTMA: the down GEMM's fp32 rows, the gate/up GEMM's
+// bf16 h rows): each epilogue warp stages 16 rows x 32 columns at a time in
 // shared memory and issues a bulk tensor store, so TMEM is released once the
-// rows are staged and the 164 KB per unit and SM drain while the next
-// unit's MMAs run (written by plain stores, all SMs' epilogues contended for
-// the write bandwidth at once and held the MMAs for ~8K cycles per unit).
+// rows are staged and the stores drain while the next unit's MMAs run
+// (written by plain stores, all SMs' epilogues contended for the write
+// bandwidth at once and held the MMAs for ~8K cycles per down unit).
 //
 // Synchronisation (cluster of 2; rank 0 = leader issues every MMA):
 //   full[s]  (leader): 128 cp.async arrivals of the leader's rows, the
@@ -173,13 +174,14 @@ __device__ __forceinline__ void mma_commit_pair_leader(uint64_t* bar) {
       : "memory");
 }
 
-template <int NT, int ST, int MT, int EPI, bool RTMA>
+template <int NT, int ST, int MT, int EPI, bool RTMA, bool OTMA>
 __global__ void __launch_bounds__(kPThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap rmap,
                              const __grid_constant__ CUtensorMap omap, const GemmArgs a) {
   using C = PCfg<NT, ST, MT>;
   static_assert(!RTMA || C::ROWS == 128, "row boxes of 128 rows");
-  static_assert(!RTMA || EPI == EPI_STORE_F32, "rows and fp32 output rows by TMA: the down GEMM's store epilogue");
+  static_assert(!RTMA || EPI == EPI_STORE_F32, "rows by TMA: the down GEMM's store epilogue");
+  static_assert(!OTMA || EPI == EPI_STORE_F32 || EPI == EPI_SWIGLU, "output rows by TMA: fp32 rows or h");
   static_assert(C::OSTAGE_OFF % 1024 == 0, "staging aligned for bulk copies");
   static_assert(EPI != EPI_SWIGLU || MT == 2, "SwiGLU needs the gate and the up tile");
   extern __shared__ uint8_t smem_raw[];
@@ -221,10 +223,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
   }
   if (warp == kPEpiWarps && lane == 0) {
     prefetch_tmap(&wmap);
-    if (RTMA) {
-      prefetch_tmap(&rmap);
-      prefetch_tmap(&omap);
-    }
+    if (RTMA) prefetch_tmap(&rmap);
+    if (OTMA) prefetch_tmap(&omap);
   }
   if (warp == 0) build_unit_prefix<NT>(a, ngroups, ustart, total_units);
   tc_fence_before();
@@ -407,6 +407,27 @@ __global__ void __launch_bounds__(kPThreads, 1)
         if (EPI == EPI_SWIGLU) {
           float g[32], v[32];
           tmem_ld_4x16(tbase + c0, tbase + c0 + 16, tbase + NT + c0, tbase + NT + c0 + 16, g, g + 16, v, v + 16);
+          if constexpr (OTMA) {  // whole 32-row chunks by bulk tensor stores, as the fp32 rows below
+            const int cb = col - lane;
+            if (nr == 32 && cb + 32 <= a.n_valid) {
+              __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(smem + C::OSTAGE_OFF) + warp * (16 * 32);
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                if (lane == 0) bulk_wait_read_all();
+                __syncwarp();
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                  stg[j * 32 + lane] = __float2bfloat16_rn(silu_f(g[hh * 16 + j]) * v[hh * 16 + j]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                  tma_store_3d(&omap, stg, cb, un.row0 + c0 + hh * 16, 0);
+                  bulk_commit();
+                }
+              }
+              continue;
+            }
+          }
           __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
           if (col < a.n_valid) {
 #pragma unroll
@@ -424,7 +445,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
           } else {
             tmem_ld_2x16(tbase + c0, tbase + c0 + 16, v[0], v[0] + 16);
           }
-          if constexpr (RTMA) {
+          if constexpr (OTMA) {
             // whole 32-row chunks of in-range columns by bulk tensor stores (a
             // box must not reach past the unit's rows: they are another
             // expert's); a partial chunk by plain stores below
@@ -483,7 +504,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
           arrive_rows<MT, EPI>(a, un.row0 + c0, min(32, un.rows - c0), chunk, cols);
       }
     }
-    if constexpr (RTMA) {  // every bulk store of this warp complete before the block leaves
+    if constexpr (OTMA) {  // every bulk store of this warp complete before the block leaves
       if (lane == 0) bulk_wait_all();
       __syncwarp();
     }
@@ -500,11 +521,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
   }
 }
 
-template <int NT, int ST, int MT, int EPI, bool RTMA = false>
+template <int NT, int ST, int MT, int EPI, bool RTMA = false, bool OTMA = false>
 cudaError_t launch_pair(const CUtensorMap& wmap, const CUtensorMap* rmap, const CUtensorMap* omap, const GemmArgs& a,
                         int num_sms, cudaStream_t stream) {
   using C = PCfg<NT, ST, MT>;
-  auto kern = grouped_gemm_pair_kernel<NT, ST, MT, EPI, RTMA>;
+  auto kern = grouped_gemm_pair_kernel<NT, ST, MT, EPI, RTMA, OTMA>;
   static std::atomic<int> configured[kMaxDevices];
   cudaError_t err = once_per_device(configured, [&] {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -536,7 +557,7 @@ cudaError_t launch_pair(const CUtensorMap& wmap, const CUtensorMap* rmap, const 
     });
     if (slots[dev] > 0 && 2 * slots[dev] < (int)cfg.gridDim.x) cfg.gridDim = dim3(2 * slots[dev], 1, 1);
   }
-  return cudaLaunchKernelEx(&cfg, kern, wmap, RTMA ? *rmap : wmap, RTMA ? *omap : wmap, a);
+  return cudaLaunchKernelEx(&cfg, kern, wmap, RTMA ? *rmap : wmap, OTMA ? *omap : wmap, a);
 }
 
 }  // namespace
@@ -560,7 +581,11 @@ cudaError_t launch_grouped_gemm_pair(const CUtensorMap& wmap, const CUtensorMap*
   if (rows_map != nullptr) {
     if (a.row_index != nullptr || epilogue != EPI_STORE_F32 || out_map == nullptr || a.k_splits != 1)
       return cudaErrorInvalidValue;
-    return launch_pair<256, 4, 2, EPI_STORE_F32, true>(wmap, rows_map, out_map, a, num_sms, stream);
+    return launch_pair<256, 4, 2, EPI_STORE_F32, true, true>(wmap, rows_map, out_map, a, num_sms, stream);
+  }
+  if (out_map != nullptr) {
+    if (epilogue != EPI_SWIGLU || a.k_splits != 1) return cudaErrorInvalidValue;
+    return launch_pair<256, 4, 2, EPI_SWIGLU, false, true>(wmap, nullptr, out_map, a, num_sms, stream);
   }
   switch (epilogue) {
     case EPI_SWIGLU: return launch_pair<256, 4, 2, EPI_SWIGLU>(wmap, nullptr, nullptr, a, num_sms, stream);

@@ -123,7 +123,9 @@ cudaError_t launch_grouped_gemm_mx(const CUtensorMap& code_map, const CUtensorMa
 // 128-byte swizzle); each SM then loads its half of a unit's rows with one
 // TMA box per stage, and writes its fp32 output rows through out_map (fp32
 // [1][rows][ld_out], boxes of 32 x 16 x 1, no swizzle) by bulk tensor
-// stores (EPI_STORE_F32, no K split).
+// stores (EPI_STORE_F32, no K split).  rows_map == nullptr, out_map !=
+// nullptr: EPI_SWIGLU writes h through out_map (bf16 [1][rows][ld_out],
+// boxes of 32 x 16 x 1) the same way.
 cudaError_t launch_grouped_gemm_pair(const CUtensorMap& wmap, const CUtensorMap* rows_map, const CUtensorMap* out_map,
                                      const GemmArgs& a, int epilogue, int num_sms, cudaStream_t stream);
 
