@@ -107,3 +107,54 @@ def test_dtype_layout_workspace_and_shared_expert_errors():
         moe.forward(x, wr, None, wgu, wd, k, ws(), t(H, 2 * I_s), None)
     with pytest.raises(TypeError, match="torch.Tensor"):
         moe.route([[0.0]], wr, None, k, ws())
+
+
+MH, MI = 512, 128  # H != 2I, so a [E, K, N] code tensor cannot pass for [E, N, K]
+
+
+def mx_args():
+    """Block-scaled FP8 weights in the library's layout: codes of W^T [E, N, K]
+    (K contiguous), scales [E, K/32, N]."""
+    u8 = torch.uint8
+    return dict(x=t(T, MH), w_router=t(MH, E, dtype=f32), bias=None,
+                gu_codes=t(E, 2 * MI, MH, dtype=u8), gu_scales=t(E, MH // 32, 2 * MI, dtype=u8),
+                dn_codes=t(E, MH, MI, dtype=u8), dn_scales=t(E, MI // 32, MH, dtype=u8))
+
+
+def call_mx(a, **kw):
+    return moe.forward_mx(a["x"], a["w_router"], a["bias"], a["gu_codes"], a["gu_scales"], a["dn_codes"],
+                          a["dn_scales"], k, ws(), **kw)
+
+
+def test_forward_mx_valid_calls_stop_at_the_device_check():
+    only_device_error(call_mx, mx_args())
+    only_device_error(call_mx, mx_args(), tiles=moe.TILES_SMALL, combine=moe.COMBINE_SEPARATE)
+    a = mx_args()
+    only_device_error(moe.forward_mx, a["x"], a["w_router"], t(E, dtype=f32), a["gu_codes"], a["gu_scales"],
+                      a["dn_codes"], a["dn_scales"], k, ws(), t(MH, 2 * I_s), t(I_s, MH))
+
+
+@pytest.mark.parametrize("what", [
+    "gu_codes_not_transposed", "dn_codes_not_transposed", "gu_scales_transposed", "dn_scales_wrong_blocks",
+])
+def test_forward_mx_refuses_wrong_weight_layouts(what):
+    a = mx_args()
+    u8 = torch.uint8
+    if what == "gu_codes_not_transposed":      # [E, K, N] is the bf16 layout, not the FP8 one
+        a["gu_codes"] = t(E, MH, 2 * MI, dtype=u8)
+    elif what == "dn_codes_not_transposed":
+        a["dn_codes"] = t(E, MI, MH, dtype=u8)
+    elif what == "gu_scales_transposed":
+        a["gu_scales"] = t(E, 2 * MI, MH // 32, dtype=u8)
+    elif what == "dn_scales_wrong_blocks":
+        a["dn_scales"] = t(E, MI // 16, MH, dtype=u8)
+    with pytest.raises(ValueError):
+        call_mx(a)
+
+
+@pytest.mark.parametrize("which", ["gu_codes", "dn_scales"])
+def test_forward_mx_refuses_non_byte_weights(which):
+    a = mx_args()
+    a[which] = a[which].to(torch.int8 if which == "gu_codes" else bf)
+    with pytest.raises(TypeError, match="must be torch.uint8"):
+        call_mx(a)
