@@ -268,7 +268,7 @@ def recorded_traffic(workload):
 
 
 # ---------------------------------------------------------------- timed runs
-TILES = {"auto": 0, "small": 1, "large": 2, "pair": 3, "fused": 4, "persistent": 5}
+TILES = {"auto": 0, "small": 1, "large": 2, "pair": 3, "persistent": 4}
 COMBINE = {"auto": 0, "fused": 1, "separate": 2}
 # further workloads timed with the default workload, reported under "extra" (their weights
 # replace the decode ones after the decode and prefill measurements)

@@ -87,12 +87,7 @@ enum {
   MOE_TILES_LARGE = 2,  /* <= 256 token rows per tile pass, 3-stage ring: prefill */
   MOE_TILES_PAIR = 3,   /* SM pairs (2-SM tcgen05 MMA): 256 weight columns per MMA, 128 per SM; <= 256
                            token rows per pass, half gathered by each SM; 4-stage ring: prefill */
-  MOE_TILES_FUSED = 4,  /* moe_forward_ex only, T <= 4: the whole layer (routing, permutation, both
-                           expert matrix-vector products, combine) in one cooperative launch with
-                           grid barriers; CUDA-core weight streams.  Needs k <= 16, E % 4 == 0,
-                           H, I, I_s multiples of 256, H <= 8192, I, I_s <= 4096.  Never chosen
-                           by AUTO (measured slower than SMALL with its K split). */
-  MOE_TILES_PERSISTENT = 5 /* moe_forward_ex only, T <= 16, E % 4 == 0, no shared expert: the whole
+  MOE_TILES_PERSISTENT = 4 /* moe_forward_ex only, T <= 16, E % 4 == 0, no shared expert: the whole
                               layer in one persistent launch on the tensor cores -- the few-token
                               router, then the gate/up and the down grouped GEMM as one sequence of
                               work units (a down unit starts once its expert's gate/up units are
@@ -162,15 +157,14 @@ int moe_abi_version(void);
  *   o_shared [T, H] f32,
  *   logits [S, T, E] f32 (S router partial slabs), router_split [3, H, E]
  *   bf16, block_hist (permute), split: K-split partial slabs of the expert
- *   GEMMs when few tokens leave SMs idle (f32; 0 bytes when unused), fused:
- *   partial slabs of the one-launch layer for T <= 4 (f32; 0 bytes above),
+ *   GEMMs when few tokens leave SMs idle (f32; 0 bytes when unused),
  *   arrivals: u32 counters of the combine in the down GEMM's epilogue (one
  *   per token and 64 output columns) and of a K-split gate/up GEMM's
  *   SwiGLU (one per row and 32 intermediate columns).  Each layer call
  *   zeroes them in its routing kernel and leaves them zero. */
 typedef struct moe_workspace_layout {
   size_t status, topk_ids, topk_w, counts, offsets, sorted_token_ids, inv_perm;
-  size_t h, o, h_shared, o_shared, logits, router_split, block_hist, split, fused;
+  size_t h, o, h_shared, o_shared, logits, router_split, block_hist, split;
   size_t arrivals;
   size_t total;
 } moe_workspace_layout_t;
@@ -342,8 +336,8 @@ moe_status_t moe_forward_ex(const uint16_t *x, const float *w_router, const floa
  * computes exactly what moe_forward_ex computes on the dequantised weights,
  * with the same rounding points; only the expert-weight bytes halve (plus
  * 1/32 for the scales).  Below scale code 3 a weight smaller than bf16's
- * least subnormal step is rounded to nearest bf16.  Everything else as moe_forward_ex, except: tile policies FUSED
- * and PERSISTENT and MOE_COMBINE_FUSED are not available
+ * least subnormal step is rounded to nearest bf16.  Everything else as moe_forward_ex, except: the tile policy
+ * PERSISTENT and MOE_COMBINE_FUSED are not available
  * (MOE_ERR_INVALID_ARG), and PAIR runs as LARGE (single-SM 256-row passes).
  * The two E4M3 NaN patterns are not supported as weights (they decode as
  * +-480, not NaN).  Codes and scales pointers 16-byte aligned. */

@@ -16,7 +16,7 @@ import os
 from . import build as _build
 
 __all__ = [
-    "MoEError", "lib", "TILES_AUTO", "TILES_SMALL", "TILES_LARGE", "TILES_PAIR", "TILES_FUSED", "TILES_PERSISTENT",
+    "MoEError", "lib", "TILES_AUTO", "TILES_SMALL", "TILES_LARGE", "TILES_PAIR", "TILES_PERSISTENT",
     "ROUTER_AUTO", "ROUTER_FMA", "ROUTER_TC", "ROUTER_SMALL",
     "SCORE_SOFTMAX", "SCORE_SOFTMAX_SELECT_BIAS", "SCORE_SIGMOID",
     "COMBINE_AUTO", "COMBINE_FUSED", "COMBINE_SEPARATE",
@@ -25,7 +25,7 @@ __all__ = [
     "STATUS",
 ]
 
-TILES_AUTO, TILES_SMALL, TILES_LARGE, TILES_PAIR, TILES_FUSED, TILES_PERSISTENT = 0, 1, 2, 3, 4, 5
+TILES_AUTO, TILES_SMALL, TILES_LARGE, TILES_PAIR, TILES_PERSISTENT = 0, 1, 2, 3, 4
 ROUTER_AUTO, ROUTER_FMA, ROUTER_TC, ROUTER_SMALL = 0, 1, 2, 3
 SCORE_SOFTMAX, SCORE_SOFTMAX_SELECT_BIAS, SCORE_SIGMOID = 0, 1, 2
 COMBINE_AUTO, COMBINE_FUSED, COMBINE_SEPARATE = 0, 1, 2
@@ -44,7 +44,7 @@ class MoEError(RuntimeError):
 class _Layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "status", "topk_ids", "topk_w", "counts", "offsets", "sorted_token_ids", "inv_perm",
-        "h", "o", "h_shared", "o_shared", "logits", "router_split", "block_hist", "split", "fused", "arrivals",
+        "h", "o", "h_shared", "o_shared", "logits", "router_split", "block_hist", "split", "arrivals",
         "total")]
 
 

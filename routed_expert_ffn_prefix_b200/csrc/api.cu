@@ -131,14 +131,6 @@ moe_workspace_layout_t make_layout(int T, int H, int E, int I, int k, int I_s) {
   // gate/up slabs, then down slabs (the persistent few-token layer holds both at once)
   const SplitPlan sp = split_plan(T, H, E, I, k, MOE_TILES_SMALL);
   L.split = take((split_gate_up_elems(T, I, k, sp) + split_down_elems(T, H, k, sp)) * 4);
-  // slabs of the one-launch few-token layer
-  size_t fused = 0;
-  if (T <= kFusedMaxT && H > 0 && I > 0) {
-    const size_t frows = tk + (I_s > 0 ? (size_t)T : 0);
-    const size_t imax = (size_t)(I > I_s ? I : I_s);
-    fused = (size_t)kFusedMaxSplit * frows * (2 * imax + H) * 4;
-  }
-  L.fused = take(fused);
   L.arrivals = take(arrival_words(T, H, E, I, k) * 4);
   L.total = off;
   return L;
@@ -576,7 +568,7 @@ moe_status_t forward_impl(const uint16_t* x, const float* w_router, const float*
   if (tile_policy < MOE_TILES_AUTO || tile_policy > MOE_TILES_PERSISTENT) return MOE_ERR_INVALID_ARG;
   if (router_impl < MOE_ROUTER_AUTO || router_impl > MOE_ROUTER_SMALL) return MOE_ERR_INVALID_ARG;
   if (!valid_scoring(scoring)) return MOE_ERR_INVALID_ARG;
-  if (mx && (tile_policy == MOE_TILES_FUSED || tile_policy == MOE_TILES_PERSISTENT || combine == MOE_COMBINE_FUSED))
+  if (mx && (tile_policy == MOE_TILES_PERSISTENT || combine == MOE_COMBINE_FUSED))
     return MOE_ERR_INVALID_ARG;  // the FP8 kernel runs the multi-kernel layer with the combine kernel
   if (!all_aligned(x, w_router, y) || (bias && !aligned16(bias))) return MOE_ERR_ALIGNMENT;
   if (mx ? !all_aligned(mx_gu->codes, mx_gu->scales, mx_dn->codes, mx_dn->scales) : !all_aligned(w_gate_up, w_down))
@@ -604,25 +596,6 @@ moe_status_t forward_impl(const uint16_t* x, const float* w_router, const float*
     return MOE_OK;
   };
   int launches = 0;
-
-  // A few tokens, on request: the whole layer in one cooperative launch.
-  if (tile_policy == MOE_TILES_FUSED) {
-    if (!fused_decode_supported(T, H, E, I, k, shared ? I_s : 0)) return MOE_ERR_INVALID_ARG;
-    float* slabs = at<float>(ws, L.fused);
-    const size_t frows = (size_t)rows + (shared ? (size_t)T : 0);
-    const int imax = I > I_s ? I : I_s;
-    float* gslabs = slabs;
-    float* dslabs = slabs + (size_t)kFusedMaxSplit * frows * 2 * imax;
-    MOE_TRY(mark(0));
-    MOE_TRY(cuda_status(launch_fused_decode(x, w_router, bias, scoring, w_gate_up, w_down,
-                                            shared ? w_sh_gate_up : nullptr, shared ? w_sh_down : nullptr,
-                                            shared ? I_s : 0, T, H, E, I, k,
-                                            at<float>(ws, L.logits), gslabs, dslabs, ids, tw, counts, offs, sids, inv,
-                                            y, st, kDefaultTimeoutNs, dev.num_sms, s)));
-    for (int i = 1; i < 7; ++i) MOE_TRY(mark(i));
-    if (options) options->launches = 1;
-    return MOE_OK;
-  }
 
   // A few tokens, on request: the whole layer in one persistent launch on the tensor cores.
   if (tile_policy == MOE_TILES_PERSISTENT) {

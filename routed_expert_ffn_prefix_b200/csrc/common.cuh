@@ -37,8 +37,7 @@ enum Site : int32_t {
   SITE_COMBINE = 7,
   SITE_SELFTEST = 8,
   SITE_TOPK = 9,
-  SITE_FUSED = 10,
-  SITE_LAYER = 11,
+  SITE_LAYER = 10,
 };
 
 __device__ __forceinline__ void raise_error(DevStatus* st, int code, int site, int aux) {

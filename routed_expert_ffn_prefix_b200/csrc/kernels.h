@@ -185,23 +185,6 @@ cudaError_t launch_swiglu_reduce(const float* partials, int nsplit, size_t split
 // would.  *arrivals must be zero on entry and is zero again on exit.
 constexpr int kSmallRouterT = 16;
 
-// The whole layer for T <= kFusedMaxT tokens in one cooperative launch
-// (fused_decode.cu): k <= kFusedMaxK, E % 4 == 0, H, I, I_s multiples of 256,
-// H <= 8192, I, I_s <= 4096.  Scratch: router slabs [small_router_slabs][T][E],
-// gate/up slabs [kFusedMaxSplit][rows][2][max(I, I_s)] and down slabs
-// [kFusedMaxSplit][rows][H] (f32; rows = T*k (+ T with a shared expert)).
-// The grid-barrier word of the status block must be zero on entry; it is
-// zero again on exit.
-constexpr int kFusedMaxT = 4;
-constexpr int kFusedMaxK = 16;
-constexpr int kFusedMaxSplit = 8;
-bool fused_decode_supported(int T, int H, int E, int I, int k, int I_s);
-cudaError_t launch_fused_decode(const uint16_t* x, const float* w_router, const float* bias, int scoring,
-                                const uint16_t* w_gate_up, const uint16_t* w_down, const uint16_t* w_sh_gate_up,
-                                const uint16_t* w_sh_down, int I_s, int T, int H, int E, int I, int k,
-                                float* rslabs, float* gslabs, float* dslabs, int32_t* ids, float* tw,
-                                int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* inv_perm,
-                                uint16_t* y, DevStatus* st, uint64_t timeout_ns, int num_sms, cudaStream_t s);
 int small_router_slabs(int H, int E);
 cudaError_t launch_router_small(const uint16_t* x, const float* w, const float* bias, int T, int H, int E, int k,
                                 int scoring, float* partial, unsigned int* arrivals, int32_t* ids, float* wout,

@@ -1,5 +1,5 @@
 // route_dev.cuh -- device pieces of the router shared by the router kernels
-// (route.cu) and the one-launch few-token layer (fused_decode.cu): the warp
+// (route.cu) and the persistent few-token layer (layer_small.cu): the warp
 // top-k and the split-H partial logits of a few tokens.
 #pragma once
 

@@ -48,15 +48,15 @@ def test_workspace_layout_is_ordered_and_aligned(lib):
     L = moe.workspace_layout(8192, 4096, 512, 1024, 10)
     offs = [L[n] for n in ("status", "topk_ids", "topk_w", "counts", "offsets", "sorted_token_ids",
                            "inv_perm", "block_hist", "logits", "router_split", "h", "o", "h_shared",
-                           "o_shared", "split", "fused", "arrivals", "total")]
+                           "o_shared", "split", "arrivals", "total")]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
     assert L["o"] - L["h"] >= 81920 * 1024 * 2          # h: [T*k, I] bf16
     assert L["h_shared"] - L["o"] >= 81920 * 4096 * 4   # o: [T*k, H] f32
     assert moe.workspace_size(8192, 4096, 512, 1024, 10) == L["total"]
     Ls = moe.workspace_layout(4096, 8192, 256, 2048, 8, 2048)
     assert Ls["split"] - Ls["o_shared"] >= 4096 * 8192 * 4
-    # many tokens: no K split and no one-launch layer, so no partial slabs
-    assert L["arrivals"] == L["fused"] == L["split"] and Ls["arrivals"] == Ls["fused"] == Ls["split"]
+    # many tokens: no K split, so no partial slabs
+    assert L["arrivals"] == L["split"] and Ls["arrivals"] == Ls["split"]
     # arrival counters of the combine in the down GEMM (one per token and 64 output columns) and one
     # done-counter per expert and 128-column gate/up block, rounded up to 256 bytes
     assert L["total"] - L["arrivals"] == (8192 * (4096 // 64) + 512 * 8 + 63) // 64 * 256
@@ -69,9 +69,7 @@ def test_workspace_layout_reserves_k_split_slabs_for_one_token(lib):
     148 SMs.  The split region holds both: 3 x 8 rows x 3072 and 2 x 8 rows x 4096 f32."""
     L = moe.workspace_layout(1, 4096, 256, 1536, 8)
     # gate/up slabs, then down slabs (the persistent few-token layer holds both)
-    assert L["fused"] - L["split"] == (3 * 8 * 3072 + 2 * 8 * 4096) * 4
-    # the one-launch layer (T <= 4): 8 K slices of gate/up (2 x I) and down (H) rows, f32
-    assert L["arrivals"] - L["fused"] == 8 * 8 * (2 * 1536 + 4096) * 4
+    assert L["arrivals"] - L["split"] == (3 * 8 * 3072 + 2 * 8 * 4096) * 4
     # arrival counters: the K-split gate/up's (8 rows x 1536/32 chunks), the down's (1 x 4096/64) and one
     # per expert and 128-column gate/up block, side by side, rounded up to 256 bytes
     assert L["total"] - L["arrivals"] == (8 * 1536 // 32 + 4096 // 64 + 256 * 12 + 63) // 64 * 256

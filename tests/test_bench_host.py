@@ -78,7 +78,7 @@ def test_recorded_traffic_follows_the_source_hash():
 
 def test_option_tables_mirror_the_library_constants():
     assert bench.TILES == {"auto": moe.TILES_AUTO, "small": moe.TILES_SMALL, "large": moe.TILES_LARGE,
-                           "pair": moe.TILES_PAIR, "fused": moe.TILES_FUSED, "persistent": moe.TILES_PERSISTENT}
+                           "pair": moe.TILES_PAIR, "persistent": moe.TILES_PERSISTENT}
     assert bench.COMBINE == {"auto": moe.COMBINE_AUTO, "fused": moe.COMBINE_FUSED,
                              "separate": moe.COMBINE_SEPARATE}
     assert bench.SCORING == {"softmax": moe.SCORE_SOFTMAX, "softmax_select_bias": moe.SCORE_SOFTMAX_SELECT_BIAS,

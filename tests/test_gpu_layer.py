@@ -34,7 +34,7 @@ CASES = {
         Config("three_shared", T=3, H=768, E=32, I=128, k=4, I_s=128),
         Config("few_bias", T=7, H=1024, E=128, I=256, k=6, bias="zipf:1.2"),  # biased few-token routing
         # the one-launch layer: shared expert, biased routing, experts chosen by several tokens
-        Config("fused_shared", T=4, H=512, E=16, I=256, k=4, I_s=256, bias="zipf:1.2"),
+        Config("few_shared", T=4, H=512, E=16, I=256, k=4, I_s=256, bias="zipf:1.2"),
         # edge cases: E % 4 != 0 above 128 experts (scalar 8-per-lane top-k), the largest k
         # (k = E = 64: every token takes every expert), and k = 1 (every weight exactly 1)
         Config("odd_e130", T=40, H=256, E=130, I=128, k=5),
@@ -162,24 +162,16 @@ def test_grouped_down_single_group():
     assert_close_output(host_f64(o), want, "o")
 
 
-def fused_ok(cfg):
-    return (cfg.T <= 4 and cfg.k <= 16 and cfg.E % 4 == 0 and cfg.H % 256 == 0 and cfg.I % 256 == 0
-            and cfg.I_s % 256 == 0)
-
-
 def persistent_ok(cfg):
     return cfg.T <= 16 and cfg.E % 4 == 0 and cfg.I_s == 0
 
 
 @pytest.mark.parametrize("router", [moe.ROUTER_FMA, moe.ROUTER_TC, moe.ROUTER_SMALL])
-@pytest.mark.parametrize("tiles", [moe.TILES_SMALL, moe.TILES_LARGE, moe.TILES_PAIR, moe.TILES_FUSED,
-                                   moe.TILES_PERSISTENT])
+@pytest.mark.parametrize("tiles", [moe.TILES_SMALL, moe.TILES_LARGE, moe.TILES_PAIR, moe.TILES_PERSISTENT])
 @pytest.mark.parametrize("name", list(CASES))
 def test_forward_matches_oracle(name, tiles, router):
     cfg, inp, ref = case(name)
     router_skip(cfg, router)
-    if tiles == moe.TILES_FUSED and (router != moe.ROUTER_SMALL or not fused_ok(cfg)):
-        pytest.skip("one-launch layer: T <= 4 and 256-multiple shapes (its router is the few-token one)")
     if tiles == moe.TILES_PERSISTENT and (router != moe.ROUTER_SMALL or not persistent_ok(cfg)):
         pytest.skip("persistent layer: T <= 16, E % 4 == 0, no shared expert (its router is the few-token one)")
     d = dev_inputs(inp)
@@ -289,36 +281,6 @@ def test_split_k_forward_bitwise_deterministic():
     assert info["launches"] == 5  # route+permute, gate/up, SwiGLU reduce, down, combine
 
 
-def test_fused_layer_one_launch_repeated_and_deterministic():
-    """The one-launch layer for a few tokens: one kernel, routing and
-    permutation bit-exact, y within tolerance and bitwise identical over
-    repeated calls, and its grid-barrier counter back at zero afterwards
-    (the status block is all zero)."""
-    import torch
-    for name in ("one_token", "decode_split", "fused_shared"):
-        cfg, inp, ref = case(name)
-        d = dev_inputs(inp)
-        ws = workspace(cfg)
-        info = {}
-        ys = []
-        for _ in range(3):
-            ys.append(moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, ws,
-                                  d["w_sh_gate_up"], d["w_sh_down"], tiles=moe.TILES_FUSED, info=info).cpu())
-        assert_ok(ws)
-        assert info["launches"] == 1
-        assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2])
-        v = moe.workspace_view(ws, cfg.T, cfg.H, cfg.E, cfg.I, cfg.k, cfg.I_s)
-        np.testing.assert_array_equal(v["topk_ids"].cpu().numpy(), ref["ids"])
-        np.testing.assert_array_equal(v["counts"].cpu().numpy(), ref["counts"])
-        np.testing.assert_array_equal(v["offsets"].cpu().numpy(), ref["offsets"])
-        np.testing.assert_array_equal(v["sorted_token_ids"].cpu().numpy(), ref["sorted_token_ids"])
-        np.testing.assert_array_equal(v["inv_perm"].cpu().numpy(), ref["inv_perm"])
-        assert np.abs(host_f64(v["topk_w"]) - ref["w"]).max() <= W_ABS
-        assert_close_output(host_f64(ys[0]), ref["y"])
-        torch.cuda.synchronize()
-        assert ws[:32].view(torch.int32).cpu().tolist() == [0] * 8
-
-
 @pytest.mark.parametrize("name", [n for n, c in CASES.items() if persistent_ok(c)])
 def test_persistent_layer_bitwise_equals_kernel_sequence(name):
     """The persistent layer runs the same tiles, K split, epilogue arithmetic
@@ -356,14 +318,6 @@ def test_persistent_layer_rejects_unsupported_shapes():
         with pytest.raises(moe.MoEError):
             moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, workspace(cfg),
                         d["w_sh_gate_up"], d["w_sh_down"], tiles=moe.TILES_PERSISTENT)
-
-
-def test_fused_policy_rejects_unsupported_shapes():
-    cfg, inp, ref = case("tiny")  # 64 tokens: beyond the one-launch layer
-    d = dev_inputs(inp)
-    with pytest.raises(moe.MoEError):
-        moe.forward(d["x"], d["w_router"], d["bias"], d["w_gate_up"], d["w_down"], cfg.k, workspace(cfg),
-                    tiles=moe.TILES_FUSED)
 
 
 def test_all_tokens_to_the_same_experts():

@@ -133,6 +133,6 @@ def test_mx_split_slab_sum_in_epilogue_equals_reduce_kernel_and_repeats():
 
 def test_mx_rejects_unsupported_options():
     cfg, inp, ref, mx, _, _ = case("mx_one_token")
-    for kw in (dict(tiles=moe.TILES_PERSISTENT), dict(tiles=moe.TILES_FUSED), dict(combine=moe.COMBINE_FUSED)):
+    for kw in (dict(tiles=moe.TILES_PERSISTENT), dict(combine=moe.COMBINE_FUSED)):
         with pytest.raises(moe.MoEError):
             run_mx(cfg, inp, mx, **{"tiles": moe.TILES_AUTO, **kw})

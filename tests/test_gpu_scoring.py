@@ -94,9 +94,8 @@ def test_route_scoring_matches_oracle(name, scoring, impl):
 
 def _tile_policies(cfg):
     out = [moe.TILES_AUTO, moe.TILES_SMALL]
-    if cfg.T <= 4 and cfg.k <= 16 and cfg.E % 4 == 0 and cfg.H % 256 == 0 and cfg.I % 256 == 0 \
-            and cfg.I_s % 256 == 0:
-        out.append(moe.TILES_FUSED)
+    if cfg.T <= 16 and cfg.E % 4 == 0 and cfg.I_s == 0:  # the persistent one-launch layer
+        out.append(moe.TILES_PERSISTENT)
     return out
 
 
