@@ -20,7 +20,7 @@ struct DevStatus {
   int32_t site;
   int32_t aux;
   uint32_t arrivals;  // block counter of the few-token router: zero between its launches
-  uint32_t grid_bar;  // grid-barrier counter of the one-launch few-token layer: zero between launches
+  uint32_t reserved0;  // unused, zero
   uint32_t exits;     // persistent few-token layer: blocks done; zero between launches
   uint32_t reserved[2];
 };
