@@ -136,3 +136,65 @@ def test_mx_rejects_unsupported_options():
     for kw in (dict(tiles=moe.TILES_PERSISTENT), dict(combine=moe.COMBINE_FUSED)):
         with pytest.raises(moe.MoEError):
             run_mx(cfg, inp, mx, **{"tiles": moe.TILES_AUTO, **kw})
+
+
+@pytest.mark.slow
+def test_mx_full_size_decode():
+    """The 512-expert decode shape (T = 512, H = 4096, I = 1024, top-10) on
+    block-scaled FP8 weights, in the launch configuration bench.py times
+    (automatic tiles): routing bit-exact on every token, h on every permuted
+    row of a sample of tokens and y on those tokens against the oracle on the
+    dequantised weights, one expert at a time."""
+    import torch
+    from test_gpu_fullsize import sample_tokens, torch_index
+    cfg = synth.CONFIGS["qwen_decode_t512"]
+    inp = synth.make_inputs(cfg, experts=False)
+    oracle.enforce_logit_gap(inp)
+    E, H, I = cfg.E, cfg.H, cfg.I
+    gu_c = torch.empty(E, 2 * I, H, dtype=torch.uint8, device="cuda")   # codes of W^T
+    gu_s = torch.empty(E, H // 32, 2 * I, dtype=torch.uint8, device="cuda")
+    dn_c = torch.empty(E, H, I, dtype=torch.uint8, device="cuda")
+    dn_s = torch.empty(E, I // 32, H, dtype=torch.uint8, device="cuda")
+    from concurrent.futures import ThreadPoolExecutor
+
+    def draw(e):
+        cg, sg = synth.mx_expert_weights(cfg, e, "gate_up")
+        cd, sd = synth.mx_expert_weights(cfg, e, "down")
+        return np.ascontiguousarray(cg.T), sg, np.ascontiguousarray(cd.T), sd
+
+    with ThreadPoolExecutor(16) as ex:
+        for e0 in range(0, E, 32):
+            for e, (cg, sg, cd, sd) in zip(range(e0, e0 + 32), ex.map(draw, range(e0, min(E, e0 + 32)))):
+                gu_c[e].copy_(torch.from_numpy(cg))
+                gu_s[e].copy_(torch.from_numpy(sg))
+                dn_c[e].copy_(torch.from_numpy(cd))
+                dn_s[e].copy_(torch.from_numpy(sd))
+    ws = moe.alloc_workspace(cfg.T, H, E, I, cfg.k)
+    y = moe.forward_mx(dev_bf16(inp.x), dev_f32(inp.w_router), None, gu_c, gu_s, dn_c, dn_s, cfg.k, ws)
+    st = moe.device_status(ws)
+    assert st == 0, moe.STATUS.get(st, st)
+
+    ids, w = oracle.topk_route(oracle.router_logits(inp.x, inp.w_router, inp.bias), cfg.k)
+    counts, offsets, sids, inv = oracle.permute(ids, E)
+    v = moe.workspace_view(ws, cfg.T, H, E, I, cfg.k)
+    np.testing.assert_array_equal(v["topk_ids"].cpu().numpy(), ids)
+    assert np.abs(host_f64(v["topk_w"]) - w).max() <= W_ABS
+    np.testing.assert_array_equal(v["offsets"].cpu().numpy(), offsets)
+    np.testing.assert_array_equal(v["sorted_token_ids"].cpu().numpy(), sids)
+    np.testing.assert_array_equal(v["inv_perm"].cpu().numpy(), inv)
+
+    def gate_up(e):
+        return oracle.mx.mx_dequant(*synth.mx_expert_weights(cfg, int(e), "gate_up"))
+
+    def down(e):
+        return oracle.mx.mx_dequant(*synth.mx_expert_weights(cfg, int(e), "down"))
+
+    toks = sample_tokens(cfg, counts, ids, n_random=4)
+    for e in np.unique(ids[toks]):
+        tt, jj = np.nonzero(ids[toks] == e)
+        rows = inv[toks[tt], jj]
+        want_h = oracle.swiglu_ffn_rows(oracle.bf16_to_f64(inp.x[toks[tt]]), gate_up(e))
+        got_h = host_f64(v["h"][torch_index(rows.astype(np.int64))])
+        assert_close_output(got_h, want_h, what=f"h of expert {int(e)}")
+    want = oracle.layer_forward_tokens(inp.x, toks, ids, w, gate_up, down)
+    assert_close_output(host_f64(y[torch_index(toks)]), want)
