@@ -189,7 +189,7 @@ __global__ void __launch_bounds__(kSmallThreads) router_small_kernel(
   __shared__ int32_t cnt[kMaxExperts];
   __shared__ int32_t warp_sums[kSmallThreads / 32];
   __shared__ int is_last;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x;
   router_partial<TT>(x, w, T, H, E, chunk, blockIdx.x, blockIdx.y, partial, rsm);
   __threadfence();
   __syncthreads();
