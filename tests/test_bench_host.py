@@ -35,6 +35,32 @@ def test_layer_accounting_counts_only_touched_experts_and_the_shared_one():
     assert acc["layer_bytes"] == 100 * 3 * H * I * 2 + 3 * H * Is * 2 + T * H * 2 + H * 256 * 4 + T * H * 2
 
 
+def test_kernel_roofline_picks_the_binding_unit():
+    """The gate/up kernel's roofline object: HBM-bound when its bytes take
+    longer at the copy peak than its FLOPs at the sustained bf16 peak (the
+    bf16 prefill shape), tensor-bound otherwise (the same shape on FP8
+    weights: half the weight bytes, the same MMAs)."""
+    pk = {"hbm_gbs": 6539.5, "bf16_tflops": 1606.0, "bf16_tflops_sustained": 1367.0}
+    cfg = synth.CONFIGS["qwen_prefill_t8192"]         # T=8192, H=4096, E=512, I=1024, k=10
+    counts = np.full(cfg.E, 160)
+    flops = 4.0 * 8192 * 10 * 4096 * 1024
+    bf = bench.layer_accounting(cfg, counts)
+    assert bf["gate_up_flops"] == flops
+    r = bench.kernel_roofline(bf, 1.5, pk, "measured", None)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["peak"] == 6539.5
+    assert abs(r["achieved"] - bf["gate_up_bytes"] / 1.5e-3 / 1e9) < 0.1
+    mx = bench.layer_accounting(cfg, counts, mx=True)
+    assert mx["gate_up_bytes"] == 512 * 4096 * 2048 * (1 + 1 / 32) + 8192 * 4096 * 2 + 81920 * 1024 * 2
+    r = bench.kernel_roofline(mx, 2.0, pk, "measured", None)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and r["peak"] == 1367.0
+    assert abs(r["achieved"] - flops / 2.0e-3 / 1e12) < 0.1
+    assert abs(r["frac"] - r["achieved"] / 1367.0) < 1e-3
+    # decode: far below the ridge on either weight format
+    dc = synth.CONFIGS["qwen_decode_t512"]
+    assert bench.kernel_roofline(bench.layer_accounting(dc, np.full(dc.E, 10), mx=True), 1.1, pk, "m",
+                                 None)["bound"] == "hbm"
+
+
 def test_clock_summary_median_and_reasons():
     clk = bench.ClockSampler(0)
 
