@@ -331,12 +331,13 @@ moe_status_t moe_forward_ex(const uint16_t *x, const float *w_router, const floa
  * shared expert stay bf16.  Passage: Qwen 3.5-397B MoE on Ironwood (TPU
  * v7x), sec. 6 "numerical validation" (accumulation across FP8 scaling
  * blocks); the Ironwood systems handbook page runs Microscaling formats.
- * Every such weight with scale code 3 or above is an exact bf16 value (4
+ * Every such weight with a scale code in 3..246 is an exact bf16 value (4
  * significant bits times a power of two, within bf16's range), so the layer
  * computes exactly what moe_forward_ex computes on the dequantised weights,
  * with the same rounding points; only the expert-weight bytes halve (plus
  * 1/32 for the scales).  Below scale code 3 a weight smaller than bf16's
- * least subnormal step is rounded to nearest bf16.  Everything else as moe_forward_ex, except: the tile policy
+ * least subnormal step is rounded to nearest bf16; above 246 a weight beyond
+ * bf16's finite range decodes to +-inf.  Everything else as moe_forward_ex, except: the tile policy
  * PERSISTENT and MOE_COMBINE_FUSED are not available
  * (MOE_ERR_INVALID_ARG), and PAIR runs as LARGE (single-SM 256-row passes).
  * The two E4M3 NaN patterns are not supported as weights (they decode as

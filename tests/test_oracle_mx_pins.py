@@ -97,6 +97,28 @@ def test_dequantised_weights_are_exact_bf16_values():
         np.testing.assert_array_equal(back, w)
 
 
+def test_exact_bf16_range_of_the_scale_codes():
+    """Every finite E4M3 value times 2^(c - 127) is a bf16 number exactly for
+    scale codes 3..246, and for no wider range: below 3 the smallest values
+    (2^-9 * 2^(c-127)) fall under bf16's least subnormal step 2^-133; above
+    246 the largest (448 * 2^(c-127)) pass bf16's largest finite value
+    (1.9921875 * 2^127).  Checked over all 254 finite codes and all 255
+    finite scale codes by widening back from bf16."""
+    codes = np.arange(256, dtype=np.uint8)
+    vals = mx.e4m3_to_f64(codes)
+    vals = vals[~np.isnan(vals)]
+    assert len(vals) == 254
+    exact = []
+    for c in range(255):
+        w = vals * 2.0 ** (c - 127)
+        back = torch.from_numpy(w).float().to(torch.bfloat16).double().numpy()
+        exact.append(bool(np.array_equal(back, w)))
+    assert [c for c in range(255) if exact[c]] == list(range(3, 247))
+    # the two limits, worked by hand
+    assert 2.0 ** -9 * 2.0 ** (2 - 127) == 2.0 ** -134 < 2.0 ** -133
+    assert 448 * 2.0 ** (247 - 127) == 1.75 * 2.0 ** 128 > 1.9921875 * 2.0 ** 127
+
+
 def test_mx_layer_is_bf16_layer_on_the_same_values():
     """The layer on dequantised fp8 weights equals the oracle's bf16-weight
     layer fed the same values as bf16 bit patterns (exact, no tolerance)."""
