@@ -111,6 +111,25 @@ def test_forward_options_scoring_is_checked(lib):
                                   ctypes.byref(opt), None) == 1
 
 
+def test_forward_options_tiles_and_combine_are_checked(lib):
+    """Tile policies run 0..4 (4 = the persistent one-launch layer) and
+    combine placements 0..2; anything else is refused on the host, and so
+    are the options the FP8-weight layer does not take (the persistent
+    layer, the combine in the down epilogue)."""
+    ws = moe.workspace_size(64, 256, 8, 128, 2)
+    assert (moe.TILES_AUTO, moe.TILES_SMALL, moe.TILES_LARGE, moe.TILES_PAIR, moe.TILES_PERSISTENT) == (0, 1, 2, 3, 4)
+    for tiles, combine in ((-1, 0), (5, 0), (0, -1), (0, 3)):
+        opt = moe._Options(tiles, 0)
+        opt.combine = combine
+        assert lib.moe_forward_ex(p(), p(), None, p(), p(), None, None, 0, 64, 256, 8, 128, 2, p(), p(), ws,
+                                  ctypes.byref(opt), None) == 1, (tiles, combine)
+    for tiles, combine in ((moe.TILES_PERSISTENT, 0), (0, moe.COMBINE_FUSED)):
+        opt = moe._Options(tiles, 0)
+        opt.combine = combine
+        assert lib.moe_forward_mx(p(), p(), None, p(), p(), p(), p(), None, None, 0, 64, 256, 8, 128, 2, p(), p(),
+                                  ws, ctypes.byref(opt), None) == 1, (tiles, combine)
+
+
 def test_forward_argument_errors_before_any_launch(lib):
     f = lib.moe_forward
     ws = moe.workspace_size(64, 256, 8, 128, 2)
